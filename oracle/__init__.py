@@ -1,0 +1,196 @@
+"""fp64 CPU oracle for exact attention -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline / reference arm may
+import this package. It shares no code with the CUDA library (``exact_attention_138_b200``) and
+neither imports the other.
+
+The arithmetic lives in ``attn_oracle.c`` (plain loops, fp64, OpenMP over independent rows);
+this module builds it with gcc when needed and marshals numpy arrays through ctypes. Inputs are
+passed as float32 arrays: fp32 inputs and bf16-rounded inputs are both represented exactly in
+float32 and are widened to float64 inside the C code.
+
+Sources of each function are cited in ``attn_oracle.c``:
+  * "Attention Mechanism: Revolusi Representasi Sequence", §3 Steps 1-4 and §4.4 (definition,
+    causal mask), §13 "FlashAttention — How It Works" (online softmax recurrence);
+  * "Efficient Attention", efficient_attention.py part 3 (row tiling in 128-row blocks);
+  * "Flash Attention Nedir?", "Online Softmax" (log-sum-exp statistic);
+  * "Apa itu FlashAttention", "Cara kerja teknik Tiling dan Recomputation" (backward recomputes
+    the softmax; the gradient formulas are the exact derivative of the definition);
+  * "Calculateur de mémoire d'attention", "La formule" (score-matrix bytes B·H·n²·e).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile attn_oracle.c into liboracle.so (plain -O2, portable x86-64/aarch64 code)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", _SRC, "-o", tmp, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        try:
+            lib = ctypes.CDLL(build())
+        except OSError:
+            lib = ctypes.CDLL(build(force=True))
+        f32p = np.ctypeslib.ndpointer(np.float32, flags="C_CONTIGUOUS")
+        f64p = np.ctypeslib.ndpointer(np.float64, flags="C_CONTIGUOUS")
+        i64p = np.ctypeslib.ndpointer(np.int64, flags="C_CONTIGUOUS")
+        i32p = np.ctypeslib.ndpointer(np.int32, flags="C_CONTIGUOUS")
+        I, D = ctypes.c_int, ctypes.c_double
+        lib.oracle_fwd.argtypes = [f32p, f32p, f32p, I, I, I, I, D, I, f64p, f64p]
+        lib.oracle_fwd_rowtiled.argtypes = [f32p, f32p, f32p, I, I, I, I, D, I, I, f64p, f64p]
+        lib.oracle_fwd_online.argtypes = [f32p, f32p, f32p, I, I, I, I, D, I, I, I, f64p, f64p]
+        lib.oracle_fwd_rows.argtypes = [f32p, f32p, f32p, I, I, I, I, D, I, i64p, I, f64p, f64p]
+        lib.oracle_bwd.argtypes = [f32p, f32p, f32p, f32p, I, I, I, I, D, I, f64p, f64p, f64p,
+                                   f64p]
+        lib.oracle_bwd_query_rows.argtypes = [f32p, f32p, f32p, f32p, I, I, I, I, D, I, i64p, I,
+                                              f64p, f64p]
+        lib.oracle_bwd_key_rows.argtypes = [f32p, f32p, f32p, f32p, I, I, I, I, D, I,
+                                            ctypes.c_long, i32p, I, f64p, f64p]
+        lib.oracle_score_matrix_bytes.argtypes = [D, D, D, D]
+        lib.oracle_score_matrix_bytes.restype = D
+        lib.oracle_num_threads.restype = I
+        lib.oracle_set_num_threads.argtypes = [I]
+        for name in ("oracle_fwd", "oracle_fwd_rowtiled", "oracle_fwd_online", "oracle_fwd_rows",
+                     "oracle_bwd", "oracle_bwd_query_rows", "oracle_bwd_key_rows"):
+            getattr(lib, name).restype = I
+        _lib = lib
+        return lib
+
+
+def _f32(x) -> np.ndarray:
+    """Accept numpy arrays or CPU torch tensors (fp32 or bf16); return contiguous float32."""
+    if hasattr(x, "detach"):  # torch tensor: widen exactly to fp32 on the CPU
+        x = x.detach().to("cpu").float().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+
+
+def _shape4(q):
+    if q.ndim == 2:
+        return 1, 1, q.shape[0], q.shape[1]
+    if q.ndim != 4:
+        raise ValueError("expected (B,H,n,d) or (n,d)")
+    return q.shape
+
+
+def _check(rc, name):
+    if rc != 0:
+        raise RuntimeError(f"{name} failed with code {rc}")
+
+
+def num_threads() -> int:
+    return _load().oracle_num_threads()
+
+
+def set_num_threads(t: int) -> None:
+    _load().oracle_set_num_threads(int(t))
+
+
+def score_matrix_bytes(B, H, n, e) -> int:
+    """Bytes of the materialised score matrix, B·H·n²·e."""
+    return int(round(_load().oracle_score_matrix_bytes(B, H, n, e)))
+
+
+def fwd(q, k, v, scale, causal=False):
+    """Definition with the full score matrix of each (b,h). Returns (O fp64, LSE fp64)."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    B, H, n, d = _shape4(q)
+    o = np.empty(q.shape, np.float64)
+    lse = np.empty(q.shape[:-1], np.float64)
+    _check(_load().oracle_fwd(q, k, v, B, H, n, d, float(scale), int(bool(causal)), o, lse),
+           "oracle_fwd")
+    return o, lse
+
+
+def fwd_rowtiled(q, k, v, scale, causal=False, block_rows=128):
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    B, H, n, d = _shape4(q)
+    o = np.empty(q.shape, np.float64)
+    lse = np.empty(q.shape[:-1], np.float64)
+    _check(_load().oracle_fwd_rowtiled(q, k, v, B, H, n, d, float(scale), int(bool(causal)),
+                                       int(block_rows), o, lse), "oracle_fwd_rowtiled")
+    return o, lse
+
+
+def fwd_online(q, k, v, scale, causal=False, block_cols=128, literal_page_form=False):
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    B, H, n, d = _shape4(q)
+    o = np.empty(q.shape, np.float64)
+    lse = np.empty(q.shape[:-1], np.float64)
+    _check(_load().oracle_fwd_online(q, k, v, B, H, n, d, float(scale), int(bool(causal)),
+                                     int(block_cols), int(bool(literal_page_form)), o, lse),
+           "oracle_fwd_online")
+    return o, lse
+
+
+def fwd_rows(q, k, v, scale, causal, rows):
+    """O and LSE for flat row indices rows[t] = (b*H + h)*n + i."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    B, H, n, d = _shape4(q)
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    o = np.empty((len(rows), d), np.float64)
+    lse = np.empty(len(rows), np.float64)
+    _check(_load().oracle_fwd_rows(q, k, v, B, H, n, d, float(scale), int(bool(causal)), rows,
+                                   len(rows), o, lse), "oracle_fwd_rows")
+    return o, lse
+
+
+def bwd(q, k, v, do, scale, causal=False):
+    """Exact derivative. Returns (dQ, dK, dV, D) in fp64."""
+    q, k, v, do = _f32(q), _f32(k), _f32(v), _f32(do)
+    B, H, n, d = _shape4(q)
+    dq = np.empty(q.shape, np.float64)
+    dk = np.empty(q.shape, np.float64)
+    dv = np.empty(q.shape, np.float64)
+    D = np.empty(q.shape[:-1], np.float64)
+    _check(_load().oracle_bwd(q, k, v, do, B, H, n, d, float(scale), int(bool(causal)), dq, dk,
+                              dv, D), "oracle_bwd")
+    return dq, dk, dv, D
+
+
+def bwd_query_rows(q, k, v, do, scale, causal, rows):
+    """dQ (and D) for flat query rows rows[t] = bh*n + i."""
+    q, k, v, do = _f32(q), _f32(k), _f32(v), _f32(do)
+    B, H, n, d = _shape4(q)
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    dq = np.empty((len(rows), d), np.float64)
+    D = np.empty(len(rows), np.float64)
+    _check(_load().oracle_bwd_query_rows(q, k, v, do, B, H, n, d, float(scale),
+                                         int(bool(causal)), rows, len(rows), dq, D),
+           "oracle_bwd_query_rows")
+    return dq, D
+
+
+def bwd_key_rows(q, k, v, do, scale, causal, bh, keys):
+    """dK and dV for key rows `keys` (indices within one head) of head bh = b*H + h."""
+    q, k, v, do = _f32(q), _f32(k), _f32(v), _f32(do)
+    B, H, n, d = _shape4(q)
+    keys = np.ascontiguousarray(np.asarray(keys, dtype=np.int32))
+    dk = np.empty((len(keys), d), np.float64)
+    dv = np.empty((len(keys), d), np.float64)
+    _check(_load().oracle_bwd_key_rows(q, k, v, do, B, H, n, d, float(scale), int(bool(causal)),
+                                       int(bh), keys, len(keys), dk, dv), "oracle_bwd_key_rows")
+    return dk, dv
