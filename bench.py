@@ -1,0 +1,377 @@
+#!/usr/bin/env python3
+"""Benchmark: exact attention forward + backward TFLOPS on B200 (bf16, causal).
+
+One step = one forward (attn_fwd) and one backward (attn_bwd) pass over one batch of the
+workload B=2, H=32, n=8192, d=128, causal, bf16, inputs iid N(0,1) x 0.5 drawn from a seeded
+CPU generator. FLOPs per step follow the convention forward = 4·B·H·n²·d (two matmuls), halved
+for the causal mask, backward = 2.5 x forward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints ONE JSON line on rank 0. With N > 1 (launched by torchrun, one process per GPU) every
+rank runs its own batch: the units are independent (b,h) problems, so the shards need no
+collective; time is the max over ranks (weak scaling). `--impl reference` times the fp64 CPU
+oracle on a bounded sample of the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd/bwd TFLOPS at 1 B200 (bf16, causal) and % of dense bf16 peak"
+WORKLOAD = "causal_bf16_2x32x8192x128"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def step_flops(B, H, n, d, causal=True):
+    fwd = 4.0 * B * H * n * n * d * (0.5 if causal else 1.0)
+    return fwd, 2.5 * fwd
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def csrc_digest():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "exact_attention_138_b200", "csrc")
+    for name in sorted(os.listdir(d)):
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if the kernel sources
+    have not changed since the counters were taken; else None."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    entry = rec.get(kernel)
+    if not entry or entry.get("csrc_sha") != csrc_digest():
+        return None
+    return entry.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [x.strip() for x in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+            os.unlink(self.path)
+        except OSError:
+            pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        smax = [num(r[2]) for r in rows if num(r[2]) is not None]
+        power = [num(r[3]) for r in rows if num(r[3]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        loaded = [x for x in sm if smax and x >= 0.3 * max(smax)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def oracle_sample(seconds_target, q, k, v, do, w, rng_seed=9):
+    """Time the fp64 oracle on a bounded sample of the workload's query rows: forward rows
+    (O, LSE) and backward dQ rows. Returns (TFLOPS credited, seconds, rows, threads)."""
+    import numpy as np
+    import oracle
+    B, H, n, d = w.B, w.H, w.n, w.d
+    total_rows = B * H * n
+    fwd, bwd = step_flops(B, H, n, d)
+    per_row = (fwd + bwd) / total_rows            # average algorithmic FLOPs of one query row
+    rng = np.random.default_rng(rng_seed)
+    probe = np.sort(rng.choice(total_rows, size=8, replace=False))
+    t0 = time.perf_counter()
+    oracle.fwd_rows(q, k, v, w.scale, True, probe)
+    oracle.bwd_query_rows(q, k, v, do, w.scale, True, probe)
+    t_probe = max(time.perf_counter() - t0, 1e-3)
+    rows_n = int(max(8, min(4096, seconds_target / t_probe * len(probe))))
+    rows = np.sort(rng.choice(total_rows, size=rows_n, replace=False))
+    t0 = time.perf_counter()
+    oracle.fwd_rows(q, k, v, w.scale, True, rows)
+    oracle.bwd_query_rows(q, k, v, do, w.scale, True, rows)
+    dt = time.perf_counter() - t0
+    return per_row * rows_n / dt / 1e12, dt, rows_n, oracle.num_threads()
+
+
+def run_reference(args, w):
+    """Reference arm: the fp64 CPU oracle (as it stands) on the machine's host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import attn_inputs
+    q, k, v, do = attn_inputs.workload_inputs(w)
+    times, flops_rate, rows_used, threads = [], [], 0, 1
+    for i in range(args.warmup + args.steps):
+        rate, dt, rows_n, threads = oracle_sample(args.ref_seconds, q, k, v, do, w, 9 + i)
+        if i >= args.warmup:
+            times.append(dt)
+            flops_rate.append(rate)
+            rows_used = rows_n
+    value = statistics.mean(flops_rate)
+    sample = (f"{rows_used} uniformly drawn query rows of {w.B}x{w.H}x{w.n}x{w.d} per step "
+              f"(forward O/LSE rows + backward dQ rows, fp64); TFLOPS credited at the "
+              f"workload's average FLOPs per query row")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000 * statistics.mean(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": w.B, "H": w.H, "n": w.n, "d": w.d,
+                   "causal": True, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    import attn_inputs
+    w = attn_inputs.WORKLOADS[WORKLOAD]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    import exact_attention_138_b200 as ea
+
+    # --- inputs: each rank draws its own batch (seed 9 + rank), rounded to bf16 on the host
+    q_h, k_h, v_h, do_h = attn_inputs.bf16_draws(w.shape, factor=w.factor,
+                                                 seed=attn_inputs.SEED + rank)
+    q, k, v, do = (t.to(dev) for t in (q_h, k_h, v_h, do_h))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.n), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(ea.attn_bwd_workspace_bytes(w.B, w.H, w.n, w.d, 0), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ea.forward(q, k, v, causal=True, scale=w.scale, out=o, lse=lse, stream=stream)
+        ea.backward(q, k, v, o, do, lse, causal=True, scale=w.scale, dq=dq, dk=dk, dv=dv,
+                    workspace=ws, stream=stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if ea.device_status() != ea.ATTN_OK:
+        raise SystemExit("device status not OK after warm-up")
+
+    # --- timed region: K steps; per-kernel events for the roofline
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for s in range(args.steps):
+            e = ev[s]
+            e[0].record(stream)
+            ea.forward(q, k, v, causal=True, scale=w.scale, out=o, lse=lse, stream=stream)
+            ea.attn_set_bwd_phase_events(e[1:5])
+            ea.backward(q, k, v, o, do, lse, causal=True, scale=w.scale, dq=dq, dk=dk, dv=dv,
+                        workspace=ws, stream=stream)
+            ea.attn_set_bwd_phase_events(None)
+            e[5].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    if ea.device_status() != ea.ATTN_OK:
+        raise SystemExit("device status not OK after the timed region")
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    pre_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    main_ms = [e[2].elapsed_time(e[3]) for e in ev]
+    conv_ms = [e[3].elapsed_time(e[4]) for e in ev]
+    bwd_ms = [e[1].elapsed_time(e[4]) for e in ev]
+    if dist is not None:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = t.item()
+
+    fwd_flops, bwd_flops = step_flops(w.B, w.H, w.n, w.d)
+    ms_per_step = total_ms / args.steps
+    value = world * (fwd_flops + bwd_flops) / (ms_per_step * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    fwd_tf = fwd_flops / (statistics.mean(fwd_ms) * 1e-3) / 1e12
+    bwd_tf = bwd_flops / (statistics.mean(bwd_ms) * 1e-3) / 1e12
+    main_tf = bwd_flops / (statistics.mean(main_ms) * 1e-3) / 1e12
+
+    # --- end to end through the public API with host buffers (pinned), copies inside the timing
+    pin = [t.pin_memory() for t in (q_h, k_h, v_h, do_h)]
+    outs_h = [torch.empty(w.shape, dtype=torch.bfloat16).pin_memory() for _ in range(4)]
+    lse_h = torch.empty((w.B, w.H, w.n), dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in pin)
+    d2h = sum(t.numel() * t.element_size() for t in outs_h) + lse_h.numel() * 4
+
+    def e2e_step():
+        for dst, src in zip((q, k, v, do), pin):
+            dst.copy_(src, non_blocking=True)
+        step()
+        for dst, src in zip(outs_h, (o, dq, dk, dv)):
+            dst.copy_(src, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(b) / args.e2e_steps
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = t.item()
+    e2e_value = world * (fwd_flops + bwd_flops) / (e2e_ms * 1e-3) / 1e12
+
+    clk = clocks.summary()
+    traffic = recorded_traffic("bwd_main_kernel")
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": w.B, "H": w.H, "n": w.n, "d": w.d, "causal": True,
+                   "input_factor": w.factor, "global_batch": w.B * world,
+                   "parallelism": f"dp{world}" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (q,k,v,dO 128 MiB each); no flush"},
+        "fwd": {"ms": statistics.mean(fwd_ms), "tflops": fwd_tf,
+                "pct_of_burst_peak": 100 * fwd_tf / burst},
+        "bwd": {"ms": statistics.mean(bwd_ms), "tflops": bwd_tf,
+                "pct_of_burst_peak": 100 * bwd_tf / burst,
+                "preprocess_ms": statistics.mean(pre_ms), "main_ms": statistics.mean(main_ms),
+                "dq_convert_ms": statistics.mean(conv_ms)},
+        "pct_of_burst_peak": 100 * (value / world) / burst,
+        "roofline": {"kernel": "bwd_main_kernel", "bound": "tensor", "achieved": main_tf,
+                     "peak": sustained, "unit": "TFLOP/s", "frac": main_tf / sustained,
+                     "peak_kind": f"bf16_tflops_sustained ({peak_src})",
+                     "traffic": traffic},
+        "e2e": {"value": e2e_value, "unit": "TFLOPS", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, dt, rows_n, threads = oracle_sample(args.cpu_seconds, q_h, k_h, v_h, do_h, w)
+        line["cpu_baseline"] = {
+            "value": rate, "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+            "sample": f"{rows_n} query rows (forward O/LSE + backward dQ, fp64) in {dt:.1f} s; "
+                      f"credited at the workload's average FLOPs per query row"}
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

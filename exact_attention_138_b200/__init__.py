@@ -1,0 +1,197 @@
+"""exact_attention_138_b200 — exact scaled dot-product attention on one B200 (sm_100a).
+
+Python binding of the C ABI in ``include/attn.h`` (``libattn.so``, built in-tree by
+``python -m exact_attention_138_b200.build``). This module only marshals arguments: device
+memory and streams come from PyTorch, every step of the computation runs in the library's
+CUDA kernels. There is no CPU fallback: if the library is missing the import fails.
+
+    O = softmax(scale · Q·K^T + M) · V      ("Attention Mechanism: Revolusi Representasi
+    Sequence", §3 Steps 1-4; causal mask M of §4.4)
+
+Raw entry points keep the C names (``attn_fwd``, ``attn_bwd``, ``attn_bwd_workspace_bytes``,
+``attn_get_device_status``, ``attn_set_wait_timeout_us``, ``attn_selftest_wait_timeout``,
+``attn_error_string``, ``attn_version``); ``forward`` / ``backward`` wrap them for torch tensors.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libattn.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "attn.h")
+
+ATTN_BF16, ATTN_FP32 = 0, 1
+ATTN_OK, ATTN_ERR_INVALID, ATTN_ERR_UNSUPPORTED = 0, 1, 2
+ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT, ATTN_ERR_WORKSPACE = 3, 4, 5
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m exact_attention_138_b200.build` "
+        "(there is no fallback implementation)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+_lib.attn_version.restype = _i
+_lib.attn_version.argtypes = []
+_lib.attn_error_string.restype = ctypes.c_char_p
+_lib.attn_error_string.argtypes = [_i]
+_lib.attn_fwd.restype = _i
+_lib.attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _i, _vp]
+_lib.attn_bwd_workspace_bytes.restype = _sz
+_lib.attn_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
+_lib.attn_bwd.restype = _i
+_lib.attn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i,
+                          _i, _i, _vp, _sz, _vp]
+_lib.attn_get_device_status.restype = _i
+_lib.attn_get_device_status.argtypes = [_vp]
+_lib.attn_set_wait_timeout_us.restype = ctypes.c_uint
+_lib.attn_set_wait_timeout_us.argtypes = [ctypes.c_uint]
+_lib.attn_selftest_wait_timeout.restype = _i
+_lib.attn_selftest_wait_timeout.argtypes = [ctypes.c_uint, _vp]
+_lib.attn_set_bwd_phase_events.restype = None
+_lib.attn_set_bwd_phase_events.argtypes = [_vp]
+
+
+class AttnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {attn_error_string(code)} (code {code})")
+
+
+def library():
+    """The loaded ctypes library (for tests that check exported symbols)."""
+    return _lib
+
+
+def declared_functions():
+    """Names of the functions declared in include/attn.h."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z0-9_]+)\s*\(", text)))
+
+
+# ---------------------------------------------------------------- raw C entry points
+def attn_version() -> int:
+    return _lib.attn_version()
+
+
+def attn_error_string(code: int) -> str:
+    return _lib.attn_error_string(int(code)).decode()
+
+
+def attn_fwd(q, k, v, o, lse, B, H, n, d, scale, causal, dtype, stream) -> int:
+    return _lib.attn_fwd(q, k, v, o, lse, B, H, n, d, scale, causal, dtype, stream)
+
+
+def attn_bwd_workspace_bytes(B, H, n, d, deterministic) -> int:
+    return _lib.attn_bwd_workspace_bytes(B, H, n, d, deterministic)
+
+
+def attn_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, H, n, d, scale, causal, dtype, deterministic,
+             workspace, ws_bytes, stream) -> int:
+    return _lib.attn_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, H, n, d, scale, causal, dtype,
+                         deterministic, workspace, ws_bytes, stream)
+
+
+def attn_get_device_status(stream=None) -> int:
+    return _lib.attn_get_device_status(stream)
+
+
+def attn_set_wait_timeout_us(us: int) -> int:
+    return _lib.attn_set_wait_timeout_us(int(us))
+
+
+def attn_selftest_wait_timeout(timeout_us: int, stream=None) -> int:
+    return _lib.attn_selftest_wait_timeout(int(timeout_us), stream)
+
+
+def attn_set_bwd_phase_events(events) -> None:
+    """events: None, or 4 torch.cuda.Event objects (created with enable_timing=True)."""
+    if events is None:
+        _lib.attn_set_bwd_phase_events(None)
+        return
+    arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    _lib.attn_set_bwd_phase_events(ctypes.cast(arr, ctypes.c_void_p))
+
+
+# ---------------------------------------------------------------- torch-tensor wrappers
+def _dims(q):
+    if q.dim() == 2:
+        return 1, 1, q.shape[0], q.shape[1]
+    if q.dim() != 4:
+        raise ValueError("expected (B, H, n, d) or (n, d) tensors")
+    return tuple(q.shape)
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return ATTN_BF16
+    if t.dtype == torch.float32:
+        return ATTN_FP32
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(rc, where):
+    if rc != ATTN_OK:
+        raise AttnError(rc, where)
+
+
+def forward(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None):
+    """O, LSE = attention(q, k, v). q, k, v: contiguous CUDA tensors (B,H,n,d) or (n,d), bf16 or
+    fp32. Returns O (same dtype/shape as q) and LSE (fp32, (B,H,n))."""
+    import torch
+    B, H, n, d = _dims(q)
+    for t in (k, v):
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError("q, k, v must have the same shape and dtype")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, n), dtype=torch.float32, device=q.device)
+    rc = attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, n, d, float(scale),
+                  int(bool(causal)), _dtype_code(q), _stream_handle(stream))
+    _check(rc, "attn_fwd")
+    return out, lse
+
+
+def backward(q, k, v, o, do, lse, causal=False, scale=None, deterministic=False, dq=None,
+             dk=None, dv=None, workspace=None, stream=None):
+    """dQ, dK, dV of attention given dO (bf16 tensors, lse from `forward`)."""
+    import torch
+    B, H, n, d = _dims(q)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = attn_bwd_workspace_bytes(B, H, n, d, int(bool(deterministic)))
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    rc = attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk),
+                  _ptr(dv), B, H, n, d, float(scale), int(bool(causal)), _dtype_code(q),
+                  int(bool(deterministic)), _ptr(workspace),
+                  workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    _check(rc, "attn_bwd")
+    return dq, dk, dv
+
+
+def device_status(stream=None) -> int:
+    """Synchronise and return/clear the device status word (ATTN_OK or ATTN_ERR_TIMEOUT)."""
+    return attn_get_device_status(_stream_handle(stream))

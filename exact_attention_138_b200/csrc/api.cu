@@ -1,0 +1,211 @@
+// C-ABI entry points of libattn.so (declared in include/attn.h): argument validation, tensor-map
+// encoding, workspace carving and kernel launches on the caller's stream.
+#include <cudaTypedefs.h>
+#include <math.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace attn {
+
+namespace {
+
+std::atomic<unsigned> g_timeout_us{2000000u};
+cudaEvent_t g_phase_events[4];
+std::atomic<bool> g_phase_on{false};
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int to_code(cudaError_t e) { return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA; }
+
+__global__ void wait_selftest_kernel(uint64_t timeout_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    // Nobody arrives on `bar`: the wait runs out, records ATTN_ERR_TIMEOUT and returns.
+    if (threadIdx.x == 0) bounded_wait(&bar, 0, &abort_flag, timeout_ns);
+    __syncthreads();
+}
+
+constexpr size_t kAlign = 256;
+size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct WsLayout {
+    size_t d_off, acc_off, sem_off, total;
+};
+
+WsLayout ws_layout(int B, int H, int n, int d, int deterministic) {
+    const size_t BH = static_cast<size_t>(B) * H;
+    const size_t n_pad = (static_cast<size_t>(n) + 127) / 128 * 128;
+    WsLayout w;
+    w.d_off = 0;
+    w.acc_off = round_up(BH * n_pad * sizeof(float));
+    w.sem_off = w.acc_off + round_up(BH * n_pad * d * sizeof(float));
+    w.total = w.sem_off + (deterministic ? round_up(BH * (n_pad / 128) * sizeof(int)) : 0);
+    return w;
+}
+
+int validate_common(int B, int H, int n, int d, float scale, int dtype) {
+    if (B < 1 || H < 1 || n < 1) return ATTN_ERR_INVALID;
+    if (!(scale > 0.f) || !isfinite(scale)) return ATTN_ERR_INVALID;
+    if (static_cast<long long>(B) * H > 0x7fffffffLL) return ATTN_ERR_INVALID;
+    if (dtype != ATTN_BF16 && dtype != ATTN_FP32) return ATTN_ERR_UNSUPPORTED;
+    if (d != 32 && d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    return ATTN_OK;
+}
+
+}  // namespace
+
+cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int BH, int n, int d) {
+    auto fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    const int chunk = d >= 64 ? 64 : d;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n),
+                          static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                             static_cast<cuuint64_t>(d) * 2 * static_cast<cuuint64_t>(n)};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(chunk), 128u, 1u};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    const CUtensorMapSwizzle swz =
+        chunk == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t launch_wait_selftest(uint64_t timeout_ns, cudaStream_t stream) {
+    wait_selftest_kernel<<<1, 32, 0, stream>>>(timeout_ns);
+    return cudaGetLastError();
+}
+
+}  // namespace attn
+
+using namespace attn;
+
+extern "C" {
+
+int attn_version(void) { return 100; }
+
+const char* attn_error_string(int code) {
+    switch (code) {
+        case ATTN_OK: return "ok";
+        case ATTN_ERR_INVALID: return "invalid argument";
+        case ATTN_ERR_UNSUPPORTED: return "unsupported configuration";
+        case ATTN_ERR_CUDA: return "CUDA error";
+        case ATTN_ERR_TIMEOUT: return "device-side wait timed out";
+        case ATTN_ERR_WORKSPACE: return "workspace too small";
+        default: return "unknown error";
+    }
+}
+
+unsigned attn_set_wait_timeout_us(unsigned us) {
+    if (us < 100u) us = 100u;
+    return g_timeout_us.exchange(us);
+}
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+             int n, int d, float scale, int causal, int dtype, void* stream) {
+    if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID;
+    int rc = validate_common(B, H, n, d, scale, dtype);
+    if (rc) return rc;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return ATTN_ERR_INVALID;
+    FwdArgs a;
+    a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
+    a.B = B; a.H = H; a.n = n; a.d = d;
+    a.scale = scale;
+    a.causal = causal ? 1 : 0;
+    a.timeout_ns = static_cast<uint64_t>(g_timeout_us.load()) * 1000ull;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = (dtype == ATTN_BF16) ? launch_fwd_bf16(a, s) : launch_fwd_f32(a, s);
+    return to_code(e);
+}
+
+size_t attn_bwd_workspace_bytes(int B, int H, int n, int d, int deterministic) {
+    if (B < 1 || H < 1 || n < 1 || d < 1) return 0;
+    return ws_layout(B, H, n, d, deterministic).total;
+}
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+             const float* lse, void* dq, void* dk, void* dv, int B, int H, int n, int d,
+             float scale, int causal, int dtype, int deterministic, void* workspace,
+             size_t ws_bytes, void* stream) {
+    if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return ATTN_ERR_INVALID;
+    int rc = validate_common(B, H, n, d, scale, dtype);
+    if (rc) return rc;
+    if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+    const void* ptrs[] = {q, k, v, o, dO, lse, dq, dk, dv};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return ATTN_ERR_INVALID;
+    WsLayout w = ws_layout(B, H, n, d, deterministic);
+    if (!workspace) return ATTN_ERR_INVALID;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_INVALID;
+    if (ws_bytes < w.total) return ATTN_ERR_WORKSPACE;
+    BwdArgs a;
+    a.q = q; a.k = k; a.v = v; a.o = o; a.dO = dO; a.lse = lse;
+    a.dq = dq; a.dk = dk; a.dv = dv;
+    a.B = B; a.H = H; a.n = n; a.d = d;
+    a.scale = scale;
+    a.causal = causal ? 1 : 0;
+    a.deterministic = deterministic ? 1 : 0;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    a.Dvec = reinterpret_cast<float*>(ws + w.d_off);
+    a.dq_acc = reinterpret_cast<float*>(ws + w.acc_off);
+    a.sems = deterministic ? reinterpret_cast<int*>(ws + w.sem_off) : nullptr;
+    a.timeout_ns = static_cast<uint64_t>(g_timeout_us.load()) * 1000ull;
+    a.phase_events = g_phase_on.load() ? g_phase_events : nullptr;
+    return to_code(launch_bwd_bf16(a, static_cast<cudaStream_t>(stream)));
+}
+
+void attn_set_bwd_phase_events(void* const* events) {
+    if (!events) {
+        g_phase_on.store(false);
+        return;
+    }
+    for (int i = 0; i < 4; ++i) g_phase_events[i] = static_cast<cudaEvent_t>(events[i]);
+    g_phase_on.store(true);
+}
+
+int attn_get_device_status(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+    }
+    return v;
+}
+
+int attn_selftest_wait_timeout(unsigned timeout_us, void* stream) {
+    if (timeout_us == 0 || timeout_us > 10000000u) return ATTN_ERR_INVALID;
+    return to_code(launch_wait_selftest(static_cast<uint64_t>(timeout_us) * 1000ull,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

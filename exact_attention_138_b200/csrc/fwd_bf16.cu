@@ -1,0 +1,409 @@
+// Forward pass, bf16 in / bf16 out, fp32 accumulation, on the sm_100a tensor cores.
+//
+// The method is the tiled forward pass with online softmax: Q, K and V are split into tiles held
+// on chip, each tile updates a running row max m and row sum l, and the running output is
+// rescaled when m grows, so the n x n score matrix never reaches device memory ("Attention
+// Mechanism: Revolusi Representasi Sequence", §13 "FlashAttention — How It Works"; "Flash
+// Attention Nedir?", sections "Tiling (Blok Bölümleme)" and "Online Softmax"). The output update
+// carries the factor exp(m_old - m_new) on the old term; the division by l is deferred to the
+// end (the same value in exact arithmetic).
+//
+// B200 mapping (one CTA per pair of 128-row query tiles of one (b,h)):
+//   warp 8      TMA producer: Q tiles once, then K_j / V_j tiles through a STAGES-deep ring.
+//   warp 9      one thread issues every tcgen05.mma:  S_g = Q_g·K_j^T (SMEM x SMEM -> TMEM) and
+//               O_g += P_g·V_j (P from TMEM, V from SMEM), and signals through tcgen05.commit.
+//   warps 0-3   softmax of query tile 0, warps 4-7 softmax of query tile 1: one thread per row
+//               (= one TMEM lane). They read S from TMEM, apply the causal mask on the diagonal
+//               tile, update m/l, rescale O in TMEM when m grows, and write P (bf16) back over S.
+//   The two query tiles alternate, so the tensor cores run one tile's MMAs while the other tile's
+//   softmax runs. TMEM (512 columns): O_0 | O_1 | S_0 (P_0) | S_1 (P_1), 128 columns each.
+//   Causal: query tile q only visits key tiles 0..q (tiles above the diagonal are skipped).
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace attn {
+
+namespace {
+
+constexpr int kFwdThreads = 384;   // 3 warpgroups
+constexpr float kLn2 = 0.69314718055994530942f;
+constexpr float kLog2e = 1.44269504088896340736f;
+
+template <int D>
+struct FwdCfg {
+    static constexpr int BM = 128;                       // query rows per tile
+    static constexpr int BN = 128;                       // keys per tile
+    static constexpr int CW = D >= 64 ? 64 : D;          // elements per swizzle row
+    static constexpr int NCH = D / CW;                   // swizzle chunks per tile row
+    static constexpr int SWB = CW * 2;                   // swizzle width in bytes
+    static constexpr uint32_t SWZ = SWB == 128 ? 2u : 4u;
+    static constexpr int CHUNK = 128 * SWB;              // bytes of one [128 rows x CW] chunk
+    static constexpr int TILE = NCH * CHUNK;             // bytes of one 128 x D tile
+    static constexpr int STAGES = D == 128 ? 2 : 3;
+    static constexpr int SMEM = (2 + 2 * STAGES) * TILE + 512;
+};
+
+struct FwdBars {
+    uint64_t q_full;
+    uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
+    uint64_t s_full[2], p_full[2], o_done[2];
+    uint64_t teardown;
+    uint32_t tmem_base;
+    int abort;
+};
+
+struct FwdKParams {
+    void* o;
+    float* lse;
+    int n, BH, n_pairs, causal;
+    float scale_log2;
+    uint64_t timeout_ns;
+};
+
+// Bounded wait that ignores the abort flag: used while draining in-flight copies/MMAs on the
+// way out, so that nothing is left writing into shared memory or TMEM after the CTA exits.
+__device__ __forceinline__ void drain_wait_fwd(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer_ns() - t0 > limit_ns) {
+            report_error(4);
+            return;
+        }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
+                    const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const FwdKParams p) {
+    using C = FwdCfg<D>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t* sQ = smem;                                   // 2 tiles
+    uint8_t* sK = smem + 2 * C::TILE;                     // STAGES tiles
+    uint8_t* sV = sK + C::STAGES * C::TILE;               // STAGES tiles
+    FwdBars* bars = reinterpret_cast<FwdBars*>(sV + C::STAGES * C::TILE);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int L = blockIdx.x;
+    const int pair = p.n_pairs - 1 - L / p.BH;           // longest causal rows first
+    const int bh = L % p.BH;
+    const int n = p.n;
+    const int n_kv = (n + C::BN - 1) / C::BN;
+    int T[2];
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+        const int qt = 2 * pair + g;
+        T[g] = (qt * C::BM >= n) ? 0 : (p.causal ? min(n_kv, qt + 1) : n_kv);
+    }
+    const int Tmax = max(T[0], T[1]);
+
+    if (threadIdx.x == 0) {
+        if ((smem_addr(smem) & 1023u) != 0) report_error(3);
+        mbar_init(&bars->q_full, 1);
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&bars->k_full[s], 1);
+            mbar_init(&bars->k_empty[s], 1);
+            mbar_init(&bars->v_full[s], 1);
+            mbar_init(&bars->v_empty[s], 1);
+        }
+        for (int g = 0; g < 2; ++g) {
+            mbar_init(&bars->s_full[g], 1);
+            mbar_init(&bars->p_full[g], 128);
+            mbar_init(&bars->o_done[g], 1);
+        }
+        mbar_init(&bars->teardown, 1);
+        bars->abort = ((smem_addr(smem) & 1023u) != 0) ? 1 : 0;
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 9) tmem_alloc(&bars->tmem_base, 512);
+    if (warp == 8 && lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+    volatile int* abort = &bars->abort;
+    const uint64_t lim = p.timeout_ns;
+
+    if (warp == 8) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0 && !*abort) {
+            uint32_t qbytes = (T[0] > 0 ? C::TILE : 0) + (T[1] > 0 ? C::TILE : 0);
+            mbar_arrive_expect_tx(&bars->q_full, qbytes);
+            for (int g = 0; g < 2; ++g)
+                if (T[g] > 0)
+                    for (int ch = 0; ch < C::NCH; ++ch)
+                        tma_load_3d(sQ + g * C::TILE + ch * C::CHUNK, &tmQ, &bars->q_full,
+                                    ch * C::CW, (2 * pair + g) * C::BM, bh);
+            int issued = 0;
+            for (int jj = 0; jj < Tmax; ++jj) {
+                const int s = jj % C::STAGES;
+                const int f = jj / C::STAGES;
+                if (f > 0 && !bounded_wait(&bars->k_empty[s], (f - 1) & 1, abort, lim)) break;
+                mbar_arrive_expect_tx(&bars->k_full[s], C::TILE);
+                for (int ch = 0; ch < C::NCH; ++ch)
+                    tma_load_3d(sK + s * C::TILE + ch * C::CHUNK, &tmK, &bars->k_full[s],
+                                ch * C::CW, jj * C::BN, bh);
+                issued = 2 * jj + 1;
+                if (f > 0 && !bounded_wait(&bars->v_empty[s], (f - 1) & 1, abort, lim)) break;
+                mbar_arrive_expect_tx(&bars->v_full[s], C::TILE);
+                for (int ch = 0; ch < C::NCH; ++ch)
+                    tma_load_3d(sV + s * C::TILE + ch * C::CHUNK, &tmV, &bars->v_full[s],
+                                ch * C::CW, jj * C::BN, bh);
+                issued = 2 * jj + 2;
+            }
+            if (*abort) {
+                // let every copy issued so far land before the CTA can exit
+                drain_wait_fwd(&bars->q_full, 0, 100000000ull);
+                for (int x = 0; x < issued; ++x) {
+                    const int jj = x >> 1;
+                    const int s = jj % C::STAGES;
+                    drain_wait_fwd((x & 1) ? &bars->v_full[s] : &bars->k_full[s],
+                               (jj / C::STAGES) & 1, 100000000ull);
+                }
+            }
+        }
+    } else if (warp == 9) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);
+            constexpr uint32_t idPV = idesc_bf16_f32(128, D, 0, 1);
+            const uint32_t sQa = smem_addr(sQ), sKa = smem_addr(sK), sVa = smem_addr(sV);
+            bool ok = bounded_wait(&bars->q_full, 0, abort, lim);
+            tc_fence_after();
+            int k_ready = -1;
+            auto wait_k = [&](int jj) -> bool {
+                if (k_ready >= jj) return true;
+                if (!bounded_wait(&bars->k_full[jj % C::STAGES], (jj / C::STAGES) & 1, abort,
+                                  lim))
+                    return false;
+                tc_fence_after();
+                k_ready = jj;
+                return true;
+            };
+            // descriptors are built once per operand tile; a k-step only moves the start
+            // address field (bits [0,14), 16-byte units), which never carries out of the field
+            // because every shared-memory address is below 256 KB.
+            auto issue_s = [&](int g, int jj) {
+                const uint64_t a0 = smem_desc(sQa + g * C::TILE, 16, 8 * C::SWB, C::SWZ);
+                const uint64_t b0 =
+                    smem_desc(sKa + (jj % C::STAGES) * C::TILE, 16, 8 * C::SWB, C::SWZ);
+#pragma unroll 1
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint32_t off = (((ks * 16) / C::CW) * C::CHUNK + ((ks * 16) % C::CW) * 2) >> 4;
+                    mma_ss(tmem + 256 + g * 128, a0 + off, b0 + off, idS, ks > 0 ? 1u : 0u);
+                }
+            };
+            auto issue_pv = [&](int g, int jj) {
+                const uint64_t b0 =
+                    smem_desc(sVa + (jj % C::STAGES) * C::TILE, C::CHUNK, 8 * C::SWB, C::SWZ);
+#pragma unroll 1
+                for (int ks = 0; ks < C::BN / 16; ++ks)
+                    mma_ts(tmem + g * 128, tmem + 256 + g * 128 + ks * 8,
+                           b0 + static_cast<uint32_t>((ks * 16 * C::SWB) >> 4), idPV,
+                           (jj > 0 || ks > 0) ? 1u : 0u);
+            };
+            if (ok) ok = wait_k(0);
+            if (ok) {
+                for (int g = 0; g < 2; ++g)
+                    if (T[g] > 0) {
+                        issue_s(g, 0);
+                        mma_commit(&bars->s_full[g]);
+                    }
+                mma_commit(&bars->k_empty[0]);
+            }
+            for (int jj = 0; ok && jj < Tmax; ++jj) {
+                bool v_ready = false;
+                for (int g = 0; g < 2 && ok; ++g) {
+                    if (jj >= T[g]) continue;
+                    if (!bounded_wait(&bars->p_full[g], jj & 1, abort, lim)) { ok = false; break; }
+                    tc_fence_after();
+                    if (!v_ready) {
+                        if (!bounded_wait(&bars->v_full[jj % C::STAGES], (jj / C::STAGES) & 1,
+                                          abort, lim)) { ok = false; break; }
+                        tc_fence_after();
+                        v_ready = true;
+                    }
+                    issue_pv(g, jj);
+                    if (jj + 1 < T[g]) {
+                        if (!wait_k(jj + 1)) { ok = false; break; }
+                        issue_s(g, jj + 1);
+                        mma_commit(&bars->s_full[g]);
+                    } else {
+                        mma_commit(&bars->o_done[g]);
+                    }
+                }
+                if (!ok) break;
+                mma_commit(&bars->v_empty[jj % C::STAGES]);
+                if (jj + 1 < Tmax) mma_commit(&bars->k_empty[(jj + 1) % C::STAGES]);
+            }
+            // all MMAs of this CTA complete before TMEM is released
+            mma_commit(&bars->teardown);
+            drain_wait_fwd(&bars->teardown, 0, 100000000ull);
+        }
+        __syncwarp();
+    } else if (warp < 8) {
+        // ---------------------------------------------------------------- softmax warpgroups
+        const int g = warp >> 2;
+        const int wq = warp & 3;
+        const int r = wq * 32 + lane;                     // row within the tile = TMEM lane
+        const int qt = 2 * pair + g;
+        const int qidx = qt * C::BM + r;
+        const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+        const uint32_t tS = tmem + lane_base + 256 + g * 128;
+        const uint32_t tO = tmem + lane_base + g * 128;
+        const float sl2 = p.scale_log2;
+        float m = -INFINITY;   // running max of scale*log2(e)*s
+        float l = 0.f;         // running sum of exp2(.. - m)
+        bool ok = true;
+        for (int jj = 0; jj < T[g]; ++jj) {
+            ok = bounded_wait(&bars->s_full[g], jj & 1, abort, lim);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            // pass 1: row max of this tile (masked), read from TMEM in 32-column chunks
+            const int kbase = jj * C::BN;
+            const bool edge = (p.causal && jj == qt) || kbase + C::BN > n;
+            float mx = -INFINITY;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t u[32];
+                tmem_ld32(tS + c * 32, u);
+                tmem_ld_wait();
+#pragma unroll
+                for (int x = 0; x < 32; ++x) {
+                    float v = __uint_as_float(u[x]);
+                    const int kidx = kbase + c * 32 + x;
+                    if (edge && (kidx >= n || (p.causal && kidx > qidx))) v = -INFINITY;
+                    mx = fmaxf(mx, v);
+                }
+            }
+            const float m_new = fmaxf(m, mx * sl2);
+            const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+            const float alpha = ex2_approx(m - m_use);
+            if (jj > 0 && __any_sync(0xffffffffu, m_new != m)) {
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t u[32];
+                    tmem_ld32(tO + c * 32, u);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int x = 0; x < 32; ++x)
+                        u[x] = __float_as_uint(__uint_as_float(u[x]) * alpha);
+                    tmem_st32(tO + c * 32, u);
+                }
+            }
+            // pass 2: P = exp2(s·scale·log2e - m), row sum, bf16 P written over the S columns
+            // already read (chunk c of S -> packed P columns 16c .. 16c+15)
+            float rs = 0.f;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t u[32];
+                tmem_ld32(tS + c * 32, u);
+                tmem_ld_wait();
+                uint32_t w[16];
+#pragma unroll
+                for (int x = 0; x < 16; ++x) {
+                    float v0 = ex2_approx(fmaf(__uint_as_float(u[2 * x]), sl2, -m_use));
+                    float v1 = ex2_approx(fmaf(__uint_as_float(u[2 * x + 1]), sl2, -m_use));
+                    if (edge) {
+                        const int k0 = kbase + c * 32 + 2 * x;
+                        if (k0 >= n || (p.causal && k0 > qidx)) v0 = 0.f;
+                        if (k0 + 1 >= n || (p.causal && k0 + 1 > qidx)) v1 = 0.f;
+                    }
+                    rs += v0 + v1;
+                    w[x] = pack_bf16x2(v0, v1);
+                }
+                tmem_st16(tS + c * 16, w);
+            }
+            l = l * alpha + rs;
+            m = m_new;
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&bars->p_full[g]);
+        }
+        if (ok && T[g] > 0) {
+            ok = bounded_wait(&bars->o_done[g], 0, abort, lim);
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok) {
+                tc_fence_after();
+                const float inv_l = 1.f / l;
+                __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) +
+                                      (static_cast<size_t>(bh) * n + qidx) * D;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t u[32];
+                    tmem_ld32(tO + c * 32, u);
+                    tmem_ld_wait();
+                    uint32_t w[16];
+#pragma unroll
+                    for (int x = 0; x < 16; ++x)
+                        w[x] = pack_bf16x2(__uint_as_float(u[2 * x]) * inv_l,
+                                           __uint_as_float(u[2 * x + 1]) * inv_l);
+                    if (qidx < n) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+                        for (int x = 0; x < 4; ++x)
+                            dst[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
+                    }
+                }
+                if (qidx < n)
+                    p.lse[static_cast<size_t>(bh) * n + qidx] = (m + __log2f(l)) * kLn2;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+template <int D>
+cudaError_t launch_fwd_bf16_d(const FwdArgs& a, cudaStream_t stream) {
+    using C = FwdCfg<D>;
+    CUtensorMap mq, mk, mv;
+    const int BH = a.B * a.H;
+    cudaError_t e;
+    if ((e = make_tmap_bf16(&mq, a.q, BH, a.n, D)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16(&mk, a.k, BH, a.n, D)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16(&mv, a.v, BH, a.n, D)) != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(fwd_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM);
+    if (e != cudaSuccess) return e;
+    FwdKParams kp;
+    kp.o = a.o;
+    kp.lse = a.lse;
+    kp.n = a.n;
+    kp.BH = BH;
+    const int nq = (a.n + 127) / 128;
+    kp.n_pairs = (nq + 1) / 2;
+    kp.causal = a.causal;
+    kp.scale_log2 = a.scale * kLog2e;
+    kp.timeout_ns = a.timeout_ns;
+    const long long grid = static_cast<long long>(kp.n_pairs) * BH;
+    if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    fwd_bf16_kernel<D><<<static_cast<unsigned>(grid), kFwdThreads, C::SMEM, stream>>>(mq, mk, mv, kp);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_bf16(const FwdArgs& a, cudaStream_t stream) {
+    switch (a.d) {
+        case 32: return launch_fwd_bf16_d<32>(a, stream);
+        case 64: return launch_fwd_bf16_d<64>(a, stream);
+        case 128: return launch_fwd_bf16_d<128>(a, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace attn

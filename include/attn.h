@@ -1,0 +1,118 @@
+/*
+ * attn.h — C ABI of libattn.so: exact scaled dot-product attention on one NVIDIA B200 (sm_100a).
+ *
+ * The operation (forward):
+ *     O = softmax(scale · Q·K^T + M) · V,     LSE_i = ln sum_j exp(scale · q_i·k_j + M_ij)
+ *   "Attention Mechanism: Revolusi Representasi Sequence", §3 "Scaled Dot-Product Attention:
+ *   Formula Inti" (Steps 1-4: scores, scaling, row softmax, weighted sum of V rows) and §4.4
+ *   "Causal / Masked Attention" (M_ij = 0 for j <= i, -inf for j > i). The row log-sum-exp is the
+ *   statistic of "Flash Attention Nedir?", section "Online Softmax"; it is returned in the natural
+ *   log so that the backward pass can rebuild P = exp(scale·q·k - LSE) tile by tile ("Apa itu
+ *   FlashAttention", "Cara kerja teknik Tiling dan Recomputation", item 2).
+ *   Q, K, V tiles are processed on chip with an online softmax, so the n x n score matrix of
+ *   "Calculateur de mémoire d'attention" ("La formule") is never written to device memory.
+ *
+ * The operation (backward), the exact derivative of the forward definition:
+ *     P = exp(scale·Q·K^T + M - LSE),  dV = P^T·dO,  dP = dO·V^T,  D_i = sum_c dO_ic·O_ic,
+ *     dS = P∘(dP - D),  dQ = scale·dS·K,  dK = scale·dS^T·Q.
+ *
+ * Layout and ownership (all calls):
+ *   - q, k, v, o, dO, dq, dk, dv: caller-owned DEVICE memory, contiguous row-major (B, H, n, d):
+ *     element (b, h, i, c) at offset ((b*H + h)*n + i)*d + c. bf16 (ATTN_BF16) or fp32
+ *     (ATTN_FP32) elements. Base addresses must be 16-byte aligned (TMA requirement).
+ *   - lse: caller-owned DEVICE memory, fp32, (B, H, n), 16-byte aligned.
+ *   - Self-attention only: the query and key lengths are both n; d is the head dimension of Q, K
+ *     and V alike.
+ *   - scale: the factor applied to Q·K^T (normally 1/sqrt(d)); any finite positive value.
+ *   - stream: a cudaStream_t (NULL = the legacy default stream). Every call is asynchronous on
+ *     that stream; the library keeps no allocation between calls except cached tensor-map
+ *     encoder entry points.
+ *
+ * Errors: each call validates its arguments before launching anything and returns ATTN_OK or
+ *   ATTN_ERR_INVALID   null pointer, B, H or n < 1, misaligned pointer, non-finite or <= 0 scale,
+ *                      workspace pointer null while ws_bytes > 0;
+ *   ATTN_ERR_UNSUPPORTED  d not in {32, 64, 128}; fp32 backward; an unknown dtype;
+ *   ATTN_ERR_WORKSPACE    ws_bytes smaller than attn_bwd_workspace_bytes();
+ *   ATTN_ERR_CUDA      a launch or encode error reported by the CUDA runtime / driver;
+ *   ATTN_ERR_TIMEOUT   reported by attn_get_device_status(): a device-side wait ran past its
+ *                      limit and the kernel returned early (outputs are then undefined).
+ */
+#ifndef ATTN_H
+#define ATTN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { ATTN_BF16 = 0, ATTN_FP32 = 1 } attn_dtype;
+
+enum {
+    ATTN_OK = 0,
+    ATTN_ERR_INVALID = 1,
+    ATTN_ERR_UNSUPPORTED = 2,
+    ATTN_ERR_CUDA = 3,
+    ATTN_ERR_TIMEOUT = 4,
+    ATTN_ERR_WORKSPACE = 5
+};
+
+/* Library ABI version (major*100 + minor). */
+int attn_version(void);
+
+/* Forward pass. Writes o (same dtype as q) and lse (fp32).
+ *   dtype ATTN_BF16: tcgen05 tensor-core kernel, fp32 accumulation, P rounded to bf16 before P·V,
+ *                    O rounded to bf16 (round-to-nearest-even).
+ *   dtype ATTN_FP32: exact fp32 kernel on the FMA pipes (no TF32), for the pages' float32 cases.
+ * causal != 0 applies the mask M of §4.4 (query i sees keys 0..i). */
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+             int B, int H, int n, int d, float scale, int causal, int dtype, void* stream);
+
+/* Bytes of device workspace attn_bwd needs for these sizes: the D vector (B·H·n fp32, padded per
+ * head to a multiple of 128 rows) and the fp32 dQ accumulator (B·H·n·d fp32, padded the same
+ * way), each rounded up to 256 bytes; with deterministic != 0 also one semaphore per query tile. */
+size_t attn_bwd_workspace_bytes(int B, int H, int n, int d, int deterministic);
+
+/* Backward pass (bf16 only). Inputs q, k, v, o, dO (bf16) and lse (fp32, from attn_fwd with the
+ * same scale and causal flag). Writes dq, dk, dv (bf16). The workspace (caller-owned device
+ * memory of at least attn_bwd_workspace_bytes() bytes, 256-byte aligned) is overwritten.
+ *   deterministic == 0: dQ partial tiles are added to the fp32 accumulator with atomic adds, so
+ *                       the rounding order (and the last bits of dq) can vary between runs.
+ *   deterministic != 0: each query tile's partials are added in increasing key-tile order, so
+ *                       repeated runs give identical bits. */
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+             const float* lse, void* dq, void* dk, void* dv,
+             int B, int H, int n, int d, float scale, int causal, int dtype, int deterministic,
+             void* workspace, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, then returns and clears the sticky device status word: ATTN_OK, or
+ * ATTN_ERR_TIMEOUT if a kernel's bounded wait expired since the last call, or ATTN_ERR_CUDA if
+ * the synchronisation itself failed. */
+int attn_get_device_status(void* stream);
+
+/* Sets the limit of every device-side wait, in microseconds (default 2,000,000 = 2 s). Values
+ * below 100 are raised to 100. Returns the previous value. */
+unsigned attn_set_wait_timeout_us(unsigned us);
+
+/* Self-test of the bounded-wait path: launches one CTA that waits on an mbarrier no thread ever
+ * arrives on, with a limit of `timeout_us` microseconds, so the wait expires and the kernel sets
+ * ATTN_ERR_TIMEOUT and returns. Returns the launch status; read the result with
+ * attn_get_device_status(). Never faults or hangs the device. */
+int attn_selftest_wait_timeout(unsigned timeout_us, void* stream);
+
+/* Measurement hook. `events` is NULL (recording off, the default) or an array of 4 cudaEvent_t
+ * created by the caller. While set, every attn_bwd call records, on its stream, events[0] before
+ * its preprocess kernel (D = rowsum(dO∘O)), events[1] before its main kernel, events[2] after
+ * the main kernel and events[3] after the dQ conversion kernel, so that a caller can time the
+ * three kernels separately with cudaEventElapsedTime. The array is copied; the events must stay
+ * valid while recording is on. Process-wide setting; not meant for concurrent callers. */
+void attn_set_bwd_phase_events(void* const* events);
+
+/* Static string for an error code. */
+const char* attn_error_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_H */

@@ -1,0 +1,98 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every function that
+include/attn.h declares, and rejects bad arguments before touching the device."""
+import ctypes
+
+import pytest
+
+import exact_attention_138_b200 as ea
+
+FAKE = 1 << 20          # an aligned, never-dereferenced pointer value (validation fails first)
+
+
+def test_every_declared_function_is_exported():
+    names = ea.declared_functions()
+    assert {"attn_fwd", "attn_bwd", "attn_bwd_workspace_bytes", "attn_get_device_status",
+            "attn_error_string", "attn_version", "attn_set_wait_timeout_us",
+            "attn_selftest_wait_timeout"} <= set(names)
+    lib = ea.library()
+    for name in names:
+        assert hasattr(lib, name), name
+
+
+def test_version_and_error_strings():
+    assert ea.attn_version() >= 100
+    for code in range(6):
+        assert ea.attn_error_string(code) and ea.attn_error_string(code) != "unknown error"
+    assert ea.attn_error_string(99) == "unknown error"
+
+
+def test_workspace_size_formula():
+    # D (fp32, per-head rows padded to 128) + dQ accumulator (fp32, same rows x d), 256-aligned
+    n_pad = 256
+    want = 2 * 3 * n_pad * 4 + 2 * 3 * n_pad * 64 * 4
+    assert ea.attn_bwd_workspace_bytes(2, 3, 200, 64, 0) == want
+    assert ea.attn_bwd_workspace_bytes(2, 3, 200, 64, 1) == want + 256   # 6 semaphores -> 256 B
+    assert ea.attn_bwd_workspace_bytes(0, 3, 200, 64, 0) == 0
+
+
+def _fwd(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, H=1, n=128, d=64, scale=0.125,
+             causal=0, dtype=ea.ATTN_BF16, stream=None)
+    a.update(kw)
+    return ea.attn_fwd(*(ctypes.c_void_p(a[x]) if x in "q k v o lse".split() else a[x]
+                         for x in "q k v o lse B H n d scale causal dtype stream".split()))
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=0), ea.ATTN_ERR_INVALID),
+    (dict(lse=0), ea.ATTN_ERR_INVALID),
+    (dict(n=0), ea.ATTN_ERR_INVALID),
+    (dict(B=0), ea.ATTN_ERR_INVALID),
+    (dict(H=-1), ea.ATTN_ERR_INVALID),
+    (dict(scale=0.0), ea.ATTN_ERR_INVALID),
+    (dict(scale=float("inf")), ea.ATTN_ERR_INVALID),
+    (dict(scale=float("nan")), ea.ATTN_ERR_INVALID),
+    (dict(d=48), ea.ATTN_ERR_UNSUPPORTED),
+    (dict(d=256), ea.ATTN_ERR_UNSUPPORTED),
+    (dict(dtype=7), ea.ATTN_ERR_UNSUPPORTED),
+    (dict(v=FAKE + 8), ea.ATTN_ERR_INVALID),       # not 16-byte aligned
+    (dict(o=FAKE + 2), ea.ATTN_ERR_INVALID),
+])
+def test_forward_rejects_bad_arguments(kw, code):
+    assert _fwd(**kw) == code
+
+
+def _bwd(**kw):
+    a = dict(B=1, H=2, n=300, d=128, scale=0.1, causal=1, dtype=ea.ATTN_BF16, det=0)
+    a.update(kw)
+    ptrs = [ctypes.c_void_p(kw.get(p, FAKE)) for p in "q k v o dO lse dq dk dv".split()]
+    need = ea.attn_bwd_workspace_bytes(a["B"], a["H"], a["n"], a["d"], a["det"]) if a["B"] > 0 else 0
+    ws = kw.get("ws", FAKE)
+    ws_bytes = kw.get("ws_bytes", need)
+    return ea.attn_bwd(*ptrs, a["B"], a["H"], a["n"], a["d"], a["scale"], a["causal"], a["dtype"],
+                       a["det"], ctypes.c_void_p(ws), ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dO=0), ea.ATTN_ERR_INVALID),
+    (dict(dv=0), ea.ATTN_ERR_INVALID),
+    (dict(dtype=ea.ATTN_FP32), ea.ATTN_ERR_UNSUPPORTED),
+    (dict(d=96), ea.ATTN_ERR_UNSUPPORTED),
+    (dict(ws=0), ea.ATTN_ERR_INVALID),
+    (dict(ws=FAKE + 16), ea.ATTN_ERR_INVALID),      # workspace must be 256-byte aligned
+    (dict(ws_bytes=1000), ea.ATTN_ERR_WORKSPACE),
+    (dict(n=0), ea.ATTN_ERR_INVALID),
+    (dict(dq=FAKE + 4), ea.ATTN_ERR_INVALID),
+])
+def test_backward_rejects_bad_arguments(kw, code):
+    assert _bwd(**kw) == code
+
+
+def test_selftest_rejects_bad_limit():
+    assert ea.attn_selftest_wait_timeout(0) == ea.ATTN_ERR_INVALID
+    assert ea.attn_selftest_wait_timeout(20_000_000) == ea.ATTN_ERR_INVALID
+
+
+def test_timeout_setter_roundtrip():
+    old = ea.attn_set_wait_timeout_us(5)
+    assert ea.attn_set_wait_timeout_us(old) == 100      # raised to the 100 us floor
