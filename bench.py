@@ -169,8 +169,10 @@ def run_reference(args, w):
     import attn_inputs
     q, k, v, do = attn_inputs.workload_inputs(w)
     times, flops_rate, rows_used, threads = [], [], 0, 1
+    # each step is a bounded sample, sized so that the whole run stays within ~2 minutes
+    per_step = min(args.ref_seconds, 120.0 / (args.warmup + args.steps))
     for i in range(args.warmup + args.steps):
-        rate, dt, rows_n, threads = oracle_sample(args.ref_seconds, q, k, v, do, w, 9 + i)
+        rate, dt, rows_n, threads = oracle_sample(per_step, q, k, v, do, w, 9 + i)
         if i >= args.warmup:
             times.append(dt)
             flops_rate.append(rate)
@@ -184,7 +186,7 @@ def run_reference(args, w):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000 * statistics.mean(times), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "B": w.B, "H": w.H, "n": w.n, "d": w.d,
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "n": w.n, "d": w.d,
                    "causal": True, "sample": sample},
         "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": threads,
                          "kind": "oracle", "sample": sample},
@@ -205,12 +207,17 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    help="named workload of attn_inputs.WORKLOADS (profiling runs use a smaller "
+                         "one; the headline is the default)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
     import attn_inputs
-    w = attn_inputs.WORKLOADS[WORKLOAD]
+    w = attn_inputs.WORKLOADS[args.workload]
+    if not (w.causal and w.dtype == "bf16" and w.backward):
+        ap.error("the bench workload must be a causal bf16 forward+backward workload")
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -259,6 +266,10 @@ def main():
 
     # --- timed region: K steps; per-kernel events for the roofline
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    for row in ev:              # torch creates the CUDA event at its first record
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
@@ -339,10 +350,11 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "B": w.B, "H": w.H, "n": w.n, "d": w.d, "causal": True,
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "n": w.n, "d": w.d, "causal": True,
                    "input_factor": w.factor, "global_batch": w.B * world,
                    "parallelism": f"dp{world}" if world > 1 else "single",
-                   "l2": "inputs larger than L2 (q,k,v,dO 128 MiB each); no flush"},
+                   "l2": f"inputs larger than L2 (q,k,v,dO {w.B*w.H*w.n*w.d*2/2**20:.0f} MiB "
+                         f"each); no flush"},
         "fwd": {"ms": statistics.mean(fwd_ms), "tflops": fwd_tf,
                 "pct_of_burst_peak": 100 * fwd_tf / burst},
         "bwd": {"ms": statistics.mean(bwd_ms), "tflops": bwd_tf,

@@ -1,7 +1,7 @@
 """exact_attention_138_b200 — exact scaled dot-product attention on one B200 (sm_100a).
 
 Python binding of the C ABI in ``include/attn.h`` (``libattn.so``, built in-tree by
-``python -m exact_attention_138_b200.build``). This module only marshals arguments: device
+``python exact_attention_138_b200/build.py``). This module only marshals arguments: device
 memory and streams come from PyTorch, every step of the computation runs in the library's
 CUDA kernels. There is no CPU fallback: if the library is missing the import fails.
 
@@ -29,7 +29,7 @@ ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT, ATTN_ERR_WORKSPACE = 3, 4, 5
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m exact_attention_138_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python exact_attention_138_b200/build.py` "
         "(there is no fallback implementation)")
 
 _lib = ctypes.CDLL(LIB_PATH)

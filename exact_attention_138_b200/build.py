@@ -1,6 +1,6 @@
 """Build libattn.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-    python -m exact_attention_138_b200.build [--force]
+    python exact_attention_138_b200/build.py [--force]
 
 The whole library is one translation unit (csrc/libattn.cu), compiled for
 compute_100a/sm_100a only, with -lineinfo for profiling, static cudart, and no link-time

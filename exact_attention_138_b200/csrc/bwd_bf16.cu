@@ -28,7 +28,7 @@ namespace attn {
 
 namespace {
 
-constexpr int kBwdThreads = 192;
+constexpr int kBwdThreads = 320;
 constexpr float kBwdLog2e = 1.44269504088896340736f;
 
 template <int D>
@@ -40,7 +40,8 @@ struct BwdCfg {
     static constexpr int CHUNK = 128 * SWB;
     static constexpr int TILE = NCH * CHUNK;              // 128 x D bf16
     static constexpr int DS_BYTES = 128 * 128 * 2;         // dS^T tile, 2 x [128 x 64] SW128
-    static constexpr int STAT_BYTES = 2 * 2 * 128 * 4;     // LSE·log2e and D, double-buffered
+    static constexpr int STAT_BYTES = 2 * 2 * 128 * 4;     // [warpgroup][buffer][LSE2 | D] x 64
+    static constexpr bool DQT = (D == 128);                // dQ computed transposed (see kernel)
     static constexpr int SMEM = 6 * TILE + DS_BYTES + STAT_BYTES + 256;
 };
 
@@ -72,10 +73,6 @@ __device__ __forceinline__ void drain_wait_bwd(uint64_t* bar, uint32_t parity, u
             report_error(4);
             return;
         }
-}
-
-__device__ __forceinline__ void compute_bar() {
-    asm volatile("bar.sync 1, 128;" ::: "memory");
 }
 
 // ------------------------------------------------------------------------------------------
@@ -163,6 +160,19 @@ __global__ void __launch_bounds__(256) bwd_dq_convert_kernel(const float* __rest
 
 // ------------------------------------------------------------------------------------------
 // Main backward kernel.
+//
+// Roles (320 threads): warps 0-3 = compute warpgroup 0 (query columns 0-63 of each tile),
+// warps 4-7 = compute warpgroup 1 (query columns 64-127), warp 8 = TMA producer, warp 9 = MMA
+// issuer. Every compute thread owns one key row (= TMEM lane) and half of the tile's columns.
+// Per query tile i the MMA thread issues, in this order,
+//     dP^T(i) [after dQ(i-1) has been drained out of the dP columns],
+//     dV += P^T(i)·dO(i) [after P^T(i) is in TMEM],   S^T(i+1) = K·Q(i+1)^T,
+//     dK += dS^T(i)·Q(i) and dQ(i) [after dS^T(i) is in shared memory],
+// while the compute warps run P(i) -> drain dQ(i-1) -> dS(i): the dQ drain of one tile and the
+// softmax of the next overlap the dK/dQ MMAs.
+// dQ: for d = 128 the MMA computes dQ^T = K^T·dS^T (TMEM lane = head-dim index, column = query),
+// so one warp-wide reduction covers 32 consecutive floats (128 B) of one dQ row; for d < 128 it
+// computes dQ = dS·K (lane = query) and each thread reduces 16-byte pieces of its row.
 // ------------------------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
@@ -175,8 +185,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint8_t* sV = sK + C::TILE;
     uint8_t* sQ = sV + C::TILE;                   // 2 stages
     uint8_t* sdO = sQ + 2 * C::TILE;              // 2 stages
-    uint8_t* sdS = sdO + 2 * C::TILE;             // 32 KB, 1024-aligned
-    float* sStat = reinterpret_cast<float*>(sdS + C::DS_BYTES);   // [2][2][128]
+    uint8_t* sdS = sdO + 2 * C::TILE;             // dS^T, 2 chunks [128 keys][64 queries], SW128
+    float* sStat = reinterpret_cast<float*>(sdS + C::DS_BYTES);   // [wg][buf][LSE2 64 | D 64]
     BwdBars* bars = reinterpret_cast<BwdBars*>(sdS + C::DS_BYTES + C::STAT_BYTES);
 
     constexpr uint32_t COL_DV = 0, COL_DK = 128, COL_S = 256, COL_DP = 384;
@@ -198,10 +208,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         mbar_init(&bars->s_full, 1);
         mbar_init(&bars->dp_full, 1);
-        mbar_init(&bars->p_full, 128);
-        mbar_init(&bars->ds_full, 128);
+        mbar_init(&bars->p_full, 256);
+        mbar_init(&bars->ds_full, 256);
         mbar_init(&bars->dq_full, 1);
-        mbar_init(&bars->dq_drained, 128);
+        mbar_init(&bars->dq_drained, 256);
         mbar_init(&bars->ds_free, 1);
         mbar_init(&bars->dkv_done, 1);
         mbar_init(&bars->teardown, 1);
@@ -210,8 +220,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         fence_barrier_init();
         fence_proxy_async_smem();
     }
-    if (warp == 5) tmem_alloc(&bars->tmem_base, 512);
-    if (warp == 4 && lane == 0) {
+    if (warp == 9) tmem_alloc(&bars->tmem_base, 512);
+    if (warp == 8 && lane == 0) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
@@ -224,7 +234,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     volatile int* abort = &bars->abort;
     const uint64_t lim = p.timeout_ns;
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ---------------------------------------------------------------- TMA producer
         if (lane == 0 && !*abort) {
             mbar_arrive_expect_tx(&bars->kv_full, 2 * C::TILE);
@@ -252,64 +262,92 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     drain_wait_bwd(&bars->q_full[it & 1], (it >> 1) & 1, 100000000ull);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);     // K-major x K-major
+            constexpr uint32_t idSS = idesc_bf16_f32(128, 128, 0, 0);    // K-major x K-major
             constexpr uint32_t idKN = idesc_bf16_f32(128, D, 0, 1);      // A K-major, B MN-major
-            constexpr uint32_t idQ = idesc_bf16_f32(128, D, 1, 1);       // A MN-major, B MN-major
+            constexpr uint32_t idDQ = C::DQT ? idesc_bf16_f32(128, 128, 1, 1)   // dQ^T
+                                             : idesc_bf16_f32(128, D, 1, 1);    // dQ
             const uint32_t aK = smem_addr(sK), aV = smem_addr(sV), aQ = smem_addr(sQ),
                            adO = smem_addr(sdO), adS = smem_addr(sdS);
+            // K-major descriptors of K_j / V_j (S^T, dP^T) and MN-major ones of K_j (dQ)
+            const uint64_t dK_kmaj = smem_desc(aK, 16, 8 * C::SWB, C::SWZ);
+            const uint64_t dV_kmaj = smem_desc(aV, 16, 8 * C::SWB, C::SWZ);
+            const uint64_t dK_mn = smem_desc(aK, C::CHUNK, 8 * C::SWB, C::SWZ);
+            const uint64_t dS_kmaj = smem_desc(adS, 16, 1024, 2u);
+            const uint64_t dS_mn = smem_desc(adS, 16384, 1024, 2u);
+            auto kstep_k = [](int ks) -> uint32_t {     // K-major k-step offset (16-byte units)
+                return static_cast<uint32_t>((((ks * 16) / C::CW) * C::CHUNK + ((ks * 16) % C::CW) * 2) >> 4);
+            };
+            auto issue_s = [&](int it) {                // S^T = K_j · Q_i^T
+                const uint64_t b0 = smem_desc(aQ + (it & 1) * C::TILE, 16, 8 * C::SWB, C::SWZ);
+#pragma unroll 1
+                for (int ks = 0; ks < D / 16; ++ks)
+                    mma_ss(tmem + COL_S, dK_kmaj + kstep_k(ks), b0 + kstep_k(ks), idSS, ks > 0);
+            };
+            auto issue_dp = [&](int it) {               // dP^T = V_j · dO_i^T
+                const uint64_t b0 = smem_desc(adO + (it & 1) * C::TILE, 16, 8 * C::SWB, C::SWZ);
+#pragma unroll 1
+                for (int ks = 0; ks < D / 16; ++ks)
+                    mma_ss(tmem + COL_DP, dV_kmaj + kstep_k(ks), b0 + kstep_k(ks), idSS, ks > 0);
+            };
             bool ok = bounded_wait(&bars->kv_full, 0, abort, lim);
+            if (ok) ok = bounded_wait(&bars->q_full[0], 0, abort, lim);
             tc_fence_after();
+            if (ok) {
+                issue_s(0);
+                mma_commit(&bars->s_full);
+                issue_dp(0);
+                mma_commit(&bars->dp_full);
+            }
             for (int it = 0; ok && it < NT; ++it) {
                 const int st = it & 1;
-                if (!(ok = bounded_wait(&bars->q_full[st], (it >> 1) & 1, abort, lim))) break;
-                tc_fence_after();
-                const uint32_t q_a = aQ + st * C::TILE, do_a = adO + st * C::TILE;
-                // S^T = K_j · Q_i^T   (M = keys, N = queries, K = d)
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t off = ((ks * 16) / C::CW) * C::CHUNK + ((ks * 16) % C::CW) * 2;
-                    mma_ss(tmem + COL_S, smem_desc(aK + off, 16, 8 * C::SWB, C::SWZ),
-                           smem_desc(q_a + off, 16, 8 * C::SWB, C::SWZ), idS, ks > 0 ? 1u : 0u);
-                }
-                mma_commit(&bars->s_full);
                 if (it > 0) {
                     if (!(ok = bounded_wait(&bars->dq_drained, (it - 1) & 1, abort, lim))) break;
                     tc_fence_after();
+                    issue_dp(it);
+                    mma_commit(&bars->dp_full);
                 }
-                // dP^T = V_j · dO_i^T
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t off = ((ks * 16) / C::CW) * C::CHUNK + ((ks * 16) % C::CW) * 2;
-                    mma_ss(tmem + COL_DP, smem_desc(aV + off, 16, 8 * C::SWB, C::SWZ),
-                           smem_desc(do_a + off, 16, 8 * C::SWB, C::SWZ), idS, ks > 0 ? 1u : 0u);
-                }
-                mma_commit(&bars->dp_full);
                 if (!(ok = bounded_wait(&bars->p_full, it & 1, abort, lim))) break;
                 tc_fence_after();
-                // dV_j += P^T · dO_i   (A = P^T from TMEM, B = dO_i MN-major; K = queries)
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    mma_ts(tmem + COL_DV, tmem + COL_S + ks * 8,
-                           smem_desc(do_a + ks * 16 * C::SWB, C::CHUNK, 8 * C::SWB, C::SWZ), idKN,
-                           (it > 0 || ks > 0) ? 1u : 0u);
+                {   // dV_j += P^T · dO_i   (P^T in TMEM: queries 0-63 at S+0.., 64-127 at S+64..)
+                    const uint64_t b0 = smem_desc(adO + st * C::TILE, C::CHUNK, 8 * C::SWB, C::SWZ);
+#pragma unroll 1
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_ts(tmem + COL_DV, tmem + COL_S + (ks >> 2) * 64 + (ks & 3) * 8,
+                               b0 + static_cast<uint32_t>((ks * 16 * C::SWB) >> 4), idKN,
+                               (it > 0 || ks > 0) ? 1u : 0u);
+                }
+                if (it + 1 < NT) {
+                    if (!(ok = bounded_wait(&bars->q_full[(it + 1) & 1], ((it + 1) >> 1) & 1,
+                                            abort, lim)))
+                        break;
+                    tc_fence_after();
+                    issue_s(it + 1);
+                    mma_commit(&bars->s_full);
+                }
                 if (!(ok = bounded_wait(&bars->ds_full, it & 1, abort, lim))) break;
                 tc_fence_after();
-                // dK_j += dS^T · Q_i   (A = dS^T K-major SW128, B = Q_i MN-major)
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    mma_ss(tmem + COL_DK,
-                           smem_desc(adS + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, 2u),
-                           smem_desc(q_a + ks * 16 * C::SWB, C::CHUNK, 8 * C::SWB, C::SWZ), idKN,
-                           (it > 0 || ks > 0) ? 1u : 0u);
-                // dQ_i = dS · K_j   (A = dS MN-major view of the same buffer, B = K_j MN-major)
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    mma_ss(tmem + COL_DP, smem_desc(adS + ks * 2048, 16384, 1024, 2u),
-                           smem_desc(aK + ks * 16 * C::SWB, C::CHUNK, 8 * C::SWB, C::SWZ), idQ,
-                           ks > 0 ? 1u : 0u);
+                {   // dK_j += dS^T · Q_i   (A = dS^T K-major, B = Q_i MN-major)
+                    const uint64_t b0 = smem_desc(aQ + st * C::TILE, C::CHUNK, 8 * C::SWB, C::SWZ);
+#pragma unroll 1
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_ss(tmem + COL_DK,
+                               dS_kmaj + static_cast<uint32_t>(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4),
+                               b0 + static_cast<uint32_t>((ks * 16 * C::SWB) >> 4), idKN,
+                               (it > 0 || ks > 0) ? 1u : 0u);
+                }
+                // dQ^T_i = K_j^T · dS^T  (d = 128)   or   dQ_i = dS · K_j   (d < 128)
+#pragma unroll 1
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint64_t kd = dK_mn + static_cast<uint32_t>((ks * 16 * C::SWB) >> 4);
+                    const uint64_t sd = dS_mn + static_cast<uint32_t>((ks * 2048) >> 4);
+                    if (C::DQT)
+                        mma_ss(tmem + COL_DP, kd, sd, idDQ, ks > 0 ? 1u : 0u);
+                    else
+                        mma_ss(tmem + COL_DP, sd, kd, idDQ, ks > 0 ? 1u : 0u);
+                }
                 mma_commit(&bars->dq_full);
                 mma_commit(&bars->ds_free);
                 mma_commit(&bars->q_empty[st]);
@@ -320,98 +358,42 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         __syncwarp();
     } else {
-        // ---------------------------------------------------------------- compute warps 0-3
-        const int r = warp * 32 + lane;                    // key row within tile = TMEM lane
+        // ---------------------------------------------------------------- compute warpgroups
+        const int g = warp >> 2;                           // warpgroup: query columns 64g..64g+63
+        const int t = threadIdx.x & 127;
+        const int r = (warp & 3) * 32 + lane;              // key row within the tile = TMEM lane
         const int kidx = j * 128 + r;
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        const int cb = g * 64;
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + lane_base + COL_S;
         const uint32_t tDP = tmem + lane_base + COL_DP;
         const float sl2 = p.scale_log2;
+        auto wg_bar = [&]() {
+            if (g == 0)
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+            else
+                asm volatile("bar.sync 2, 128;" ::: "memory");
+        };
+        auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
+            return __all_sync(0xffffffffu, bounded_wait(bar, par, abort, lim));
+        };
+        float pr[64];
         bool ok = true;
-        for (int it = 0; it < NT; ++it) {
+
+        // dQ partial of tile `it` out of TMEM into the fp32 accumulator
+        auto drain = [&](int it) -> bool {
             const int i = i_begin + it;
-            const int buf = it & 1;
-            float* sL = sStat + buf * 256;
-            float* sD = sL + 128;
-            {
-                const int q = i * 128 + r;
-                sL[r] = (q < n) ? p.lse[static_cast<size_t>(bh) * n + q] * kBwdLog2e : INFINITY;
-                sD[r] = (q < n) ? p.Dvec[static_cast<size_t>(bh) * p.n_pad + q] : 0.f;
-            }
-            compute_bar();
-            ok = __all_sync(0xffffffffu, bounded_wait(&bars->s_full, it & 1, abort, lim));
-            if (!ok) break;
+            if (!wait_all(&bars->dq_full, it & 1)) return false;
             tc_fence_after();
-            float pr[128];
-            {
-                uint32_t u[32];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    tmem_ld32(tS + c * 32, u);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int x = 0; x < 32; ++x) pr[c * 32 + x] = __uint_as_float(u[x]);
-                }
-            }
-            const bool edge = (p.causal && i == j) || (kidx >= n);
-#pragma unroll
-            for (int c = 0; c < 128; ++c) {
-                float v = ex2_approx(fmaf(pr[c], sl2, -sL[c]));
-                if (edge && (kidx >= n || (p.causal && i * 128 + c < kidx))) v = 0.f;
-                pr[c] = v;
-            }
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t u[32];
-#pragma unroll
-                for (int x = 0; x < 32; ++x) u[x] = pack_bf16x2(pr[h * 64 + 2 * x], pr[h * 64 + 2 * x + 1]);
-                tmem_st32(tS + h * 32, u);
-            }
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&bars->p_full);
-
-            ok = __all_sync(0xffffffffu, bounded_wait(&bars->dp_full, it & 1, abort, lim));
-            if (ok && it > 0) ok = __all_sync(0xffffffffu, bounded_wait(&bars->ds_free, (it - 1) & 1, abort, lim));
-            if (!ok) break;
-            tc_fence_after();
-            uint8_t* ds_row = sdS + r * 128;
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                uint32_t u[32];
-                tmem_ld32(tDP + cc * 32, u);
-                tmem_ld_wait();
-                uint32_t w[16];
-#pragma unroll
-                for (int x = 0; x < 16; ++x) {
-                    const int c0 = cc * 32 + 2 * x;
-                    const float d0 = pr[c0] * (__uint_as_float(u[2 * x]) - sD[c0]);
-                    const float d1 = pr[c0 + 1] * (__uint_as_float(u[2 * x + 1]) - sD[c0 + 1]);
-                    w[x] = pack_bf16x2(d0, d1);
-                }
-                // queries cc*32 .. cc*32+31: chunk cc/2, 16-byte units (cc&1)*4 .. +3, swizzled
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const int unit = (cc & 1) * 4 + t;
-                    uint4* dst = reinterpret_cast<uint4*>(ds_row + (cc >> 1) * 16384 +
-                                                          ((unit ^ (r & 7)) << 4));
-                    *dst = make_uint4(w[4 * t], w[4 * t + 1], w[4 * t + 2], w[4 * t + 3]);
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(&bars->ds_full);
-
-            ok = __all_sync(0xffffffffu, bounded_wait(&bars->dq_full, it & 1, abort, lim));
-            if (!ok) break;
-            tc_fence_after();
-            int* sem = p.deterministic ? p.sems + static_cast<size_t>(bh) * p.nq + i : nullptr;
-            if (sem) {
-                // add this CTA's partial only after every lower key tile has added its own
+            if (p.deterministic) {
+                // add this tile's partial only after every lower key tile has added its own
+                // (each CTA contributes two halves, one per warpgroup)
+                volatile int* sem = p.sems + static_cast<size_t>(bh) * p.nq + i;
+                const int need = 2 * (p.causal ? j : j);
                 bool got = true;
-                if (r == 0) {
+                if (t == 0) {
                     const uint64_t t0 = globaltimer_ns();
-                    while (atomicAdd(sem, 0) != j) {
+                    while (*sem < need) {
                         if (*abort || globaltimer_ns() - t0 > lim) {
                             *abort = 1;
                             report_error(4);
@@ -422,60 +404,150 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     }
                     __threadfence();
                 }
-                compute_bar();
+                wg_bar();
                 if (*abort) got = false;
-                ok = __all_sync(0xffffffffu, got);
-                if (!ok) {
-                    // release dQ's TMEM columns so the MMA warp does not wait for them
+                if (!__all_sync(0xffffffffu, got)) {
                     tc_fence_before();
                     mbar_arrive(&bars->dq_drained);
-                    break;
+                    return false;
                 }
             }
-            float* acc_row = p.dq_acc + (static_cast<size_t>(bh) * p.n_pad + i * 128 + r) * D;
+            float* acc_tile = p.dq_acc + (static_cast<size_t>(bh) * p.n_pad + i * 128) * D;
+            if constexpr (C::DQT) {
+                // lane r = head-dim index; columns = queries cb .. cb+63
+#pragma unroll 1
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t u[32];
+                    tmem_ld32(tDP + cb + c * 32, u);
+                    tmem_ld_wait();
 #pragma unroll
-            for (int cc = 0; cc < D / 32; ++cc) {
-                uint32_t u[32];
-                tmem_ld32(tDP + cc * 32, u);
-                tmem_ld_wait();
+                    for (int x = 0; x < 32; ++x)
+                        red_add_f32(acc_tile + (cb + c * 32 + x) * D + r, __uint_as_float(u[x]));
+                }
+            } else {
+                // lane r = query row; columns = head-dim g*D/2 .. (g+1)*D/2-1
+                float* row = acc_tile + r * D + g * (D / 2);
+                if constexpr (D / 2 == 32) {
+                    uint32_t u[32];
+                    tmem_ld32(tDP + g * 32, u);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int x = 0; x < 8; ++x)
-                    atomicAdd(reinterpret_cast<float4*>(acc_row + cc * 32 + 4 * x),
-                              make_float4(__uint_as_float(u[4 * x]), __uint_as_float(u[4 * x + 1]),
-                                          __uint_as_float(u[4 * x + 2]), __uint_as_float(u[4 * x + 3])));
+                    for (int x = 0; x < 8; ++x)
+                        red_add_v4_f32(row + 4 * x, __uint_as_float(u[4 * x]), __uint_as_float(u[4 * x + 1]),
+                                       __uint_as_float(u[4 * x + 2]), __uint_as_float(u[4 * x + 3]));
+                } else {
+                    uint32_t u[16];
+                    tmem_ld16(tDP + g * 16, u);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int x = 0; x < 4; ++x)
+                        red_add_v4_f32(row + 4 * x, __uint_as_float(u[4 * x]), __uint_as_float(u[4 * x + 1]),
+                                       __uint_as_float(u[4 * x + 2]), __uint_as_float(u[4 * x + 3]));
+                }
             }
             tc_fence_before();
             mbar_arrive(&bars->dq_drained);
-            if (sem) {
+            if (p.deterministic) {
                 __threadfence();
-                compute_bar();
-                if (r == 0) atomicAdd(sem, 1);
+                wg_bar();
+                if (t == 0) atomicAdd(p.sems + static_cast<size_t>(bh) * p.nq + i, 1);
             }
+            return true;
+        };
+
+        for (int it = 0; it < NT; ++it) {
+            const int i = i_begin + it;
+            float* sL = sStat + (g * 2 + (it & 1)) * 128;
+            float* sD = sL + 64;
+            {
+                const int qq = i * 128 + cb + (t & 63);
+                if (t < 64)
+                    sL[t] = (qq < n) ? p.lse[static_cast<size_t>(bh) * n + qq] * kBwdLog2e : INFINITY;
+                else
+                    sD[t - 64] = (qq < n) ? p.Dvec[static_cast<size_t>(bh) * p.n_pad + qq] : 0.f;
+            }
+            wg_bar();
+            // ---- P^T = exp2(S^T·scale·log2e - LSE·log2e), masked; bf16 copy into TMEM
+            if (!(ok = wait_all(&bars->s_full, it & 1))) break;
+            tc_fence_after();
+            const bool edge = (p.causal && i == j) || (kidx >= n);
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t u[32];
+                tmem_ld32(tS + cb + c * 32, u);
+                tmem_ld_wait();
+#pragma unroll
+                for (int x = 0; x < 32; ++x) {
+                    const int col = c * 32 + x;
+                    float v = ex2_approx(fmaf(__uint_as_float(u[x]), sl2, -sL[col]));
+                    if (edge && (kidx >= n || (p.causal && i * 128 + cb + col < kidx))) v = 0.f;
+                    pr[col] = v;
+                }
+            }
+            {
+                uint32_t w[32];
+#pragma unroll
+                for (int x = 0; x < 32; ++x) w[x] = pack_bf16x2(pr[2 * x], pr[2 * x + 1]);
+                tmem_st32(tS + g * 64, w);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&bars->p_full);
+            // ---- drain the previous tile's dQ while the MMAs of this tile run
+            if (it > 0 && !(ok = drain(it - 1))) break;
+            // ---- dS^T = P^T ∘ (dP^T - D) -> bf16 into shared memory (chunk g, swizzled)
+            if (!(ok = wait_all(&bars->dp_full, it & 1))) break;
+            if (it > 0 && !(ok = wait_all(&bars->ds_free, (it - 1) & 1))) break;
+            tc_fence_after();
+            uint8_t* ds_row = sdS + g * 16384 + r * 128;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t u[32];
+                tmem_ld32(tDP + cb + c * 32, u);
+                tmem_ld_wait();
+                uint32_t w[16];
+#pragma unroll
+                for (int x = 0; x < 16; ++x) {
+                    const int c0 = c * 32 + 2 * x;
+                    const float d0 = pr[c0] * (__uint_as_float(u[2 * x]) - sD[c0]);
+                    const float d1 = pr[c0 + 1] * (__uint_as_float(u[2 * x + 1]) - sD[c0 + 1]);
+                    w[x] = pack_bf16x2(d0, d1);
+                }
+#pragma unroll
+                for (int tt = 0; tt < 4; ++tt) {
+                    const int unit = c * 4 + tt;
+                    *reinterpret_cast<uint4*>(ds_row + ((unit ^ (r & 7)) << 4)) =
+                        make_uint4(w[4 * tt], w[4 * tt + 1], w[4 * tt + 2], w[4 * tt + 3]);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bars->ds_full);
         }
-        if (ok) ok = __all_sync(0xffffffffu, bounded_wait(&bars->dkv_done, 0, abort, lim));
+        if (ok && NT > 0) ok = drain(NT - 1);
+        if (ok) ok = wait_all(&bars->dkv_done, 0);
         if (ok) {
             tc_fence_after();
-            const size_t orow = (static_cast<size_t>(bh) * n + kidx) * D;
-#pragma unroll
+            const size_t orow = (static_cast<size_t>(bh) * n + kidx) * D + g * (D / 2);
+#pragma unroll 1
             for (int which = 0; which < 2; ++which) {
-                const uint32_t tacc = tmem + lane_base + (which == 0 ? COL_DV : COL_DK);
+                const uint32_t tacc = tmem + lane_base + (which == 0 ? COL_DV : COL_DK) + g * (D / 2);
                 const float mul = which == 0 ? 1.f : p.scale;
-                __nv_bfloat16* dst = which == 0 ? p.dv : p.dk;
-#pragma unroll
-                for (int cc = 0; cc < D / 32; ++cc) {
-                    uint32_t u[32];
-                    tmem_ld32(tacc + cc * 32, u);
+                __nv_bfloat16* dst = (which == 0 ? p.dv : p.dk) + orow;
+#pragma unroll 1
+                for (int cc = 0; cc < D / 2; cc += 16) {
+                    uint32_t u[16];
+                    tmem_ld16(tacc + cc, u);
                     tmem_ld_wait();
-                    uint32_t w[16];
+                    uint32_t w[8];
 #pragma unroll
-                    for (int x = 0; x < 16; ++x)
+                    for (int x = 0; x < 8; ++x)
                         w[x] = pack_bf16x2(__uint_as_float(u[2 * x]) * mul,
                                            __uint_as_float(u[2 * x + 1]) * mul);
                     if (kidx < n) {
-                        uint4* o = reinterpret_cast<uint4*>(dst + orow + cc * 32);
-#pragma unroll
-                        for (int x = 0; x < 4; ++x)
-                            o[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
+                        uint4* o = reinterpret_cast<uint4*>(dst + cc);
+                        o[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                        o[1] = make_uint4(w[4], w[5], w[6], w[7]);
                     }
                 }
             }
@@ -484,7 +556,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
@@ -498,7 +570,7 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
     const int n_pad = nq * 128;
     cudaError_t e;
     const cudaEvent_t* ev = a.phase_events;
-    if (ev && (e = cudaEventRecord(ev[0], stream)) != cudaSuccess) return e;
+    if (ev && ev[0] && (e = cudaEventRecord(ev[0], stream)) != cudaSuccess) return e;
     // 1. preprocess
     {
         const long long rows = static_cast<long long>(BH) * n_pad;
@@ -539,11 +611,11 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
         kp.timeout_ns = a.timeout_ns;
         const long long grid = static_cast<long long>(nq) * BH;
         if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-        if (ev && (e = cudaEventRecord(ev[1], stream)) != cudaSuccess) return e;
+        if (ev && ev[1] && (e = cudaEventRecord(ev[1], stream)) != cudaSuccess) return e;
         bwd_main_kernel<D><<<static_cast<unsigned>(grid), kBwdThreads, C::SMEM, stream>>>(
             mq, mk, mv, mdo, kp);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        if (ev && (e = cudaEventRecord(ev[2], stream)) != cudaSuccess) return e;
+        if (ev && ev[2] && (e = cudaEventRecord(ev[2], stream)) != cudaSuccess) return e;
     }
     // 3. dQ convert
     {
@@ -553,7 +625,7 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
         bwd_dq_convert_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
             a.dq_acc, static_cast<__nv_bfloat16*>(a.dq), a.n, n_pad, total8, a.scale);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        if (ev && (e = cudaEventRecord(ev[3], stream)) != cudaSuccess) return e;
+        if (ev && ev[3] && (e = cudaEventRecord(ev[3], stream)) != cudaSuccess) return e;
     }
     return cudaSuccess;
 }

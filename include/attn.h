@@ -104,8 +104,8 @@ int attn_selftest_wait_timeout(unsigned timeout_us, void* stream);
  * created by the caller. While set, every attn_bwd call records, on its stream, events[0] before
  * its preprocess kernel (D = rowsum(dO∘O)), events[1] before its main kernel, events[2] after
  * the main kernel and events[3] after the dQ conversion kernel, so that a caller can time the
- * three kernels separately with cudaEventElapsedTime. The array is copied; the events must stay
- * valid while recording is on. Process-wide setting; not meant for concurrent callers. */
+ * three kernels separately with cudaEventElapsedTime. NULL entries are skipped. The array is
+ * copied; the events must stay valid while recording is on. Process-wide setting; not meant for concurrent callers. */
 void attn_set_bwd_phase_events(void* const* events);
 
 /* Static string for an error code. */
