@@ -267,63 +267,69 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
-            // pass 1: row max of this tile (masked), read from TMEM in 32-column chunks
-            const int kbase = jj * C::BN;
-            const bool edge = (p.causal && jj == qt) || kbase + C::BN > n;
-            float mx = -INFINITY;
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                uint32_t u[32];
-                tmem_ld32(tS + c * 32, u);
-                tmem_ld_wait();
+            // S row of this tile: four 32-column loads, one wait
+            uint32_t u[128];
 #pragma unroll
-                for (int x = 0; x < 32; ++x) {
-                    float v = __uint_as_float(u[x]);
-                    const int kidx = kbase + c * 32 + x;
-                    if (edge && (kidx >= n || (p.causal && kidx > qidx))) v = -INFINITY;
-                    mx = fmaxf(mx, v);
+            for (int c = 0; c < 4; ++c)
+                tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[c * 32]));
+            tmem_ld_wait();
+            reg_fence<128>(u);
+            const int kbase = jj * C::BN;
+            if ((p.causal && jj == qt) || kbase + C::BN > n) {
+#pragma unroll
+                for (int c = 0; c < 128; ++c) {
+                    const int kidx = kbase + c;
+                    if (kidx >= n || (p.causal && kidx > qidx)) u[c] = __float_as_uint(-INFINITY);
                 }
             }
-            const float m_new = fmaxf(m, mx * sl2);
-            const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-            const float alpha = ex2_approx(m - m_use);
-            if (jj > 0 && __any_sync(0xffffffffu, m_new != m)) {
+            float mx0 = __uint_as_float(u[0]), mx1 = __uint_as_float(u[1]);
+            float mx2 = __uint_as_float(u[2]), mx3 = __uint_as_float(u[3]);
+#pragma unroll
+            for (int c = 4; c < 128; c += 4) {
+                mx0 = fmaxf(mx0, __uint_as_float(u[c]));
+                mx1 = fmaxf(mx1, __uint_as_float(u[c + 1]));
+                mx2 = fmaxf(mx2, __uint_as_float(u[c + 2]));
+                mx3 = fmaxf(mx3, __uint_as_float(u[c + 3]));
+            }
+            const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+            // Lazy rescaling: the reference max m only moves when the tile max exceeds it by more
+            // than 8 (a factor 2^8 on P); otherwise P = exp2(s·c - m) is simply allowed to exceed
+            // 1. The final O/l and LSE = m + log2 l use the same m, so the result is unchanged.
+            if (jj == 0) {
+                m = m_tile;
+            } else if (__any_sync(0xffffffffu, m_tile > m + 8.f)) {
+                float alpha = 1.f;
+                if (m_tile > m + 8.f) {
+                    alpha = ex2_approx(m - m_tile);
+                    m = m_tile;
+                    l *= alpha;
+                }
 #pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
-                    uint32_t u[32];
-                    tmem_ld32(tO + c * 32, u);
+                    uint32_t o[32];
+                    tmem_ld32(tO + c * 32, o);
                     tmem_ld_wait();
+                    reg_fence<32>(o);
 #pragma unroll
                     for (int x = 0; x < 32; ++x)
-                        u[x] = __float_as_uint(__uint_as_float(u[x]) * alpha);
-                    tmem_st32(tO + c * 32, u);
+                        o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+                    tmem_st32(tO + c * 32, o);
                 }
             }
-            // pass 2: P = exp2(s·scale·log2e - m), row sum, bf16 P written over the S columns
-            // already read (chunk c of S -> packed P columns 16c .. 16c+15)
-            float rs = 0.f;
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                uint32_t u[32];
-                tmem_ld32(tS + c * 32, u);
-                tmem_ld_wait();
-                uint32_t w[16];
+            const float m_use = (m == -INFINITY) ? 0.f : m;
+            float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
-                for (int x = 0; x < 16; ++x) {
-                    float v0 = ex2_approx(fmaf(__uint_as_float(u[2 * x]), sl2, -m_use));
-                    float v1 = ex2_approx(fmaf(__uint_as_float(u[2 * x + 1]), sl2, -m_use));
-                    if (edge) {
-                        const int k0 = kbase + c * 32 + 2 * x;
-                        if (k0 >= n || (p.causal && k0 > qidx)) v0 = 0.f;
-                        if (k0 + 1 >= n || (p.causal && k0 + 1 > qidx)) v1 = 0.f;
-                    }
-                    rs += v0 + v1;
-                    w[x] = pack_bf16x2(v0, v1);
-                }
-                tmem_st16(tS + c * 16, w);
+            for (int c = 0; c < 128; c += 2) {
+                const float p0 = ex2_approx(fmaf(__uint_as_float(u[c]), sl2, -m_use));
+                const float p1 = ex2_approx(fmaf(__uint_as_float(u[c + 1]), sl2, -m_use));
+                rs0 += p0;
+                rs1 += p1;
+                u[c / 2] = pack_bf16x2(p0, p1);
             }
-            l = l * alpha + rs;
-            m = m_new;
+            l += rs0 + rs1;
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+                tmem_st32(tS + h * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[h * 32]));
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&bars->p_full[g]);

@@ -81,9 +81,11 @@ def test_forward_large_magnitude_stays_finite(cuda_device):
         o, lse, _ = cuda_forward(q, k, v, causal, 1 / math.sqrt(128))
         ro, rlse = oracle.fwd(q, k, v, 1 / math.sqrt(128), causal)
         assert torch.isfinite(o).all()
-        # O is within bf16 rounding of the oracle scaled by |v| (up to ~30 here)
-        assert np.abs(to_np(o) - ro).max() <= 30 * TOL_O["bf16"]
-        assert np.abs(to_np(lse) - rlse).max() <= 30 * TOL_LSE["bf16"]
+        # |V| reaches ~120 here, where one bf16 ulp of O is 0.5: the O bound scales with max|V|
+        # (1e-2 of it, about 5x the bf16 rounding of O and P); LSE (~|s| ~ 1e3) relative 1e-5
+        vmax = float(v.float().abs().max())
+        assert np.abs(to_np(o) - ro).max() <= TOL_O["bf16"] * vmax
+        assert np.abs(to_np(lse) - rlse).max() <= 1e-5 * np.abs(rlse).max()
 
 
 def test_forward_repeatable(cuda_device):
