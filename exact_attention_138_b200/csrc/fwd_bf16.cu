@@ -28,6 +28,15 @@ namespace {
 constexpr int kFwdThreads = 384;   // 3 warpgroups
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
+#ifndef ATTN_FWD_EXP_FMA_PER8
+#define ATTN_FWD_EXP_FMA_PER8 0
+#endif
+#ifndef ATTN_FWD_PINGPONG
+#define ATTN_FWD_PINGPONG 0
+#endif
+constexpr int kExpFmaPer8 = ATTN_FWD_EXP_FMA_PER8;   // column pairs (of every 8) whose exp2 runs
+                                                     // on the FMA pipe
+constexpr bool kPingPong = ATTN_FWD_PINGPONG != 0;   // softmax warpgroups take turns
 
 template <int D>
 struct FwdCfg {
@@ -46,7 +55,7 @@ struct FwdCfg {
 struct FwdBars {
     uint64_t q_full;
     uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
-    uint64_t s_full[2], p_full[2], o_done[2];
+    uint64_t s_full[2], p_full[2], o_done[2], sm_done[2];
     uint64_t teardown;
     uint32_t tmem_base;
     int abort;
@@ -112,6 +121,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             mbar_init(&bars->s_full[g], 1);
             mbar_init(&bars->p_full[g], 128);
             mbar_init(&bars->o_done[g], 1);
+            mbar_init(&bars->sm_done[g], 128);
         }
         mbar_init(&bars->teardown, 1);
         bars->abort = ((smem_addr(smem) & 1023u) != 0) ? 1 : 0;
@@ -131,6 +141,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     volatile int* abort = &bars->abort;
     const uint64_t lim = p.timeout_ns;
 
+    if (warp >= 8) {
+    // The producer warpgroup (loader, MMA issuer, two idle warps) hands most of its registers
+    // to the softmax warpgroups: 2·128·208 + 128·80 = 63488 <= 384·168, the launch allocation.
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 80;");
     if (warp == 8) {
         // ---------------------------------------------------------------- TMA producer
         if (lane == 0 && !*abort) {
@@ -187,27 +201,35 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 k_ready = jj;
                 return true;
             };
-            // descriptors are built once per operand tile; a k-step only moves the start
-            // address field (bits [0,14), 16-byte units), which never carries out of the field
-            // because every shared-memory address is below 256 KB.
+            // Lean issue path: descriptors per operand tile computed once, each k-step adds a
+            // constant to the low word, loops fully unrolled. The issuing lane shares its SM
+            // sub-partition with two busy softmax warps, so every instruction here costs.
+            SDesc dQ[2], dK[C::STAGES], dV[C::STAGES];
+#pragma unroll
+            for (int g = 0; g < 2; ++g) dQ[g] = sdesc(sQa + g * C::TILE, 16, 8 * C::SWB, C::SWZ);
+#pragma unroll
+            for (int st = 0; st < C::STAGES; ++st) {
+                dK[st] = sdesc(sKa + st * C::TILE, 16, 8 * C::SWB, C::SWZ);
+                dV[st] = sdesc(sVa + st * C::TILE, C::CHUNK, 8 * C::SWB, C::SWZ);
+            }
             auto issue_s = [&](int g, int jj) {
-                const uint64_t a0 = smem_desc(sQa + g * C::TILE, 16, 8 * C::SWB, C::SWZ);
-                const uint64_t b0 =
-                    smem_desc(sKa + (jj % C::STAGES) * C::TILE, 16, 8 * C::SWB, C::SWZ);
-#pragma unroll 1
+                const SDesc a = dQ[g], b = dK[jj % C::STAGES];
+                const uint32_t d = tmem + 256 + g * 128;
+#pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t off = (((ks * 16) / C::CW) * C::CHUNK + ((ks * 16) % C::CW) * 2) >> 4;
-                    mma_ss(tmem + 256 + g * 128, a0 + off, b0 + off, idS, ks > 0 ? 1u : 0u);
+                    const uint32_t off =
+                        static_cast<uint32_t>((((ks * 16) / C::CW) * C::CHUNK + ((ks * 16) % C::CW) * 2) >> 4);
+                    mma_ss(d, sdesc_at(a, off), sdesc_at(b, off), idS, ks > 0 ? 1u : 0u);
                 }
             };
             auto issue_pv = [&](int g, int jj) {
-                const uint64_t b0 =
-                    smem_desc(sVa + (jj % C::STAGES) * C::TILE, C::CHUNK, 8 * C::SWB, C::SWZ);
-#pragma unroll 1
-                for (int ks = 0; ks < C::BN / 16; ++ks)
-                    mma_ts(tmem + g * 128, tmem + 256 + g * 128 + ks * 8,
-                           b0 + static_cast<uint32_t>((ks * 16 * C::SWB) >> 4), idPV,
-                           (jj > 0 || ks > 0) ? 1u : 0u);
+                const SDesc b = dV[jj % C::STAGES];
+                const uint32_t d = tmem + g * 128, a = tmem + 256 + g * 128;
+                mma_ts(d, a, sdesc_at(b, 0), idPV, jj > 0 ? 1u : 0u);
+#pragma unroll
+                for (int ks = 1; ks < C::BN / 16; ++ks)
+                    mma_ts(d, a + ks * 8, sdesc_at(b, static_cast<uint32_t>((ks * 16 * C::SWB) >> 4)),
+                           idPV, 1u);
             };
             if (ok) ok = wait_k(0);
             if (ok) {
@@ -248,7 +270,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             drain_wait_fwd(&bars->teardown, 0, 100000000ull);
         }
         __syncwarp();
-    } else if (warp < 8) {
+    }
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 208;");
         // ---------------------------------------------------------------- softmax warpgroups
         const int g = warp >> 2;
         const int wq = warp & 3;
@@ -263,7 +287,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         float l = 0.f;         // running sum of exp2(.. - m)
         bool ok = true;
         for (int jj = 0; jj < T[g]; ++jj) {
-            ok = bounded_wait(&bars->s_full[g], jj & 1, abort, lim);
+            // Ping-pong: the two softmax warpgroups take turns (tile 0 of step jj, tile 1 of step
+            // jj, tile 0 of step jj+1, ...), so each has the exp units to itself while the tensor
+            // cores run the other tile's MMAs.
+            ok = true;
+            if (!kPingPong) {
+            } else if (g == 0 && jj > 0 && T[1] > 0)
+                ok = bounded_wait(&bars->sm_done[1], (jj - 1) & 1, abort, lim);
+            else if (g == 1 && jj < T[0])
+                ok = bounded_wait(&bars->sm_done[0], jj & 1, abort, lim);
+            ok = ok && bounded_wait(&bars->s_full[g], jj & 1, abort, lim);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
@@ -275,21 +308,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             tmem_ld_wait();
             reg_fence<128>(u);
             const int kbase = jj * C::BN;
-            if ((p.causal && jj == qt) || kbase + C::BN > n) {
+            const bool edge = (p.causal && jj == qt) || kbase + C::BN > n;
+            if (edge) {
 #pragma unroll
                 for (int c = 0; c < 128; ++c) {
                     const int kidx = kbase + c;
                     if (kidx >= n || (p.causal && kidx > qidx)) u[c] = __float_as_uint(-INFINITY);
                 }
             }
-            float mx0 = __uint_as_float(u[0]), mx1 = __uint_as_float(u[1]);
-            float mx2 = __uint_as_float(u[2]), mx3 = __uint_as_float(u[3]);
+            float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-            for (int c = 4; c < 128; c += 4) {
-                mx0 = fmaxf(mx0, __uint_as_float(u[c]));
-                mx1 = fmaxf(mx1, __uint_as_float(u[c + 1]));
-                mx2 = fmaxf(mx2, __uint_as_float(u[c + 2]));
-                mx3 = fmaxf(mx3, __uint_as_float(u[c + 3]));
+            for (int c = 0; c < 128; c += 8) {
+                mx0 = fmax3(mx0, __uint_as_float(u[c]), __uint_as_float(u[c + 1]));
+                mx1 = fmax3(mx1, __uint_as_float(u[c + 2]), __uint_as_float(u[c + 3]));
+                mx2 = fmax3(mx2, __uint_as_float(u[c + 4]), __uint_as_float(u[c + 5]));
+                mx3 = fmax3(mx3, __uint_as_float(u[c + 6]), __uint_as_float(u[c + 7]));
             }
             const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
             // Lazy rescaling: the reference max m only moves when the tile max exceeds it by more
@@ -317,15 +350,43 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 }
             }
             const float m_use = (m == -INFINITY) ? 0.f : m;
-            float rs0 = 0.f, rs1 = 0.f;
+            const uint64_t sl2x2 = f2_pack(sl2, sl2);
+            const uint64_t nm2 = f2_pack(-m_use, -m_use);
+            uint64_t rsa = f2_pack(0.f, 0.f), rsb = f2_pack(0.f, 0.f);
+            if (edge) {
+                // tiles with masked (-inf) scores: every exponential on the MUFU, exact zeros
 #pragma unroll
-            for (int c = 0; c < 128; c += 2) {
-                const float p0 = ex2_approx(fmaf(__uint_as_float(u[c]), sl2, -m_use));
-                const float p1 = ex2_approx(fmaf(__uint_as_float(u[c + 1]), sl2, -m_use));
-                rs0 += p0;
-                rs1 += p1;
-                u[c / 2] = pack_bf16x2(p0, p1);
+                for (int c = 0; c < 128; c += 2) {
+                    float x0, x1;
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(u[c]), __uint_as_float(u[c + 1])),
+                                     sl2x2, nm2), x0, x1);
+                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                    if (c & 2) rsb = f2_add(rsb, f2_pack(p0, p1));
+                    else rsa = f2_add(rsa, f2_pack(p0, p1));
+                    u[c / 2] = pack_bf16x2(p0, p1);
+                }
+            } else {
+                // kExpFmaPer8 of every 8 column pairs use the FMA-pipe exp2, the rest the MUFU
+#pragma unroll
+                for (int c = 0; c < 128; c += 2) {
+                    float x0, x1, p0, p1;
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(u[c]), __uint_as_float(u[c + 1])),
+                                     sl2x2, nm2), x0, x1);
+                    if (((c / 2) & 7) >= 8 - kExpFmaPer8) {
+                        exp2_fma_x2(x0, x1, p0, p1);
+                    } else {
+                        p0 = ex2_approx(x0);
+                        p1 = ex2_approx(x1);
+                    }
+                    if (c & 2) rsb = f2_add(rsb, f2_pack(p0, p1));
+                    else rsa = f2_add(rsa, f2_pack(p0, p1));
+                    u[c / 2] = pack_bf16x2(p0, p1);
+                }
             }
+            float ra0, ra1, rb0, rb1;
+            f2_unpack(rsa, ra0, ra1);
+            f2_unpack(rsb, rb0, rb1);
+            const float rs0 = ra0 + rb0, rs1 = ra1 + rb1;
             l += rs0 + rs1;
 #pragma unroll
             for (int h = 0; h < 2; ++h)
@@ -333,6 +394,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&bars->p_full[g]);
+            mbar_arrive(&bars->sm_done[g]);
         }
         if (ok && T[g] > 0) {
             ok = bounded_wait(&bars->o_done[g], 0, abort, lim);

@@ -221,6 +221,21 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
     return d;
 }
 
+// The same descriptor split into its two 32-bit words. A k-step only moves the start-address
+// field (low 14 bits of the low word, 16-byte units); shared-memory addresses stay below 256 KB,
+// so the addition never carries into the LBO field and the high word stays fixed.
+struct SDesc {
+    uint32_t lo, hi;
+};
+__device__ __forceinline__ SDesc sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo,
+                                       uint32_t swizzle_code) {
+    const uint64_t d = smem_desc(saddr, lbo, sbo, swizzle_code);
+    return SDesc{static_cast<uint32_t>(d), static_cast<uint32_t>(d >> 32)};
+}
+__device__ __forceinline__ uint64_t sdesc_at(SDesc d, uint32_t off16) {
+    return (static_cast<uint64_t>(d.hi) << 32) | (d.lo + off16);
+}
+
 // Instruction descriptor of tcgen05.mma.kind::f16 with bf16 A/B and fp32 accumulation:
 //   [4,6) D format (1 = f32)   [7,10) A format (1 = bf16)   [10,13) B format (1 = bf16)
 //   [15] A major (0 = K, 1 = MN)   [16] B major   [17,23) N >> 3   [24,29) M >> 4
@@ -280,6 +295,58 @@ __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// ---- packed fp32x2 arithmetic (two lanes of fp32 in one 64-bit register pair) ----
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^x for two values on the FMA pipe (no MUFU). Reduction x = n + f with n = round(x) obtained
+// by adding 1.5·2^23 (the integer lands in the low mantissa bits), f in [-1/2, 1/2]; 2^f from a
+// degree-3 polynomial fitted by the Remez exchange algorithm for minimax relative error
+// (coefficients derived in exp2_poly_fit.py; max relative error 7.5e-5 in fp32), and 2^n applied
+// by adding n to the exponent field with one integer multiply-add on the bit patterns.
+// Inputs are clamped to >= -125 so that the result stays a normal number; the true value there
+// is below 2.4e-38. Used only where no element is masked to -inf.
+__device__ __forceinline__ void exp2_fma_x2(float x0, float x1, float& y0, float& y1) {
+    constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
+    x0 = fmaxf(x0, -125.f);
+    x1 = fmaxf(x1, -125.f);
+    const uint64_t x = f2_pack(x0, x1);
+    const uint64_t j = f2_add(x, f2_pack(kMagic, kMagic));
+    const uint64_t nround = f2_add(j, f2_pack(-kMagic, -kMagic));
+    const uint64_t f = f2_fma(nround, f2_pack(-1.f, -1.f), x);
+    uint64_t p = f2_fma(f2_pack(0.0551716685295105f, 0.0551716685295105f), f,
+                        f2_pack(0.2426111251115799f, 0.2426111251115799f));
+    p = f2_fma(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+    p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+    float p0, p1, j0, j1;
+    f2_unpack(p, p0, p1);
+    f2_unpack(j, j0, j1);
+    // bits(j) = 0x4B400000 + n, so bits(j) * 2^23 == n << 23 (mod 2^32)
+    y0 = __uint_as_float(__float_as_uint(j0) * 8388608u + __float_as_uint(p0));
+    y1 = __uint_as_float(__float_as_uint(j1) * 8388608u + __float_as_uint(p1));
 }
 
 // Two floats -> packed bf16x2 (round to nearest even); `lo` goes to the low 16 bits.
