@@ -271,26 +271,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                              : idesc_bf16_f32(128, D, 1, 1);    // dQ
             const uint32_t aK = smem_addr(sK), aV = smem_addr(sV), aQ = smem_addr(sQ),
                            adO = smem_addr(sdO), adS = smem_addr(sdS);
-            // K-major descriptors of K_j / V_j (S^T, dP^T) and MN-major ones of K_j (dQ)
-            const uint64_t dK_kmaj = smem_desc(aK, 16, 8 * C::SWB, C::SWZ);
-            const uint64_t dV_kmaj = smem_desc(aV, 16, 8 * C::SWB, C::SWZ);
-            const uint64_t dK_mn = smem_desc(aK, C::CHUNK, 8 * C::SWB, C::SWZ);
-            const uint64_t dS_kmaj = smem_desc(adS, 16, 1024, 2u);
-            const uint64_t dS_mn = smem_desc(adS, 16384, 1024, 2u);
-            auto kstep_k = [](int ks) -> uint32_t {     // K-major k-step offset (16-byte units)
+            // Descriptor words of every operand view, built once (the issuing lane shares its SM
+            // sub-partition with busy compute warps: keep the per-MMA instruction count minimal).
+            const SDesc K_k = sdesc(aK, 16, 8 * C::SWB, C::SWZ);          // K_j, K-major
+            const SDesc V_k = sdesc(aV, 16, 8 * C::SWB, C::SWZ);          // V_j, K-major
+            const SDesc K_mn = sdesc(aK, C::CHUNK, 8 * C::SWB, C::SWZ);   // K_j, MN-major
+            const SDesc dS_k = sdesc(adS, 16, 1024, 2u);                  // dS^T, K-major
+            const SDesc dS_mn = sdesc(adS, 16384, 1024, 2u);              // dS^T, MN-major
+            // stage 1 sits TILE bytes after stage 0: its start field is (TILE >> 4) larger
+            const SDesc Q_k = sdesc(aQ, 16, 8 * C::SWB, C::SWZ);
+            const SDesc Q_mn = sdesc(aQ, C::CHUNK, 8 * C::SWB, C::SWZ);
+            const SDesc dO_k = sdesc(adO, 16, 8 * C::SWB, C::SWZ);
+            const SDesc dO_mn = sdesc(adO, C::CHUNK, 8 * C::SWB, C::SWZ);
+            auto stage = [](SDesc d, int st) { return SDesc{d.lo + st * (C::TILE >> 4), d.hi}; };
+            // k-step offsets (16-byte units): K-major over d, MN-major over 16 rows
+            auto koff = [](int ks) -> uint32_t {
                 return static_cast<uint32_t>((((ks * 16) / C::CW) * C::CHUNK + ((ks * 16) % C::CW) * 2) >> 4);
             };
+            auto roff = [](int ks) -> uint32_t { return static_cast<uint32_t>((ks * 16 * C::SWB) >> 4); };
             auto issue_s = [&](int it) {                // S^T = K_j · Q_i^T
-                const uint64_t b0 = smem_desc(aQ + (it & 1) * C::TILE, 16, 8 * C::SWB, C::SWZ);
-#pragma unroll 1
+                const SDesc bq = stage(Q_k, it & 1);
+#pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks)
-                    mma_ss(tmem + COL_S, dK_kmaj + kstep_k(ks), b0 + kstep_k(ks), idSS, ks > 0);
+                    mma_ss(tmem + COL_S, sdesc_at(K_k, koff(ks)), sdesc_at(bq, koff(ks)), idSS,
+                           ks > 0 ? 1u : 0u);
             };
             auto issue_dp = [&](int it) {               // dP^T = V_j · dO_i^T
-                const uint64_t b0 = smem_desc(adO + (it & 1) * C::TILE, 16, 8 * C::SWB, C::SWZ);
-#pragma unroll 1
+                const SDesc bo = stage(dO_k, it & 1);
+#pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks)
-                    mma_ss(tmem + COL_DP, dV_kmaj + kstep_k(ks), b0 + kstep_k(ks), idSS, ks > 0);
+                    mma_ss(tmem + COL_DP, sdesc_at(V_k, koff(ks)), sdesc_at(bo, koff(ks)), idSS,
+                           ks > 0 ? 1u : 0u);
             };
             bool ok = bounded_wait(&bars->kv_full, 0, abort, lim);
             if (ok) ok = bounded_wait(&bars->q_full[0], 0, abort, lim);
@@ -312,12 +323,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 if (!(ok = bounded_wait(&bars->p_full, it & 1, abort, lim))) break;
                 tc_fence_after();
                 {   // dV_j += P^T · dO_i   (P^T in TMEM: queries 0-63 at S+0.., 64-127 at S+64..)
-                    const uint64_t b0 = smem_desc(adO + st * C::TILE, C::CHUNK, 8 * C::SWB, C::SWZ);
-#pragma unroll 1
-                    for (int ks = 0; ks < 8; ++ks)
+                    const SDesc bo = stage(dO_mn, st);
+                    mma_ts(tmem + COL_DV, tmem + COL_S, sdesc_at(bo, 0), idKN, it > 0 ? 1u : 0u);
+#pragma unroll
+                    for (int ks = 1; ks < 8; ++ks)
                         mma_ts(tmem + COL_DV, tmem + COL_S + (ks >> 2) * 64 + (ks & 3) * 8,
-                               b0 + static_cast<uint32_t>((ks * 16 * C::SWB) >> 4), idKN,
-                               (it > 0 || ks > 0) ? 1u : 0u);
+                               sdesc_at(bo, roff(ks)), idKN, 1u);
                 }
                 if (it + 1 < NT) {
                     if (!(ok = bounded_wait(&bars->q_full[(it + 1) & 1], ((it + 1) >> 1) & 1,
@@ -330,19 +341,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 if (!(ok = bounded_wait(&bars->ds_full, it & 1, abort, lim))) break;
                 tc_fence_after();
                 {   // dK_j += dS^T · Q_i   (A = dS^T K-major, B = Q_i MN-major)
-                    const uint64_t b0 = smem_desc(aQ + st * C::TILE, C::CHUNK, 8 * C::SWB, C::SWZ);
-#pragma unroll 1
-                    for (int ks = 0; ks < 8; ++ks)
+                    const SDesc bq = stage(Q_mn, st);
+                    mma_ss(tmem + COL_DK, sdesc_at(dS_k, 0), sdesc_at(bq, 0), idKN, it > 0 ? 1u : 0u);
+#pragma unroll
+                    for (int ks = 1; ks < 8; ++ks)
                         mma_ss(tmem + COL_DK,
-                               dS_kmaj + static_cast<uint32_t>(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4),
-                               b0 + static_cast<uint32_t>((ks * 16 * C::SWB) >> 4), idKN,
-                               (it > 0 || ks > 0) ? 1u : 0u);
+                               sdesc_at(dS_k, static_cast<uint32_t>(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4)),
+                               sdesc_at(bq, roff(ks)), idKN, 1u);
                 }
                 // dQ^T_i = K_j^T · dS^T  (d = 128)   or   dQ_i = dS · K_j   (d < 128)
-#pragma unroll 1
+#pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
-                    const uint64_t kd = dK_mn + static_cast<uint32_t>((ks * 16 * C::SWB) >> 4);
-                    const uint64_t sd = dS_mn + static_cast<uint32_t>((ks * 2048) >> 4);
+                    const uint64_t kd = sdesc_at(K_mn, roff(ks));
+                    const uint64_t sd = sdesc_at(dS_mn, static_cast<uint32_t>((ks * 2048) >> 4));
                     if (C::DQT)
                         mma_ss(tmem + COL_DP, kd, sd, idDQ, ks > 0 ? 1u : 0u);
                     else
