@@ -54,17 +54,20 @@ constexpr size_t kAlign = 256;
 size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct WsLayout {
-    size_t d_off, acc_off, sem_off, total;
+    size_t d_off, l2_off, acc_off, sem_off, total;
 };
 
+// D (fp32) | LSE·log2e (fp32) | dQ accumulator (fp32, d per row) | semaphores (one per 64 rows),
+// every per-row array padded per head to a multiple of 128 rows.
 WsLayout ws_layout(int B, int H, int n, int d, int deterministic) {
     const size_t BH = static_cast<size_t>(B) * H;
     const size_t n_pad = (static_cast<size_t>(n) + 127) / 128 * 128;
     WsLayout w;
     w.d_off = 0;
-    w.acc_off = round_up(BH * n_pad * sizeof(float));
+    w.l2_off = round_up(BH * n_pad * sizeof(float));
+    w.acc_off = w.l2_off + round_up(BH * n_pad * sizeof(float));
     w.sem_off = w.acc_off + round_up(BH * n_pad * d * sizeof(float));
-    w.total = w.sem_off + (deterministic ? round_up(BH * (n_pad / 128) * sizeof(int)) : 0);
+    w.total = w.sem_off + (deterministic ? round_up(BH * (n_pad / 64) * sizeof(int)) : 0);
     return w;
 }
 
@@ -79,7 +82,8 @@ int validate_common(int B, int H, int n, int d, float scale, int dtype) {
 
 }  // namespace
 
-cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int BH, int n, int d) {
+cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int BH, int n, int d,
+                           int box_rows) {
     auto fn = encode_fn();
     if (!fn) return cudaErrorNotSupported;
     const int chunk = d >= 64 ? 64 : d;
@@ -87,7 +91,7 @@ cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int BH, int n, in
                           static_cast<cuuint64_t>(BH)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
                              static_cast<cuuint64_t>(d) * 2 * static_cast<cuuint64_t>(n)};
-    cuuint32_t box[3] = {static_cast<cuuint32_t>(chunk), 128u, 1u};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(chunk), static_cast<cuuint32_t>(box_rows), 1u};
     cuuint32_t estr[3] = {1u, 1u, 1u};
     const CUtensorMapSwizzle swz =
         chunk == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
@@ -174,6 +178,7 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
     a.deterministic = deterministic ? 1 : 0;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     a.Dvec = reinterpret_cast<float*>(ws + w.d_off);
+    a.L2vec = reinterpret_cast<float*>(ws + w.l2_off);
     a.dq_acc = reinterpret_cast<float*>(ws + w.acc_off);
     a.sems = deterministic ? reinterpret_cast<int*>(ws + w.sem_off) : nullptr;
     a.timeout_ns = static_cast<uint64_t>(g_timeout_us.load()) * 1000ull;

@@ -56,6 +56,7 @@ struct BwdBars {
 struct BwdKParams {
     const float* lse;
     const float* Dvec;
+    const float* L2vec;
     float* dq_acc;
     int* sems;
     __nv_bfloat16* dk;
@@ -76,12 +77,14 @@ __device__ __forceinline__ void drain_wait_bwd(uint64_t* bar, uint32_t parity, u
 }
 
 // ------------------------------------------------------------------------------------------
-// Preprocess: D_i = sum_c dO_ic·O_ic (fp32), zero the dQ accumulator rows (padded per head to a
-// multiple of 128) and the semaphores.
+// Preprocess: D_i = sum_c dO_ic·O_ic (fp32) and LSE_i·log2(e), both padded per head to a multiple
+// of 128 rows (0 and +inf on the padding), zero the dQ accumulator rows and the semaphores.
 // ------------------------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ O,
                                                              const __nv_bfloat16* __restrict__ dO,
+                                                             const float* __restrict__ lse,
+                                                             float* __restrict__ L2vec,
                                                              float* __restrict__ Dvec,
                                                              float* __restrict__ dq_acc,
                                                              int* __restrict__ sems, int n,
@@ -123,7 +126,11 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __nv_bfloat16
 #pragma unroll
         for (int off = LPR / 2; off > 0; off >>= 1)
             acc += __shfl_xor_sync(0xffffffffu, acc, off, LPR);
-        if (row < rows && part == 0) Dvec[row] = valid ? acc : 0.f;
+        if (row < rows && part == 0) {
+            Dvec[row] = valid ? acc : 0.f;
+            // LSE in log2 units; +inf on padding rows makes their P exactly 0 downstream
+            L2vec[row] = valid ? lse[src / D] * 1.44269504088896340736f : INFINITY;
+        }
     }
     if (sems) {
         for (long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; t < n_sems;
@@ -573,6 +580,413 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
 }
 
+// ------------------------------------------------------------------------------------------
+// Main backward kernel for d = 128 with 64-row query tiles.
+//
+// Same per-tile mathematics as bwd_main_kernel, arranged so that the dQ partial never blocks the
+// other MMAs: with 64 query rows per tile, TMEM holds
+//     dV [0,128) | dK [128,256) | S^T [256,320) | dP^T [320,384) | dQ^T x2 [384,448),[448,512)
+// so dQ^T is double-buffered in its own columns. Roles (352 threads):
+//   warps 0-3, 4-7  compute warpgroups, query columns 0-31 and 32-63 of each tile; one thread per
+//                   key row (TMEM lane).
+//   warp 8          TMA producer: K_j, V_j once; Q_i, dO_i (64 rows) and the matching 64 values of
+//                   LSE·log2e and D through a 3-deep ring.
+//   warp 9          MMA issuer, per tile:  dP^T(i) -> [P^T(i)] dV += P^T dO -> S^T(i+1) ->
+//                   [dS^T(i)] dK += dS^T Q -> dQ^T(i) = K^T dS^T (into buffer i mod 2).
+//   warp 10         dQ reducer: the compute warps copy dQ^T(i) out of TMEM into a shared-memory
+//                   staging tile laid out like the accumulator rows (64 x 128 fp32, 32 KB
+//                   contiguous in global memory); this warp adds it with one bulk reduction.
+// In the compute loop a tile goes P(i) -> dS(i) -> stage dQ(i-1), so staging overlaps the MMAs.
+// ------------------------------------------------------------------------------------------
+namespace q64 {
+constexpr int kThreads = 352;
+constexpr int BQ = 64;                     // query rows per tile
+constexpr int KTILE = 128 * 128 * 2;       // K_j or V_j: 2 chunks [128 rows][64 d], SW128
+constexpr int QTILE = 64 * 128 * 2;        // Q_i or dO_i: 2 chunks [64 rows][64 d]
+constexpr int QCHUNK = 64 * 128;           // bytes of one [64 rows][64 d] chunk
+constexpr int STAGES = 3;
+constexpr int DS_BYTES = 128 * 64 * 2;     // dS^T [128 keys][64 queries], one SW128 chunk
+constexpr int STG_BYTES = 64 * 128 * 4;    // dQ staging [64 queries][128 d] fp32
+constexpr int OFF_K = 0, OFF_V = KTILE, OFF_Q = 2 * KTILE, OFF_DO = OFF_Q + STAGES * QTILE;
+constexpr int OFF_DS = OFF_DO + STAGES * QTILE, OFF_STG = OFF_DS + DS_BYTES;
+constexpr int OFF_L2 = OFF_STG + STG_BYTES, OFF_DV = OFF_L2 + STAGES * 256;
+constexpr int OFF_BARS = OFF_DV + STAGES * 256;
+constexpr int SMEM = OFF_BARS + 256;
+
+struct Bars {
+    uint64_t kv_full;
+    uint64_t q_full[STAGES], q_empty[STAGES];
+    uint64_t s_full, dp_full, p_full, ds_full, ds_free, dkv_done, teardown;
+    uint64_t dq_full[2], dq_drained[2];
+    uint64_t stg_full, stg_free;
+    uint32_t tmem_base;
+    int abort;
+};
+static_assert(sizeof(Bars) <= 256, "barrier block");
+}  // namespace q64
+
+__global__ void __launch_bounds__(q64::kThreads, 1)
+    bwd_main_q64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                        const BwdKParams p) {
+    using namespace q64;
+    constexpr int D = 128;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t* sK = smem + OFF_K;
+    uint8_t* sV = smem + OFF_V;
+    uint8_t* sQ = smem + OFF_Q;
+    uint8_t* sdO = smem + OFF_DO;
+    uint8_t* sdS = smem + OFF_DS;
+    float* sStg = reinterpret_cast<float*>(smem + OFF_STG);
+    float* sL2 = reinterpret_cast<float*>(smem + OFF_L2);     // [STAGES][64]
+    float* sDv = reinterpret_cast<float*>(smem + OFF_DV);     // [STAGES][64]
+    Bars* bars = reinterpret_cast<Bars*>(smem + OFF_BARS);
+
+    constexpr uint32_t COL_DV = 0, COL_DK = 128, COL_S = 256, COL_DP = 320, COL_DQ = 384;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int L = blockIdx.x;
+    const int j = L / p.BH;                        // key tile (128 keys): small j first
+    const int bh = L % p.BH;
+    const int n = p.n;
+    const int nq = p.n_pad / BQ;                   // 64-row query tiles per head (padded)
+    const int i_begin = p.causal ? 2 * j : 0;
+    const int NT = nq - i_begin;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars->kv_full, 1);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&bars->q_full[s], 1);
+            mbar_init(&bars->q_empty[s], 1);
+        }
+        mbar_init(&bars->s_full, 1);
+        mbar_init(&bars->dp_full, 1);
+        mbar_init(&bars->p_full, 256);
+        mbar_init(&bars->ds_full, 256);
+        mbar_init(&bars->ds_free, 1);
+        mbar_init(&bars->dkv_done, 1);
+        mbar_init(&bars->teardown, 1);
+        for (int b2 = 0; b2 < 2; ++b2) {
+            mbar_init(&bars->dq_full[b2], 1);
+            mbar_init(&bars->dq_drained[b2], 256);
+        }
+        mbar_init(&bars->stg_full, 256);
+        mbar_init(&bars->stg_free, 1);
+        bars->abort = ((smem_addr(smem) & 1023u) != 0) ? 1 : 0;
+        if (bars->abort) report_error(3);
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 9) tmem_alloc(&bars->tmem_base, 512);
+    if (warp == 8 && lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        tma_prefetch_desc(&tmdO);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+    volatile int* abort = &bars->abort;
+    const uint64_t lim = p.timeout_ns;
+
+    if (warp == 8) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0 && !*abort) {
+            mbar_arrive_expect_tx(&bars->kv_full, 2 * KTILE);
+            for (int ch = 0; ch < 2; ++ch) {
+                tma_load_3d(sK + ch * 16384, &tmK, &bars->kv_full, ch * 64, j * 128, bh);
+                tma_load_3d(sV + ch * 16384, &tmV, &bars->kv_full, ch * 64, j * 128, bh);
+            }
+            int issued = 0;
+            for (int it = 0; it < NT; ++it) {
+                const int st = it % STAGES, f = it / STAGES;
+                if (f > 0 && !bounded_wait(&bars->q_empty[st], (f - 1) & 1, abort, lim)) break;
+                const int i = i_begin + it;
+                mbar_arrive_expect_tx(&bars->q_full[st], 2 * QTILE + 2 * 256);
+                for (int ch = 0; ch < 2; ++ch) {
+                    tma_load_3d(sQ + st * QTILE + ch * QCHUNK, &tmQ, &bars->q_full[st], ch * 64,
+                                i * BQ, bh);
+                    tma_load_3d(sdO + st * QTILE + ch * QCHUNK, &tmdO, &bars->q_full[st], ch * 64,
+                                i * BQ, bh);
+                }
+                const size_t row0 = static_cast<size_t>(bh) * p.n_pad + i * BQ;
+                bulk_load(sL2 + st * 64, p.L2vec + row0, 256, &bars->q_full[st]);
+                bulk_load(sDv + st * 64, p.Dvec + row0, 256, &bars->q_full[st]);
+                issued = it + 1;
+            }
+            if (*abort) {
+                drain_wait_bwd(&bars->kv_full, 0, 100000000ull);
+                for (int it = (issued > STAGES ? issued - STAGES : 0); it < issued; ++it)
+                    drain_wait_bwd(&bars->q_full[it % STAGES], (it / STAGES) & 1, 100000000ull);
+            }
+        }
+    } else if (warp == 9) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idS = idesc_bf16_f32(128, 64, 0, 0);      // S^T, dP^T
+            constexpr uint32_t idKV = idesc_bf16_f32(128, 128, 0, 1);    // dV, dK
+            constexpr uint32_t idQ = idesc_bf16_f32(128, 64, 1, 1);      // dQ^T
+            const uint32_t aK = smem_addr(sK), aV = smem_addr(sV), aQ = smem_addr(sQ),
+                           adO = smem_addr(sdO), adS = smem_addr(sdS);
+            const SDesc K_k = sdesc(aK, 16, 1024, 2u), V_k = sdesc(aV, 16, 1024, 2u);
+            const SDesc K_mn = sdesc(aK, 16384, 1024, 2u);
+            const SDesc dS_k = sdesc(adS, 16, 1024, 2u), dS_mn = sdesc(adS, 16384, 1024, 2u);
+            const SDesc Q_k = sdesc(aQ, 16, 1024, 2u), Q_mn = sdesc(aQ, QCHUNK, 1024, 2u);
+            const SDesc dO_k = sdesc(adO, 16, 1024, 2u), dO_mn = sdesc(adO, QCHUNK, 1024, 2u);
+            auto stage = [](SDesc d, int st) { return SDesc{d.lo + st * (QTILE >> 4), d.hi}; };
+            // k-step offsets over d: operand with 128 rows (16 KB chunks) / 64 rows (8 KB chunks)
+            auto k128 = [](int ks) -> uint32_t { return static_cast<uint32_t>(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4); };
+            auto k64 = [](int ks) -> uint32_t { return static_cast<uint32_t>(((ks >> 2) * QCHUNK + (ks & 3) * 32) >> 4); };
+            auto issue_s = [&](int it) {
+                const SDesc bq = stage(Q_k, it % STAGES);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_ss(tmem + COL_S, sdesc_at(K_k, k128(ks)), sdesc_at(bq, k64(ks)), idS, ks > 0 ? 1u : 0u);
+            };
+            auto issue_dp = [&](int it) {
+                const SDesc bo = stage(dO_k, it % STAGES);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_ss(tmem + COL_DP, sdesc_at(V_k, k128(ks)), sdesc_at(bo, k64(ks)), idS, ks > 0 ? 1u : 0u);
+            };
+            bool ok = bounded_wait(&bars->kv_full, 0, abort, lim);
+            if (ok) ok = bounded_wait(&bars->q_full[0], 0, abort, lim);
+            tc_fence_after();
+            if (ok) {
+                issue_s(0);
+                mma_commit(&bars->s_full);
+            }
+            for (int it = 0; ok && it < NT; ++it) {
+                const int st = it % STAGES;
+                // dP^T(i): its columns were last read for dS^T(i-1), which ds_full(i-1) covered
+                issue_dp(it);
+                mma_commit(&bars->dp_full);
+                if (!(ok = bounded_wait(&bars->p_full, it & 1, abort, lim))) break;
+                tc_fence_after();
+                {   // dV += P^T · dO  (P^T: queries 0-31 at S+0.., 32-63 at S+32..)
+                    const SDesc bo = stage(dO_mn, st);
+                    mma_ts(tmem + COL_DV, tmem + COL_S, sdesc_at(bo, 0), idKV, it > 0 ? 1u : 0u);
+#pragma unroll
+                    for (int ks = 1; ks < 4; ++ks)
+                        mma_ts(tmem + COL_DV, tmem + COL_S + (ks >> 1) * 32 + (ks & 1) * 8,
+                               sdesc_at(bo, static_cast<uint32_t>((ks * 2048) >> 4)), idKV, 1u);
+                }
+                if (it + 1 < NT) {
+                    const int st1 = (it + 1) % STAGES;
+                    if (!(ok = bounded_wait(&bars->q_full[st1], ((it + 1) / STAGES) & 1, abort, lim))) break;
+                    tc_fence_after();
+                    issue_s(it + 1);
+                    mma_commit(&bars->s_full);
+                }
+                if (!(ok = bounded_wait(&bars->ds_full, it & 1, abort, lim))) break;
+                tc_fence_after();
+                {   // dK += dS^T · Q
+                    const SDesc bq = stage(Q_mn, st);
+                    mma_ss(tmem + COL_DK, sdesc_at(dS_k, 0), sdesc_at(bq, 0), idKV, it > 0 ? 1u : 0u);
+#pragma unroll
+                    for (int ks = 1; ks < 4; ++ks)
+                        mma_ss(tmem + COL_DK, sdesc_at(dS_k, static_cast<uint32_t>((ks * 32) >> 4)),
+                               sdesc_at(bq, static_cast<uint32_t>((ks * 2048) >> 4)), idKV, 1u);
+                }
+                const int b2 = it & 1;
+                if (it >= 2) {
+                    if (!(ok = bounded_wait(&bars->dq_drained[b2], ((it - 2) >> 1) & 1, abort, lim))) break;
+                    tc_fence_after();
+                }
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)      // dQ^T = K^T · dS^T  (M = d, N = 64 queries)
+                    mma_ss(tmem + COL_DQ + b2 * 64, sdesc_at(K_mn, static_cast<uint32_t>((ks * 2048) >> 4)),
+                           sdesc_at(dS_mn, static_cast<uint32_t>((ks * 2048) >> 4)), idQ, ks > 0 ? 1u : 0u);
+                mma_commit(&bars->dq_full[b2]);
+                mma_commit(&bars->ds_free);
+                mma_commit(&bars->q_empty[st]);
+            }
+            if (ok) mma_commit(&bars->dkv_done);
+            mma_commit(&bars->teardown);
+            drain_wait_bwd(&bars->teardown, 0, 100000000ull);
+        }
+        __syncwarp();
+    } else if (warp == 10) {
+        // ---------------------------------------------------------------- dQ reducer
+        if (lane == 0) {
+            for (int it = 0; it < NT; ++it) {
+                if (!bounded_wait(&bars->stg_full, it & 1, abort, lim)) break;
+                const int i = i_begin + it;
+                float* dst = p.dq_acc + (static_cast<size_t>(bh) * p.n_pad + i * BQ) * D;
+                volatile int* sem = p.deterministic ? p.sems + static_cast<size_t>(bh) * nq + i : nullptr;
+                if (sem) {
+                    // contributions to one query tile are added in increasing key-tile order
+                    const uint64_t t0 = globaltimer_ns();
+                    bool got = true;
+                    while (*sem < j) {
+                        if (*abort || globaltimer_ns() - t0 > lim) {
+                            *abort = 1;
+                            report_error(4);
+                            got = false;
+                            break;
+                        }
+                        __nanosleep(64);
+                    }
+                    if (!got) break;
+                    __threadfence();
+                }
+                bulk_reduce_add_f32(dst, sStg, STG_BYTES);
+                bulk_commit();
+                if (sem) {
+                    bulk_wait_all();                 // the adds are done, not only the reads
+                    __threadfence();
+                    atomicAdd(const_cast<int*>(sem), 1);
+                } else {
+                    bulk_wait_read_all();            // staging may be overwritten
+                }
+                mbar_arrive(&bars->stg_free);
+            }
+            bulk_wait_all();
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------------- compute warpgroups
+        const int g = warp >> 2;                           // query columns 32g .. 32g+31
+        const int r = (warp & 3) * 32 + lane;              // key row = TMEM lane
+        const int kidx = j * 128 + r;
+        const int cb = g * 32;
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const float sl2 = p.scale_log2;
+        auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
+            return __all_sync(0xffffffffu, bounded_wait(bar, par, abort, lim));
+        };
+        float pr[32];
+        bool ok = true;
+
+        // dQ^T(it) (lane = head-dim index r, columns = queries) -> staging [query][d]
+        auto stage_dq = [&](int it) -> bool {
+            const int b2 = it & 1;
+            if (!wait_all(&bars->dq_full[b2], (it >> 1) & 1)) return false;
+            if (it > 0 && !wait_all(&bars->stg_free, (it - 1) & 1)) return false;
+            tc_fence_after();
+            uint32_t u[32];
+            tmem_ld32(tmem + lane_base + COL_DQ + b2 * 64 + cb, u);
+            tmem_ld_wait();
+            reg_fence<32>(u);
+            tc_fence_before();
+            mbar_arrive(&bars->dq_drained[b2]);
+#pragma unroll
+            for (int x = 0; x < 32; ++x) sStg[(cb + x) * D + r] = __uint_as_float(u[x]);
+            fence_proxy_async_smem();
+            mbar_arrive(&bars->stg_full);
+            return true;
+        };
+
+        for (int it = 0; it < NT; ++it) {
+            const int i = i_begin + it;
+            const int st = it % STAGES;
+            const float* L2 = sL2 + st * 64 + cb;
+            const float* Dv = sDv + st * 64 + cb;
+            // ---- P^T = exp2(S^T·scale·log2e - LSE·log2e), masked; bf16 into TMEM over S^T
+            if (!(ok = wait_all(&bars->s_full, it & 1))) break;
+            tc_fence_after();
+            {
+                uint32_t u[32];
+                tmem_ld32(tmem + lane_base + COL_S + cb, u);
+                tmem_ld_wait();
+                reg_fence<32>(u);
+                const bool edge = (p.causal && i * BQ < (j + 1) * 128) || (kidx >= n);
+#pragma unroll
+                for (int x = 0; x < 32; x += 4) {
+                    const float4 l4 = *reinterpret_cast<const float4*>(L2 + x);
+                    pr[x] = ex2_approx(fmaf(__uint_as_float(u[x]), sl2, -l4.x));
+                    pr[x + 1] = ex2_approx(fmaf(__uint_as_float(u[x + 1]), sl2, -l4.y));
+                    pr[x + 2] = ex2_approx(fmaf(__uint_as_float(u[x + 2]), sl2, -l4.z));
+                    pr[x + 3] = ex2_approx(fmaf(__uint_as_float(u[x + 3]), sl2, -l4.w));
+                }
+                if (edge) {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x)
+                        if (kidx >= n || (p.causal && i * BQ + cb + x < kidx)) pr[x] = 0.f;
+                }
+                uint32_t w[16];
+#pragma unroll
+                for (int x = 0; x < 16; ++x) w[x] = pack_bf16x2(pr[2 * x], pr[2 * x + 1]);
+                tmem_st16(tmem + lane_base + COL_S + cb, w);
+                tmem_st_wait();
+            }
+            tc_fence_before();
+            mbar_arrive(&bars->p_full);
+            // ---- dS^T = P^T ∘ (dP^T - D) -> bf16 into shared memory (row r, swizzled)
+            if (!(ok = wait_all(&bars->dp_full, it & 1))) break;
+            if (it > 0 && !(ok = wait_all(&bars->ds_free, (it - 1) & 1))) break;
+            tc_fence_after();
+            {
+                uint32_t u[32];
+                tmem_ld32(tmem + lane_base + COL_DP + cb, u);
+                tmem_ld_wait();
+                reg_fence<32>(u);
+                uint32_t w[16];
+#pragma unroll
+                for (int x = 0; x < 16; x += 2) {
+                    const float4 d4 = *reinterpret_cast<const float4*>(Dv + 2 * x);
+                    w[x] = pack_bf16x2(pr[2 * x] * (__uint_as_float(u[2 * x]) - d4.x),
+                                       pr[2 * x + 1] * (__uint_as_float(u[2 * x + 1]) - d4.y));
+                    w[x + 1] = pack_bf16x2(pr[2 * x + 2] * (__uint_as_float(u[2 * x + 2]) - d4.z),
+                                           pr[2 * x + 3] * (__uint_as_float(u[2 * x + 3]) - d4.w));
+                }
+                uint8_t* ds_row = sdS + r * 128;
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const int unit = g * 4 + t;
+                    *reinterpret_cast<uint4*>(ds_row + ((unit ^ (r & 7)) << 4)) =
+                        make_uint4(w[4 * t], w[4 * t + 1], w[4 * t + 2], w[4 * t + 3]);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bars->ds_full);
+            // ---- the previous tile's dQ^T into the staging tile, while this tile's MMAs run
+            if (it > 0 && !(ok = stage_dq(it - 1))) break;
+        }
+        if (ok && NT > 0) ok = stage_dq(NT - 1);
+        if (ok) ok = wait_all(&bars->dkv_done, 0);
+        if (ok) {
+            tc_fence_after();
+            const size_t orow = (static_cast<size_t>(bh) * n + kidx) * D + g * 64;
+#pragma unroll 1
+            for (int which = 0; which < 2; ++which) {
+                const uint32_t tacc = tmem + lane_base + (which == 0 ? COL_DV : COL_DK) + g * 64;
+                const float mul = which == 0 ? 1.f : p.scale;
+                __nv_bfloat16* dst = (which == 0 ? p.dv : p.dk) + orow;
+#pragma unroll 1
+                for (int cc = 0; cc < 64; cc += 32) {
+                    uint32_t u[32];
+                    tmem_ld32(tacc + cc, u);
+                    tmem_ld_wait();
+                    reg_fence<32>(u);
+                    uint32_t w[16];
+#pragma unroll
+                    for (int x = 0; x < 16; ++x)
+                        w[x] = pack_bf16x2(__uint_as_float(u[2 * x]) * mul,
+                                           __uint_as_float(u[2 * x + 1]) * mul);
+                    if (kidx < n) {
+                        uint4* o = reinterpret_cast<uint4*>(dst + cc);
+#pragma unroll
+                        for (int x = 0; x < 4; ++x)
+                            o[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
 template <int D>
 cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
     using C = BwdCfg<D>;
@@ -588,14 +1002,48 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
         const int rpw = 32 / (D / 8);
         long long blocks = (rows + (8 * rpw) - 1) / (8 * rpw);
         if (blocks > 148 * 16) blocks = 148 * 16;
-        const int n_sems = a.deterministic ? BH * nq : 0;
+        const int n_sems = a.deterministic ? BH * (n_pad / 64) : 0;
         bwd_preprocess_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-            static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dO),
-            a.Dvec, a.dq_acc, a.deterministic ? a.sems : nullptr, a.n, n_pad, rows, n_sems);
+            static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dO), a.lse,
+            a.L2vec, a.Dvec, a.dq_acc, a.deterministic ? a.sems : nullptr, a.n, n_pad, rows,
+            n_sems);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     // 2. main
-    {
+    if constexpr (D == 128) {
+        CUtensorMap mq, mk, mv, mdo;
+        if ((e = make_tmap_bf16(&mq, a.q, BH, a.n, D, q64::BQ)) != cudaSuccess) return e;
+        if ((e = make_tmap_bf16(&mk, a.k, BH, a.n, D)) != cudaSuccess) return e;
+        if ((e = make_tmap_bf16(&mv, a.v, BH, a.n, D)) != cudaSuccess) return e;
+        if ((e = make_tmap_bf16(&mdo, a.dO, BH, a.n, D, q64::BQ)) != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(bwd_main_q64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 q64::SMEM);
+        if (e != cudaSuccess) return e;
+        BwdKParams kp;
+        kp.lse = a.lse;
+        kp.Dvec = a.Dvec;
+        kp.L2vec = a.L2vec;
+        kp.dq_acc = a.dq_acc;
+        kp.sems = a.sems;
+        kp.dk = static_cast<__nv_bfloat16*>(a.dk);
+        kp.dv = static_cast<__nv_bfloat16*>(a.dv);
+        kp.n = a.n;
+        kp.n_pad = n_pad;
+        kp.BH = BH;
+        kp.nq = nq;
+        kp.causal = a.causal;
+        kp.deterministic = a.deterministic;
+        kp.scale = a.scale;
+        kp.scale_log2 = a.scale * kBwdLog2e;
+        kp.timeout_ns = a.timeout_ns;
+        const long long grid = static_cast<long long>(nq) * BH;
+        if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+        if (ev && ev[1] && (e = cudaEventRecord(ev[1], stream)) != cudaSuccess) return e;
+        bwd_main_q64_kernel<<<static_cast<unsigned>(grid), q64::kThreads, q64::SMEM, stream>>>(
+            mq, mk, mv, mdo, kp);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if (ev && ev[2] && (e = cudaEventRecord(ev[2], stream)) != cudaSuccess) return e;
+    } else {
         CUtensorMap mq, mk, mv, mdo;
         if ((e = make_tmap_bf16(&mq, a.q, BH, a.n, D)) != cudaSuccess) return e;
         if ((e = make_tmap_bf16(&mk, a.k, BH, a.n, D)) != cudaSuccess) return e;
@@ -607,6 +1055,7 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
         BwdKParams kp;
         kp.lse = a.lse;
         kp.Dvec = a.Dvec;
+        kp.L2vec = a.L2vec;
         kp.dq_acc = a.dq_acc;
         kp.sems = a.sems;
         kp.dk = static_cast<__nv_bfloat16*>(a.dk);

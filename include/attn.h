@@ -68,9 +68,10 @@ int attn_version(void);
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              int B, int H, int n, int d, float scale, int causal, int dtype, void* stream);
 
-/* Bytes of device workspace attn_bwd needs for these sizes: the D vector (B·H·n fp32, padded per
- * head to a multiple of 128 rows) and the fp32 dQ accumulator (B·H·n·d fp32, padded the same
- * way), each rounded up to 256 bytes; with deterministic != 0 also one semaphore per query tile. */
+/* Bytes of device workspace attn_bwd needs for these sizes: the D vector and the LSE·log2(e)
+ * vector (B·H·n fp32 each, padded per head to a multiple of 128 rows) and the fp32 dQ accumulator
+ * (B·H·n·d fp32, padded the same way), each rounded up to 256 bytes; with deterministic != 0 also
+ * one int semaphore per 64 query rows. */
 size_t attn_bwd_workspace_bytes(int B, int H, int n, int d, int deterministic);
 
 /* Backward pass (bf16 only). Inputs q, k, v, o, dO (bf16) and lse (fp32, from attn_fwd with the

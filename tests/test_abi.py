@@ -27,11 +27,11 @@ def test_version_and_error_strings():
 
 
 def test_workspace_size_formula():
-    # D (fp32, per-head rows padded to 128) + dQ accumulator (fp32, same rows x d), 256-aligned
+    # D and LSE·log2e (fp32, per-head rows padded to 128) + dQ accumulator (fp32, same rows x d)
     n_pad = 256
-    want = 2 * 3 * n_pad * 4 + 2 * 3 * n_pad * 64 * 4
+    want = 2 * (2 * 3 * n_pad * 4) + 2 * 3 * n_pad * 64 * 4
     assert ea.attn_bwd_workspace_bytes(2, 3, 200, 64, 0) == want
-    assert ea.attn_bwd_workspace_bytes(2, 3, 200, 64, 1) == want + 256   # 6 semaphores -> 256 B
+    assert ea.attn_bwd_workspace_bytes(2, 3, 200, 64, 1) == want + 256   # 24 semaphores -> 256 B
     assert ea.attn_bwd_workspace_bytes(0, 3, 200, 64, 0) == 0
 
 
