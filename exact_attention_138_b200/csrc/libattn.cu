@@ -4,3 +4,4 @@
 #include "fwd_bf16.cu"
 #include "fwd_f32.cu"
 #include "bwd_bf16.cu"
+#include "bwd_noalloc.cu"

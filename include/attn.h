@@ -86,6 +86,23 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
              int B, int H, int n, int d, float scale, int causal, int dtype, int deterministic,
              void* workspace, size_t ws_bytes, void* stream);
 
+/* Backward pass without a caller workspace, for callers that cannot allocate device memory where
+ * they run it (e.g. code inside a host framework that owns all device allocations, or a loop that
+ * must not call cudaMalloc). The pages have no counterpart to this entry point.
+ * Same arguments, validation, kernels and results as attn_bwd, except that the scratch memory is a
+ * fixed 32 MiB device array owned by the library: it is reserved on every GPU where the library's
+ * device code is loaded, until the process exits, and nothing is allocated or freed per call.
+ * Returns ATTN_ERR_WORKSPACE, launching nothing, when attn_bwd_workspace_bytes(B, H, n, d,
+ * deterministic) exceeds 32 MiB (33,554,432 bytes). All calls on a device share the array and
+ * leave their contents in it; each call rewrites or zeroes what it reads, but calls whose kernels
+ * overlap on the GPU (unordered streams, concurrent host threads) race and give wrong results.
+ * The first call on each device looks up the array's device address (cudaGetSymbolAddress, with
+ * that device current): make that first call before any stream capture. */
+int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                     const float* lse, void* dq, void* dk, void* dv,
+                     int B, int H, int n, int d, float scale, int causal, int dtype,
+                     int deterministic, void* stream);
+
 /* Synchronises `stream`, then returns and clears the sticky device status word: ATTN_OK, or
  * ATTN_ERR_TIMEOUT if a kernel's bounded wait expired since the last call, or ATTN_ERR_CUDA if
  * the synchronisation itself failed. */
