@@ -59,9 +59,9 @@ def csrc_digest():
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, if the kernel sources
-    have not changed since the counters were taken; else None."""
+def recorded_traffic(kernel, workload):
+    """DRAM bytes (read + write) per launch of `kernel` on `workload` from the committed ncu
+    summary, if the kernel sources have not changed since the counters were taken; else None."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(path) as f:
@@ -69,7 +69,7 @@ def recorded_traffic(kernel):
     except (OSError, ValueError):
         return None
     entry = rec.get(kernel)
-    if not entry or entry.get("csrc_sha") != csrc_digest():
+    if not entry or entry.get("csrc_sha") != csrc_digest() or entry.get("workload") != workload:
         return None
     return entry.get("bytes_per_launch")
 
@@ -139,26 +139,27 @@ class ClockSampler:
 
 def oracle_sample(seconds_target, q, k, v, do, w, rng_seed=9):
     """Time the fp64 oracle on a bounded sample of the workload's query rows: forward rows
-    (O, LSE) and backward dQ rows. Returns (TFLOPS credited, seconds, rows, threads)."""
+    (O, LSE) and backward dQ rows, in batches of uniformly drawn rows until about
+    `seconds_target` seconds have been spent. Returns (TFLOPS credited, seconds, rows, threads);
+    each row is credited with the workload's average algorithmic FLOPs per query row."""
     import numpy as np
     import oracle
     B, H, n, d = w.B, w.H, w.n, w.d
     total_rows = B * H * n
     fwd, bwd = step_flops(B, H, n, d)
-    per_row = (fwd + bwd) / total_rows            # average algorithmic FLOPs of one query row
+    per_row = (fwd + bwd) / total_rows
     rng = np.random.default_rng(rng_seed)
-    probe = np.sort(rng.choice(total_rows, size=8, replace=False))
-    t0 = time.perf_counter()
-    oracle.fwd_rows(q, k, v, w.scale, True, probe)
-    oracle.bwd_query_rows(q, k, v, do, w.scale, True, probe)
-    t_probe = max(time.perf_counter() - t0, 1e-3)
-    rows_n = int(max(8, min(4096, seconds_target / t_probe * len(probe))))
-    rows = np.sort(rng.choice(total_rows, size=rows_n, replace=False))
-    t0 = time.perf_counter()
-    oracle.fwd_rows(q, k, v, w.scale, True, rows)
-    oracle.bwd_query_rows(q, k, v, do, w.scale, True, rows)
-    dt = time.perf_counter() - t0
-    return per_row * rows_n / dt / 1e12, dt, rows_n, oracle.num_threads()
+    qf, kf, vf, dof = (oracle._f32(t) for t in (q, k, v, do))   # widen once, outside the timing
+    rows_done, spent, batch = 0, 0.0, 64
+    while spent < seconds_target:
+        rows = np.sort(rng.choice(total_rows, size=batch, replace=False))
+        t0 = time.perf_counter()
+        oracle.fwd_rows(qf, kf, vf, w.scale, True, rows)
+        oracle.bwd_query_rows(qf, kf, vf, dof, w.scale, True, rows)
+        spent += time.perf_counter() - t0
+        rows_done += batch
+        batch = min(batch * 2, 2048)
+    return per_row * rows_done / spent / 1e12, spent, rows_done, oracle.num_threads()
 
 
 def run_reference(args, w):
@@ -200,7 +201,7 @@ def run_reference(args, w):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
@@ -344,7 +345,8 @@ def main():
     e2e_value = world * (fwd_flops + bwd_flops) / (e2e_ms * 1e-3) / 1e12
 
     clk = clocks.summary()
-    traffic = recorded_traffic("bwd_main_kernel")
+    main_kernel = "bwd_main_q64_kernel" if w.d == 128 else "bwd_main_kernel"
+    traffic = recorded_traffic(main_kernel, w.name)
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -362,7 +364,7 @@ def main():
                 "preprocess_ms": statistics.mean(pre_ms), "main_ms": statistics.mean(main_ms),
                 "dq_convert_ms": statistics.mean(conv_ms)},
         "pct_of_burst_peak": 100 * (value / world) / burst,
-        "roofline": {"kernel": "bwd_main_kernel", "bound": "tensor", "achieved": main_tf,
+        "roofline": {"kernel": main_kernel, "bound": "tensor", "achieved": main_tf,
                      "peak": sustained, "unit": "TFLOP/s", "frac": main_tf / sustained,
                      "peak_kind": f"bf16_tflops_sustained ({peak_src})",
                      "traffic": traffic},

@@ -61,7 +61,7 @@ struct BwdKParams {
     int* sems;
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
-    int n, n_pad, BH, nq, causal, deterministic;
+    int n, n_pad, BH, nq, causal, deterministic, group;
     float scale, scale_log2;
     uint64_t timeout_ns;
 };
@@ -200,9 +200,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    // Heads in groups of p.group (a group's Q, dO, K, V and dQ rows stay in L2); within a group,
+    // key tiles go from small j (most causal work) to large j across the group's heads.
     const int L = blockIdx.x;
-    const int j = L / p.BH;                        // key tile: small j (most work) first
-    const int bh = L % p.BH;
+    const int gbase = (L / (p.group * p.nq)) * p.group;
+    const int gsize = min(p.group, p.BH - gbase);
+    const int r_in = L - gbase * p.nq;
+    const int j = r_in / gsize;
+    const int bh = gbase + r_in % gsize;
     const int n = p.n;
     const int i_begin = p.causal ? j : 0;
     const int NT = p.nq - i_begin;
@@ -646,9 +651,13 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    // Heads in groups of p.group (see bwd_main_kernel); key tiles of 128 keys, small j first.
     const int L = blockIdx.x;
-    const int j = L / p.BH;                        // key tile (128 keys): small j first
-    const int bh = L % p.BH;
+    const int gbase = (L / (p.group * p.nq)) * p.group;
+    const int gsize = min(p.group, p.BH - gbase);
+    const int r_in = L - gbase * p.nq;
+    const int j = r_in / gsize;
+    const int bh = gbase + r_in % gsize;
     const int n = p.n;
     const int nq = p.n_pad / BQ;                   // 64-row query tiles per head (padded)
     const int i_begin = p.causal ? 2 * j : 0;
@@ -993,6 +1002,14 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
     const int BH = a.B * a.H;
     const int nq = (a.n + 127) / 128;
     const int n_pad = nq * 128;
+    // heads per group: Q, dO, K, V (bf16) and the fp32 dQ rows of one head take (8 + 4)·n·d
+    // bytes; keep a group's within ~48 MB of L2
+    int group;
+    {
+        const long long per_head = 12LL * n_pad * D;
+        long long g = (48LL << 20) / (per_head > 0 ? per_head : 1);
+        group = static_cast<int>(g < 1 ? 1 : (g > BH ? BH : g));
+    }
     cudaError_t e;
     const cudaEvent_t* ev = a.phase_events;
     if (ev && ev[0] && (e = cudaEventRecord(ev[0], stream)) != cudaSuccess) return e;
@@ -1033,6 +1050,7 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
         kp.nq = nq;
         kp.causal = a.causal;
         kp.deterministic = a.deterministic;
+        kp.group = group;
         kp.scale = a.scale;
         kp.scale_log2 = a.scale * kBwdLog2e;
         kp.timeout_ns = a.timeout_ns;
@@ -1066,6 +1084,7 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
         kp.nq = nq;
         kp.causal = a.causal;
         kp.deterministic = a.deterministic;
+        kp.group = group;
         kp.scale = a.scale;
         kp.scale_log2 = a.scale * kBwdLog2e;
         kp.timeout_ns = a.timeout_ns;

@@ -64,7 +64,7 @@ struct FwdBars {
 struct FwdKParams {
     void* o;
     float* lse;
-    int n, BH, n_pairs, causal;
+    int n, BH, n_pairs, causal, group;
     float scale_log2;
     uint64_t timeout_ns;
 };
@@ -95,9 +95,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    // Heads are processed in groups of p.group (sized so that a group's K and V stay in L2);
+    // within a group, tile pairs go longest-first (causal) across the group's heads.
     const int L = blockIdx.x;
-    const int pair = p.n_pairs - 1 - L / p.BH;           // longest causal rows first
-    const int bh = L % p.BH;
+    const int gbase = (L / (p.group * p.n_pairs)) * p.group;
+    const int gsize = min(p.group, p.BH - gbase);
+    const int r_in = L - gbase * p.n_pairs;
+    const int pair = p.n_pairs - 1 - r_in / gsize;
+    const int bh = gbase + r_in % gsize;
     const int n = p.n;
     const int n_kv = (n + C::BN - 1) / C::BN;
     int T[2];
@@ -455,6 +460,12 @@ cudaError_t launch_fwd_bf16_d(const FwdArgs& a, cudaStream_t stream) {
     const int nq = (a.n + 127) / 128;
     kp.n_pairs = (nq + 1) / 2;
     kp.causal = a.causal;
+    // heads per group: K and V of one head take 4·n·d bytes; keep a group's within ~32 MB of L2
+    {
+        const long long per_head = 4LL * a.n * D;
+        long long g = (32LL << 20) / (per_head > 0 ? per_head : 1);
+        kp.group = static_cast<int>(g < 1 ? 1 : (g > BH ? BH : g));
+    }
     kp.scale_log2 = a.scale * kLog2e;
     kp.timeout_ns = a.timeout_ns;
     const long long grid = static_cast<long long>(kp.n_pairs) * BH;
