@@ -39,6 +39,27 @@ def step_flops(B, H, n, d, causal=True):
     return fwd, 2.5 * fwd
 
 
+def rank_seed(rank):
+    """Each rank draws its own batch: seed 9 + rank (rank 0 reproduces the single-GPU inputs)."""
+    return 9 + rank
+
+
+def max_over_ranks(value, dist=None, device="cpu"):
+    """Max of a per-rank scalar over all ranks (identity without a process group)."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.item()
+
+
+def whole_job_tflops(flops_per_rank, world, ms_per_step):
+    """Weak scaling: every rank processes its own batch; the job's rate is all ranks' FLOPs over
+    the slowest rank's time."""
+    return world * flops_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -240,8 +261,7 @@ def main():
     import exact_attention_138_b200 as ea
 
     # --- inputs: each rank draws its own batch (seed 9 + rank), rounded to bf16 on the host
-    q_h, k_h, v_h, do_h = attn_inputs.bf16_draws(w.shape, factor=w.factor,
-                                                 seed=attn_inputs.SEED + rank)
+    q_h, k_h, v_h, do_h = attn_inputs.bf16_draws(w.shape, factor=w.factor, seed=rank_seed(rank))
     q, k, v, do = (t.to(dev) for t in (q_h, k_h, v_h, do_h))
     o = torch.empty_like(q)
     lse = torch.empty((w.B, w.H, w.n), dtype=torch.float32, device=dev)
@@ -297,14 +317,11 @@ def main():
     main_ms = [e[2].elapsed_time(e[3]) for e in ev]
     conv_ms = [e[3].elapsed_time(e[4]) for e in ev]
     bwd_ms = [e[1].elapsed_time(e[4]) for e in ev]
-    if dist is not None:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = t.item()
+    total_ms = max_over_ranks(total_ms, dist, dev)
 
     fwd_flops, bwd_flops = step_flops(w.B, w.H, w.n, w.d)
     ms_per_step = total_ms / args.steps
-    value = world * (fwd_flops + bwd_flops) / (ms_per_step * 1e-3) / 1e12
+    value = whole_job_tflops(fwd_flops + bwd_flops, world, ms_per_step)
     peaks, peak_src = load_peaks()
     burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
@@ -338,11 +355,8 @@ def main():
     b.record(stream)
     torch.cuda.synchronize()
     e2e_ms = a.elapsed_time(b) / args.e2e_steps
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = t.item()
-    e2e_value = world * (fwd_flops + bwd_flops) / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
+    e2e_value = whole_job_tflops(fwd_flops + bwd_flops, world, e2e_ms)
 
     clk = clocks.summary()
     main_kernel = "bwd_main_q64_kernel" if w.d == 128 else "bwd_main_kernel"
