@@ -603,6 +603,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 //                   contiguous in global memory); this warp adds it with one bulk reduction.
 // In the compute loop a tile goes P(i) -> dS(i) -> stage dQ(i-1), so staging overlaps the MMAs.
 // ------------------------------------------------------------------------------------------
+// Single-lane issue helpers for a converged warp (see elect_one).
+#define MMA_SS(...) do { if (elect_one()) mma_ss(__VA_ARGS__); } while (0)
+#define MMA_TS(...) do { if (elect_one()) mma_ts(__VA_ARGS__); } while (0)
+#define MMA_COMMIT(bar) do { if (elect_one()) mma_commit(bar); } while (0)
+
 namespace q64 {
 constexpr int kThreads = 352;
 constexpr int BQ = 64;                     // query rows per tile
@@ -734,7 +739,8 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
         }
     } else if (warp == 9) {
         // ---------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        // The whole warp runs this loop (warp-uniform state); one elected lane issues.
+        {
             constexpr uint32_t idS = idesc_bf16_f32(128, 64, 0, 0);      // S^T, dP^T
             constexpr uint32_t idKV = idesc_bf16_f32(128, 128, 0, 1);    // dV, dK
             constexpr uint32_t idQ = idesc_bf16_f32(128, 64, 1, 1);      // dQ^T
@@ -753,68 +759,68 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
                 const SDesc bq = stage(Q_k, it % STAGES);
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    mma_ss(tmem + COL_S, sdesc_at(K_k, k128(ks)), sdesc_at(bq, k64(ks)), idS, ks > 0 ? 1u : 0u);
+                    MMA_SS(tmem + COL_S, sdesc_at(K_k, k128(ks)), sdesc_at(bq, k64(ks)), idS, ks > 0 ? 1u : 0u);
             };
             auto issue_dp = [&](int it) {
                 const SDesc bo = stage(dO_k, it % STAGES);
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    mma_ss(tmem + COL_DP, sdesc_at(V_k, k128(ks)), sdesc_at(bo, k64(ks)), idS, ks > 0 ? 1u : 0u);
+                    MMA_SS(tmem + COL_DP, sdesc_at(V_k, k128(ks)), sdesc_at(bo, k64(ks)), idS, ks > 0 ? 1u : 0u);
             };
-            bool ok = bounded_wait(&bars->kv_full, 0, abort, lim);
-            if (ok) ok = bounded_wait(&bars->q_full[0], 0, abort, lim);
+            bool ok = bounded_wait_warp(&bars->kv_full, 0, abort, lim);
+            if (ok) ok = bounded_wait_warp(&bars->q_full[0], 0, abort, lim);
             tc_fence_after();
             if (ok) {
                 issue_s(0);
-                mma_commit(&bars->s_full);
+                MMA_COMMIT(&bars->s_full);
             }
             for (int it = 0; ok && it < NT; ++it) {
                 const int st = it % STAGES;
                 // dP^T(i): its columns were last read for dS^T(i-1), which ds_full(i-1) covered
                 issue_dp(it);
-                mma_commit(&bars->dp_full);
-                if (!(ok = bounded_wait(&bars->p_full, it & 1, abort, lim))) break;
+                MMA_COMMIT(&bars->dp_full);
+                if (!(ok = bounded_wait_warp(&bars->p_full, it & 1, abort, lim))) break;
                 tc_fence_after();
                 {   // dV += P^T · dO  (P^T: queries 0-31 at S+0.., 32-63 at S+32..)
                     const SDesc bo = stage(dO_mn, st);
-                    mma_ts(tmem + COL_DV, tmem + COL_S, sdesc_at(bo, 0), idKV, it > 0 ? 1u : 0u);
+                    MMA_TS(tmem + COL_DV, tmem + COL_S, sdesc_at(bo, 0), idKV, it > 0 ? 1u : 0u);
 #pragma unroll
                     for (int ks = 1; ks < 4; ++ks)
-                        mma_ts(tmem + COL_DV, tmem + COL_S + (ks >> 1) * 32 + (ks & 1) * 8,
+                        MMA_TS(tmem + COL_DV, tmem + COL_S + (ks >> 1) * 32 + (ks & 1) * 8,
                                sdesc_at(bo, static_cast<uint32_t>((ks * 2048) >> 4)), idKV, 1u);
                 }
                 if (it + 1 < NT) {
                     const int st1 = (it + 1) % STAGES;
-                    if (!(ok = bounded_wait(&bars->q_full[st1], ((it + 1) / STAGES) & 1, abort, lim))) break;
+                    if (!(ok = bounded_wait_warp(&bars->q_full[st1], ((it + 1) / STAGES) & 1, abort, lim))) break;
                     tc_fence_after();
                     issue_s(it + 1);
-                    mma_commit(&bars->s_full);
+                    MMA_COMMIT(&bars->s_full);
                 }
-                if (!(ok = bounded_wait(&bars->ds_full, it & 1, abort, lim))) break;
+                if (!(ok = bounded_wait_warp(&bars->ds_full, it & 1, abort, lim))) break;
                 tc_fence_after();
                 {   // dK += dS^T · Q
                     const SDesc bq = stage(Q_mn, st);
-                    mma_ss(tmem + COL_DK, sdesc_at(dS_k, 0), sdesc_at(bq, 0), idKV, it > 0 ? 1u : 0u);
+                    MMA_SS(tmem + COL_DK, sdesc_at(dS_k, 0), sdesc_at(bq, 0), idKV, it > 0 ? 1u : 0u);
 #pragma unroll
                     for (int ks = 1; ks < 4; ++ks)
-                        mma_ss(tmem + COL_DK, sdesc_at(dS_k, static_cast<uint32_t>((ks * 32) >> 4)),
+                        MMA_SS(tmem + COL_DK, sdesc_at(dS_k, static_cast<uint32_t>((ks * 32) >> 4)),
                                sdesc_at(bq, static_cast<uint32_t>((ks * 2048) >> 4)), idKV, 1u);
                 }
                 const int b2 = it & 1;
                 if (it >= 2) {
-                    if (!(ok = bounded_wait(&bars->dq_drained[b2], ((it - 2) >> 1) & 1, abort, lim))) break;
+                    if (!(ok = bounded_wait_warp(&bars->dq_drained[b2], ((it - 2) >> 1) & 1, abort, lim))) break;
                     tc_fence_after();
                 }
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)      // dQ^T = K^T · dS^T  (M = d, N = 64 queries)
-                    mma_ss(tmem + COL_DQ + b2 * 64, sdesc_at(K_mn, static_cast<uint32_t>((ks * 2048) >> 4)),
+                    MMA_SS(tmem + COL_DQ + b2 * 64, sdesc_at(K_mn, static_cast<uint32_t>((ks * 2048) >> 4)),
                            sdesc_at(dS_mn, static_cast<uint32_t>((ks * 2048) >> 4)), idQ, ks > 0 ? 1u : 0u);
-                mma_commit(&bars->dq_full[b2]);
-                mma_commit(&bars->ds_free);
-                mma_commit(&bars->q_empty[st]);
+                MMA_COMMIT(&bars->dq_full[b2]);
+                MMA_COMMIT(&bars->ds_free);
+                MMA_COMMIT(&bars->q_empty[st]);
             }
-            if (ok) mma_commit(&bars->dkv_done);
-            mma_commit(&bars->teardown);
+            if (ok) MMA_COMMIT(&bars->dkv_done);
+            MMA_COMMIT(&bars->teardown);
             drain_wait_bwd(&bars->teardown, 0, 100000000ull);
         }
         __syncwarp();

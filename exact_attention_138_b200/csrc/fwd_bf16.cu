@@ -81,6 +81,11 @@ __device__ __forceinline__ void drain_wait_fwd(uint64_t* bar, uint32_t parity, u
         }
 }
 
+// Single-lane issue helpers for a converged warp (see elect_one).
+#define FMMA_SS(...) do { if (elect_one()) mma_ss(__VA_ARGS__); } while (0)
+#define FMMA_TS(...) do { if (elect_one()) mma_ts(__VA_ARGS__); } while (0)
+#define FMMA_COMMIT(bar) do { if (elect_one()) mma_commit(bar); } while (0)
+
 template <int D>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
@@ -190,16 +195,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
     } else if (warp == 9) {
         // ---------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        // The whole warp runs this loop (warp-uniform state); one elected lane issues.
+        {
             constexpr uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);
             constexpr uint32_t idPV = idesc_bf16_f32(128, D, 0, 1);
             const uint32_t sQa = smem_addr(sQ), sKa = smem_addr(sK), sVa = smem_addr(sV);
-            bool ok = bounded_wait(&bars->q_full, 0, abort, lim);
+            bool ok = bounded_wait_warp(&bars->q_full, 0, abort, lim);
             tc_fence_after();
             int k_ready = -1;
             auto wait_k = [&](int jj) -> bool {
                 if (k_ready >= jj) return true;
-                if (!bounded_wait(&bars->k_full[jj % C::STAGES], (jj / C::STAGES) & 1, abort,
+                if (!bounded_wait_warp(&bars->k_full[jj % C::STAGES], (jj / C::STAGES) & 1, abort,
                                   lim))
                     return false;
                 tc_fence_after();
@@ -224,16 +230,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 for (int ks = 0; ks < D / 16; ++ks) {
                     const uint32_t off =
                         static_cast<uint32_t>((((ks * 16) / C::CW) * C::CHUNK + ((ks * 16) % C::CW) * 2) >> 4);
-                    mma_ss(d, sdesc_at(a, off), sdesc_at(b, off), idS, ks > 0 ? 1u : 0u);
+                    FMMA_SS(d, sdesc_at(a, off), sdesc_at(b, off), idS, ks > 0 ? 1u : 0u);
                 }
             };
             auto issue_pv = [&](int g, int jj) {
                 const SDesc b = dV[jj % C::STAGES];
                 const uint32_t d = tmem + g * 128, a = tmem + 256 + g * 128;
-                mma_ts(d, a, sdesc_at(b, 0), idPV, jj > 0 ? 1u : 0u);
+                FMMA_TS(d, a, sdesc_at(b, 0), idPV, jj > 0 ? 1u : 0u);
 #pragma unroll
                 for (int ks = 1; ks < C::BN / 16; ++ks)
-                    mma_ts(d, a + ks * 8, sdesc_at(b, static_cast<uint32_t>((ks * 16 * C::SWB) >> 4)),
+                    FMMA_TS(d, a + ks * 8, sdesc_at(b, static_cast<uint32_t>((ks * 16 * C::SWB) >> 4)),
                            idPV, 1u);
             };
             if (ok) ok = wait_k(0);
@@ -241,18 +247,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 for (int g = 0; g < 2; ++g)
                     if (T[g] > 0) {
                         issue_s(g, 0);
-                        mma_commit(&bars->s_full[g]);
+                        FMMA_COMMIT(&bars->s_full[g]);
                     }
-                mma_commit(&bars->k_empty[0]);
+                FMMA_COMMIT(&bars->k_empty[0]);
             }
             for (int jj = 0; ok && jj < Tmax; ++jj) {
                 bool v_ready = false;
                 for (int g = 0; g < 2 && ok; ++g) {
                     if (jj >= T[g]) continue;
-                    if (!bounded_wait(&bars->p_full[g], jj & 1, abort, lim)) { ok = false; break; }
+                    if (!bounded_wait_warp(&bars->p_full[g], jj & 1, abort, lim)) { ok = false; break; }
                     tc_fence_after();
                     if (!v_ready) {
-                        if (!bounded_wait(&bars->v_full[jj % C::STAGES], (jj / C::STAGES) & 1,
+                        if (!bounded_wait_warp(&bars->v_full[jj % C::STAGES], (jj / C::STAGES) & 1,
                                           abort, lim)) { ok = false; break; }
                         tc_fence_after();
                         v_ready = true;
@@ -261,17 +267,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     if (jj + 1 < T[g]) {
                         if (!wait_k(jj + 1)) { ok = false; break; }
                         issue_s(g, jj + 1);
-                        mma_commit(&bars->s_full[g]);
+                        FMMA_COMMIT(&bars->s_full[g]);
                     } else {
-                        mma_commit(&bars->o_done[g]);
+                        FMMA_COMMIT(&bars->o_done[g]);
                     }
                 }
                 if (!ok) break;
-                mma_commit(&bars->v_empty[jj % C::STAGES]);
-                if (jj + 1 < Tmax) mma_commit(&bars->k_empty[(jj + 1) % C::STAGES]);
+                FMMA_COMMIT(&bars->v_empty[jj % C::STAGES]);
+                if (jj + 1 < Tmax) FMMA_COMMIT(&bars->k_empty[(jj + 1) % C::STAGES]);
             }
             // all MMAs of this CTA complete before TMEM is released
-            mma_commit(&bars->teardown);
+            FMMA_COMMIT(&bars->teardown);
             drain_wait_fwd(&bars->teardown, 0, 100000000ull);
         }
         __syncwarp();

@@ -83,6 +83,12 @@ __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, vol
     }
 }
 
+// bounded_wait for a converged warp: every lane waits and all agree on the outcome.
+__device__ __forceinline__ bool bounded_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                  uint64_t limit_ns) {
+    return __all_sync(0xffffffffu, bounded_wait(bar, parity, abort, limit_ns));
+}
+
 // ------------------------------------------------------------------------------------------
 // Fences
 // ------------------------------------------------------------------------------------------
@@ -293,6 +299,20 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// One lane of a converged warp (the lowest active one) returns true. Issuing MMAs from a
+// converged warp keeps loop state and descriptors warp-uniform, so they can live in uniform
+// registers; the elected lane is the same on every call while the whole warp is active, which
+// tcgen05.commit needs (it tracks the MMAs of the issuing thread).
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
 }
 
 // Arrive once on `bar` when every tcgen05 operation issued so far by this thread completes.
