@@ -598,10 +598,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 //                   LSE·log2e and D through a 3-deep ring.
 //   warp 9          MMA issuer, per tile:  dP^T(i) -> [P^T(i)] dV += P^T dO -> S^T(i+1) ->
 //                   [dS^T(i)] dK += dS^T Q -> dQ^T(i) = K^T dS^T (into buffer i mod 2).
-//   warp 10         dQ reducer: the compute warps copy dQ^T(i) out of TMEM into a shared-memory
-//                   staging tile laid out like the accumulator rows (64 x 128 fp32, 32 KB
-//                   contiguous in global memory); this warp adds it with one bulk reduction.
-// In the compute loop a tile goes P(i) -> dS(i) -> stage dQ(i-1), so staging overlaps the MMAs.
+//   warps 12-15     dQ drain warpgroup: copies dQ^T(i) out of TMEM (one head-dim row per thread)
+//                   into a shared-memory staging tile laid out like the accumulator rows (64 x 128
+//                   fp32, 32 KB contiguous in global memory); one elected lane then adds it with
+//                   a single bulk reduction. This work never sits on the compute warps' path.
 // ------------------------------------------------------------------------------------------
 // Single-lane issue helpers for a converged warp (see elect_one).
 #define MMA_SS(...) do { if (elect_one()) mma_ss(__VA_ARGS__); } while (0)
@@ -609,7 +609,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #define MMA_COMMIT(bar) do { if (elect_one()) mma_commit(bar); } while (0)
 
 namespace q64 {
-constexpr int kThreads = 352;
+constexpr int kThreads = 512;              // warps 10-11 idle: the drain warpgroup must start at
+                                           // warp 12 to cover TMEM lane quarters 0-3
 constexpr int BQ = 64;                     // query rows per tile
 constexpr int KTILE = 128 * 128 * 2;       // K_j or V_j: 2 chunks [128 rows][64 d], SW128
 constexpr int QTILE = 64 * 128 * 2;        // Q_i or dO_i: 2 chunks [64 rows][64 d]
@@ -628,7 +629,7 @@ struct Bars {
     uint64_t q_full[STAGES], q_empty[STAGES];
     uint64_t s_full, dp_full, p_full, ds_full, ds_free, dkv_done, teardown;
     uint64_t dq_full[2], dq_drained[2];
-    uint64_t stg_full, stg_free;
+    uint64_t drain_sync[2];
     uint32_t tmem_base;
     int abort;
 };
@@ -683,10 +684,10 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
         mbar_init(&bars->teardown, 1);
         for (int b2 = 0; b2 < 2; ++b2) {
             mbar_init(&bars->dq_full[b2], 1);
-            mbar_init(&bars->dq_drained[b2], 256);
+            mbar_init(&bars->dq_drained[b2], 128);
         }
-        mbar_init(&bars->stg_full, 256);
-        mbar_init(&bars->stg_free, 1);
+        mbar_init(&bars->drain_sync[0], 128);
+        mbar_init(&bars->drain_sync[1], 128);
         bars->abort = ((smem_addr(smem) & 1023u) != 0) ? 1 : 0;
         if (bars->abort) report_error(3);
         fence_barrier_init();
@@ -824,18 +825,45 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
             drain_wait_bwd(&bars->teardown, 0, 100000000ull);
         }
         __syncwarp();
-    } else if (warp == 10) {
-        // ---------------------------------------------------------------- dQ reducer
-        if (lane == 0) {
-            for (int it = 0; it < NT; ++it) {
-                if (!bounded_wait(&bars->stg_full, it & 1, abort, lim)) break;
+    } else if (warp >= 12) {
+        // ---------------------------------------------------------------- dQ drain warpgroup
+        const int r = (warp & 3) * 32 + lane;              // head-dim row = TMEM lane
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const bool leader = (warp == 12);
+        uint32_t sync_phase[2] = {0, 0};
+        // Warpgroup barrier on an mbarrier with a bounded wait (no thread can hang on it).
+        auto wg_sync = [&](int s) -> bool {
+            mbar_arrive(&bars->drain_sync[s]);
+            const bool okw = bounded_wait_warp(&bars->drain_sync[s], sync_phase[s], abort, lim);
+            sync_phase[s] ^= 1;
+            return okw;
+        };
+        for (int it = 0; it < NT; ++it) {
+            const int b2 = it & 1;
+            if (!bounded_wait_warp(&bars->dq_full[b2], (it >> 1) & 1, abort, lim)) break;
+            tc_fence_after();
+            uint32_t u[64];
+            tmem_ld32(tmem + lane_base + COL_DQ + b2 * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+            tmem_ld32(tmem + lane_base + COL_DQ + b2 * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+            tmem_ld_wait();
+            reg_fence<64>(u);
+            tc_fence_before();
+            mbar_arrive(&bars->dq_drained[b2]);
+            // the previous tile's bulk reduction must have read the staging tile
+            if (leader && lane == 0) bulk_wait_read_all();
+            if (!wg_sync(0)) break;
+#pragma unroll
+            for (int x = 0; x < 64; ++x) sStg[x * D + r] = __uint_as_float(u[x]);
+            fence_proxy_async_smem();
+            if (!wg_sync(1)) break;
+            if (leader && lane == 0) {
                 const int i = i_begin + it;
                 float* dst = p.dq_acc + (static_cast<size_t>(bh) * p.n_pad + i * BQ) * D;
                 volatile int* sem = p.deterministic ? p.sems + static_cast<size_t>(bh) * nq + i : nullptr;
+                bool got = true;
                 if (sem) {
                     // contributions to one query tile are added in increasing key-tile order
                     const uint64_t t0 = globaltimer_ns();
-                    bool got = true;
                     while (*sem < j) {
                         if (*abort || globaltimer_ns() - t0 > lim) {
                             *abort = 1;
@@ -845,24 +873,23 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
                         }
                         __nanosleep(64);
                     }
-                    if (!got) break;
                     __threadfence();
                 }
-                bulk_reduce_add_f32(dst, sStg, STG_BYTES);
-                bulk_commit();
-                if (sem) {
-                    bulk_wait_all();                 // the adds are done, not only the reads
-                    __threadfence();
-                    atomicAdd(const_cast<int*>(sem), 1);
-                } else {
-                    bulk_wait_read_all();            // staging may be overwritten
+                if (got) {
+                    bulk_reduce_add_f32(dst, sStg, STG_BYTES);
+                    bulk_commit();
+                    if (sem) {
+                        bulk_wait_all();             // the adds are done, not only the reads
+                        __threadfence();
+                        atomicAdd(const_cast<int*>(sem), 1);
+                    }
                 }
-                mbar_arrive(&bars->stg_free);
             }
-            bulk_wait_all();
+            if (*abort) break;
         }
+        if (leader && lane == 0) bulk_wait_all();
         __syncwarp();
-    } else {
+    } else if (warp < 8) {
         // ---------------------------------------------------------------- compute warpgroups
         const int g = warp >> 2;                           // query columns 32g .. 32g+31
         const int r = (warp & 3) * 32 + lane;              // key row = TMEM lane
@@ -875,25 +902,6 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
         };
         float pr[32];
         bool ok = true;
-
-        // dQ^T(it) (lane = head-dim index r, columns = queries) -> staging [query][d]
-        auto stage_dq = [&](int it) -> bool {
-            const int b2 = it & 1;
-            if (!wait_all(&bars->dq_full[b2], (it >> 1) & 1)) return false;
-            if (it > 0 && !wait_all(&bars->stg_free, (it - 1) & 1)) return false;
-            tc_fence_after();
-            uint32_t u[32];
-            tmem_ld32(tmem + lane_base + COL_DQ + b2 * 64 + cb, u);
-            tmem_ld_wait();
-            reg_fence<32>(u);
-            tc_fence_before();
-            mbar_arrive(&bars->dq_drained[b2]);
-#pragma unroll
-            for (int x = 0; x < 32; ++x) sStg[(cb + x) * D + r] = __uint_as_float(u[x]);
-            fence_proxy_async_smem();
-            mbar_arrive(&bars->stg_full);
-            return true;
-        };
 
         for (int it = 0; it < NT; ++it) {
             const int i = i_begin + it;
@@ -959,10 +967,7 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&bars->ds_full);
-            // ---- the previous tile's dQ^T into the staging tile, while this tile's MMAs run
-            if (it > 0 && !(ok = stage_dq(it - 1))) break;
         }
-        if (ok && NT > 0) ok = stage_dq(NT - 1);
         if (ok) ok = wait_all(&bars->dkv_done, 0);
         if (ok) {
             tc_fence_after();
