@@ -17,6 +17,9 @@ Sources of each function are cited in ``attn_oracle.c``:
   * "Apa itu FlashAttention", "Cara kerja teknik Tiling dan Recomputation" (backward recomputes
     the softmax; the gradient formulas are the exact derivative of the definition);
   * "Calculateur de mémoire d'attention", "La formule" (score-matrix bytes B·H·n²·e).
+  * "Attention Mechanism ...", §12 "GQA vs MQA — KV Cache Optimization": query heads in groups of
+    g = H / H_kv share one K/V head; the page expands K and V with repeat_interleave(g, dim=1)
+    and then runs standard attention, which is exactly what fwd_gqa / bwd_gqa do.
 """
 from __future__ import annotations
 
@@ -194,3 +197,34 @@ def bwd_key_rows(q, k, v, do, scale, causal, bh, keys):
     _check(_load().oracle_bwd_key_rows(q, k, v, do, B, H, n, d, float(scale), int(bool(causal)),
                                        int(bh), keys, len(keys), dk, dv), "oracle_bwd_key_rows")
     return dk, dv
+
+
+# ---------------------------------------------------------------------------------------------
+# Grouped-query attention ("Attention Mechanism ...", §12): K, V have H_kv heads; query head h
+# uses K/V head h // (H // H_kv). Forward and backward run on the expanded K/V (the page's
+# repeat_interleave step); the gradient of a shared K/V head is the sum over its query heads.
+# ---------------------------------------------------------------------------------------------
+def _expand_kv(x, H):
+    x = _f32(x)
+    B, Hkv = x.shape[0], x.shape[1]
+    if H % Hkv != 0:
+        raise ValueError("H must be a multiple of H_kv")
+    return np.ascontiguousarray(np.repeat(x, H // Hkv, axis=1))
+
+
+def fwd_gqa(q, k, v, scale, causal=False):
+    q = _f32(q)
+    H = q.shape[1]
+    return fwd(q, _expand_kv(k, H), _expand_kv(v, H), scale, causal)
+
+
+def bwd_gqa(q, k, v, do, scale, causal=False):
+    """Returns (dQ with H heads, dK and dV with H_kv heads, D)."""
+    q = _f32(q)
+    B, H, n, d = q.shape
+    Hkv = _f32(k).shape[1]
+    dq, dk, dv, D = bwd(q, _expand_kv(k, H), _expand_kv(v, H), do, scale, causal)
+    g = H // Hkv
+    dk = dk.reshape(B, Hkv, g, n, d).sum(axis=2)
+    dv = dv.reshape(B, Hkv, g, n, d).sum(axis=2)
+    return dq, dk, dv, D

@@ -336,3 +336,54 @@ def test_bf16_draws_are_rounded_and_reproducible():
     assert all(torch.equal(x, y) for x, y in zip(a, b))
     assert all(x.dtype == torch.bfloat16 for x in a)
     assert float(a[0].float().abs().max()) < 4.0
+
+
+# --------------------------------------------------------------------------------------------
+# Grouped-query attention ("Attention Mechanism ...", §12 "GQA vs MQA")
+# --------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_with_all_kv_heads_is_mha(causal):
+    q, k, v, do = (_rand((2, 4, 40, 16), s) for s in (60, 61, 62, 63))
+    o, lse = oracle.fwd(q, k, v, 0.25, causal)
+    og, lseg = oracle.fwd_gqa(q, k, v, 0.25, causal)
+    assert np.array_equal(o, og) and np.array_equal(lse, lseg)
+    ref = oracle.bwd(q, k, v, do, 0.25, causal)
+    got = oracle.bwd_gqa(q, k, v, do, 0.25, causal)
+    for a, b in zip(ref, got):
+        assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("Hkv,causal", [(2, False), (2, True), (1, True)])
+def test_gqa_matches_torch_repeat_interleave_autograd(Hkv, causal):
+    # The page's recipe, run by torch in fp64 with autograd: repeat_interleave(g, dim=1), then
+    # standard attention; gradients flow back through the repeat into the shared K/V heads.
+    H, n, d, scale = 4, 12, 8, 0.3
+    q, do = _rand((1, H, n, d), 64), _rand((1, H, n, d), 65)
+    k, v = _rand((1, Hkv, n, d), 66), _rand((1, Hkv, n, d), 67)
+    Q, K, V = (torch.from_numpy(x.astype(np.float64)).requires_grad_() for x in (q, k, v))
+    g = H // Hkv
+    S = Q @ K.repeat_interleave(g, dim=1).transpose(-1, -2) * scale
+    if causal:
+        S = S.masked_fill(torch.ones(n, n, dtype=torch.bool).triu(1), float("-inf"))
+    O = torch.softmax(S, -1) @ V.repeat_interleave(g, dim=1)
+    O.backward(torch.from_numpy(do.astype(np.float64)))
+    o, _ = oracle.fwd_gqa(q, k, v, scale, causal)
+    dq, dk, dv, _ = oracle.bwd_gqa(q, k, v, do, scale, causal)
+    np.testing.assert_allclose(o, O.detach().numpy(), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dq, Q.grad.numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dk, K.grad.numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dv, V.grad.numpy(), rtol=0, atol=1e-12)
+
+
+def test_mqa_heads_with_equal_queries_agree():
+    # MQA (one K/V head): query heads with identical queries give identical outputs, and the
+    # shared dV is the sum over heads of P^T dO (here: H times one head's dV for equal dO)
+    qh, doh = _rand((1, 1, 30, 8), 68), _rand((1, 1, 30, 8), 69)
+    q, do = np.repeat(qh, 3, axis=1), np.repeat(doh, 3, axis=1)
+    k, v = _rand((1, 1, 30, 8), 70), _rand((1, 1, 30, 8), 71)
+    o, _ = oracle.fwd_gqa(q, k, v, 0.35, True)
+    assert np.array_equal(o[:, 0], o[:, 1]) and np.array_equal(o[:, 0], o[:, 2])
+    _, dk, dv, _ = oracle.bwd_gqa(q, k, v, do, 0.35, True)
+    _, dk1, dv1, _ = oracle.bwd(qh, k, v, doh, 0.35, True)
+    np.testing.assert_allclose(dv, 3 * dv1, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dk, 3 * dk1, rtol=0, atol=1e-13)
