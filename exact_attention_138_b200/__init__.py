@@ -41,6 +41,11 @@ _lib.attn_error_string.restype = ctypes.c_char_p
 _lib.attn_error_string.argtypes = [_i]
 _lib.attn_fwd.restype = _i
 _lib.attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _i, _vp]
+_lib.attn_fwd_gqa.restype = _i
+_lib.attn_fwd_gqa.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _i, _vp]
+_lib.attn_bwd_gqa.restype = _i
+_lib.attn_bwd_gqa.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f,
+                              _i, _i, _i, _vp, _sz, _vp]
 _lib.attn_bwd_workspace_bytes.restype = _sz
 _lib.attn_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
 _lib.attn_bwd.restype = _i
@@ -85,6 +90,16 @@ def attn_error_string(code: int) -> str:
 
 def attn_fwd(q, k, v, o, lse, B, H, n, d, scale, causal, dtype, stream) -> int:
     return _lib.attn_fwd(q, k, v, o, lse, B, H, n, d, scale, causal, dtype, stream)
+
+
+def attn_fwd_gqa(q, k, v, o, lse, B, H, Hkv, n, d, scale, causal, dtype, stream) -> int:
+    return _lib.attn_fwd_gqa(q, k, v, o, lse, B, H, Hkv, n, d, scale, causal, dtype, stream)
+
+
+def attn_bwd_gqa(q, k, v, o, dO, lse, dq, dk, dv, B, H, Hkv, n, d, scale, causal, dtype,
+                 deterministic, workspace, ws_bytes, stream) -> int:
+    return _lib.attn_bwd_gqa(q, k, v, o, dO, lse, dq, dk, dv, B, H, Hkv, n, d, scale, causal,
+                             dtype, deterministic, workspace, ws_bytes, stream)
 
 
 def attn_bwd_workspace_bytes(B, H, n, d, deterministic) -> int:
@@ -151,31 +166,48 @@ def _check(rc, where):
         raise AttnError(rc, where)
 
 
+def _kv_heads(q, k, v):
+    """K/V head count: equal to q's (multi-head) or a divisor of it (grouped-query, k and v of
+    shape (B, Hkv, n, d))."""
+    B, H, n, d = _dims(q)
+    kd = _dims(k)
+    if k.dim() != q.dim() or v.shape != k.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("k and v must match each other and q's dtype")
+    if kd[0] != B or kd[2] != n or kd[3] != d or H % kd[1] != 0:
+        raise ValueError("k, v must be (B, Hkv, n, d) with H a multiple of Hkv")
+    return kd[1]
+
+
 def forward(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None):
-    """O, LSE = attention(q, k, v). q, k, v: contiguous CUDA tensors (B,H,n,d) or (n,d), bf16 or
-    fp32. Returns O (same dtype/shape as q) and LSE (fp32, (B,H,n))."""
+    """O, LSE = attention(q, k, v). q: contiguous CUDA tensor (B,H,n,d) or (n,d), bf16 or fp32;
+    k, v: same shape, or (B,Hkv,n,d) for grouped-query attention. Returns O (same dtype/shape as
+    q) and LSE (fp32, (B,H,n))."""
     import torch
     B, H, n, d = _dims(q)
-    for t in (k, v):
-        if t.shape != q.shape or t.dtype != q.dtype:
-            raise ValueError("q, k, v must have the same shape and dtype")
+    Hkv = _kv_heads(q, k, v)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, n), dtype=torch.float32, device=q.device)
-    rc = attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, n, d, float(scale),
-                  int(bool(causal)), _dtype_code(q), _stream_handle(stream))
+    if Hkv == H:
+        rc = attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, n, d, float(scale),
+                      int(bool(causal)), _dtype_code(q), _stream_handle(stream))
+    else:
+        rc = attn_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Hkv, n, d,
+                          float(scale), int(bool(causal)), _dtype_code(q), _stream_handle(stream))
     _check(rc, "attn_fwd")
     return out, lse
 
 
 def backward(q, k, v, o, do, lse, causal=False, scale=None, deterministic=False, dq=None,
              dk=None, dv=None, workspace=None, stream=None):
-    """dQ, dK, dV of attention given dO (bf16 tensors, lse from `forward`)."""
+    """dQ, dK, dV of attention given dO (bf16 tensors, lse from `forward`). For grouped-query
+    inputs dK, dV have k's (B, Hkv, n, d) shape and sum over each group's query heads."""
     import torch
     B, H, n, d = _dims(q)
+    Hkv = _kv_heads(q, k, v)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     dq = torch.empty_like(q) if dq is None else dq
@@ -184,10 +216,16 @@ def backward(q, k, v, o, do, lse, causal=False, scale=None, deterministic=False,
     need = attn_bwd_workspace_bytes(B, H, n, d, int(bool(deterministic)))
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    rc = attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk),
-                  _ptr(dv), B, H, n, d, float(scale), int(bool(causal)), _dtype_code(q),
-                  int(bool(deterministic)), _ptr(workspace),
-                  workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    ws_bytes = workspace.numel() * workspace.element_size()
+    if Hkv == H:
+        rc = attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk),
+                      _ptr(dv), B, H, n, d, float(scale), int(bool(causal)), _dtype_code(q),
+                      int(bool(deterministic)), _ptr(workspace), ws_bytes, _stream_handle(stream))
+    else:
+        rc = attn_bwd_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
+                          _ptr(dk), _ptr(dv), B, H, Hkv, n, d, float(scale), int(bool(causal)),
+                          _dtype_code(q), int(bool(deterministic)), _ptr(workspace), ws_bytes,
+                          _stream_handle(stream))
     _check(rc, "attn_bwd")
     return dq, dk, dv
 

@@ -131,16 +131,17 @@ unsigned attn_set_wait_timeout_us(unsigned us) {
     return g_timeout_us.exchange(us);
 }
 
-int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-             int n, int d, float scale, int causal, int dtype, void* stream) {
+static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                    int H, int Hkv, int n, int d, float scale, int causal, int dtype, void* stream) {
     if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID;
     int rc = validate_common(B, H, n, d, scale, dtype);
     if (rc) return rc;
+    if (Hkv < 1 || H % Hkv != 0) return ATTN_ERR_INVALID;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
         return ATTN_ERR_INVALID;
     FwdArgs a;
     a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
-    a.B = B; a.H = H; a.n = n; a.d = d;
+    a.B = B; a.H = H; a.n = n; a.d = d; a.Hkv = Hkv;
     a.scale = scale;
     a.causal = causal ? 1 : 0;
     a.timeout_ns = static_cast<uint64_t>(g_timeout_us.load()) * 1000ull;
@@ -149,18 +150,29 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
     return to_code(e);
 }
 
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+             int n, int d, float scale, int causal, int dtype, void* stream) {
+    return fwd_impl(q, k, v, o, lse, B, H, H, n, d, scale, causal, dtype, stream);
+}
+
+int attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int Hkv, int n, int d, float scale, int causal, int dtype, void* stream) {
+    return fwd_impl(q, k, v, o, lse, B, H, Hkv, n, d, scale, causal, dtype, stream);
+}
+
 size_t attn_bwd_workspace_bytes(int B, int H, int n, int d, int deterministic) {
     if (B < 1 || H < 1 || n < 1 || d < 1) return 0;
     return ws_layout(B, H, n, d, deterministic).total;
 }
 
-int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
-             const float* lse, void* dq, void* dk, void* dv, int B, int H, int n, int d,
-             float scale, int causal, int dtype, int deterministic, void* workspace,
-             size_t ws_bytes, void* stream) {
+static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                    const float* lse, void* dq, void* dk, void* dv, int B, int H, int Hkv, int n,
+                    int d, float scale, int causal, int dtype, int deterministic, void* workspace,
+                    size_t ws_bytes, void* stream) {
     if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return ATTN_ERR_INVALID;
     int rc = validate_common(B, H, n, d, scale, dtype);
     if (rc) return rc;
+    if (Hkv < 1 || H % Hkv != 0) return ATTN_ERR_INVALID;
     if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
     const void* ptrs[] = {q, k, v, o, dO, lse, dq, dk, dv};
     for (const void* p : ptrs)
@@ -172,7 +184,7 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
     BwdArgs a;
     a.q = q; a.k = k; a.v = v; a.o = o; a.dO = dO; a.lse = lse;
     a.dq = dq; a.dk = dk; a.dv = dv;
-    a.B = B; a.H = H; a.n = n; a.d = d;
+    a.B = B; a.H = H; a.n = n; a.d = d; a.Hkv = Hkv;
     a.scale = scale;
     a.causal = causal ? 1 : 0;
     a.deterministic = deterministic ? 1 : 0;
@@ -184,6 +196,22 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
     a.timeout_ns = static_cast<uint64_t>(g_timeout_us.load()) * 1000ull;
     a.phase_events = g_phase_on.load() ? g_phase_events : nullptr;
     return to_code(launch_bwd_bf16(a, static_cast<cudaStream_t>(stream)));
+}
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+             const float* lse, void* dq, void* dk, void* dv, int B, int H, int n, int d,
+             float scale, int causal, int dtype, int deterministic, void* workspace,
+             size_t ws_bytes, void* stream) {
+    return bwd_impl(q, k, v, o, dO, lse, dq, dk, dv, B, H, H, n, d, scale, causal, dtype,
+                    deterministic, workspace, ws_bytes, stream);
+}
+
+int attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                 const float* lse, void* dq, void* dk, void* dv, int B, int H, int Hkv, int n,
+                 int d, float scale, int causal, int dtype, int deterministic, void* workspace,
+                 size_t ws_bytes, void* stream) {
+    return bwd_impl(q, k, v, o, dO, lse, dq, dk, dv, B, H, Hkv, n, d, scale, causal, dtype,
+                    deterministic, workspace, ws_bytes, stream);
 }
 
 void attn_set_bwd_phase_events(void* const* events) {

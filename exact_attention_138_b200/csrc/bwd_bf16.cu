@@ -62,6 +62,7 @@ struct BwdKParams {
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
     int n, n_pad, BH, nq, causal, deterministic, group;
+    int kv_group;     // query heads per K/V head; BH counts K/V heads (one CTA row per K/V head)
     float scale, scale_log2;
     uint64_t timeout_ns;
 };
@@ -207,10 +208,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int gsize = min(p.group, p.BH - gbase);
     const int r_in = L - gbase * p.nq;
     const int j = r_in / gsize;
-    const int bh = gbase + r_in % gsize;
+    const int kvbh = gbase + r_in % gsize;        // K/V head of this CTA
     const int n = p.n;
     const int i_begin = p.causal ? j : 0;
-    const int NT = p.nq - i_begin;
+    const int NT = p.nq - i_begin;                // query tiles per query head
+    const int NTT = NT * p.kv_group;              // over all query heads sharing this K/V head
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->kv_full, 1);
@@ -251,20 +253,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (lane == 0 && !*abort) {
             mbar_arrive_expect_tx(&bars->kv_full, 2 * C::TILE);
             for (int ch = 0; ch < C::NCH; ++ch) {
-                tma_load_3d(sK + ch * C::CHUNK, &tmK, &bars->kv_full, ch * C::CW, j * 128, bh);
-                tma_load_3d(sV + ch * C::CHUNK, &tmV, &bars->kv_full, ch * C::CW, j * 128, bh);
+                tma_load_3d(sK + ch * C::CHUNK, &tmK, &bars->kv_full, ch * C::CW, j * 128, kvbh);
+                tma_load_3d(sV + ch * C::CHUNK, &tmV, &bars->kv_full, ch * C::CW, j * 128, kvbh);
             }
             int issued = 0;
-            for (int it = 0; it < NT; ++it) {
+            for (int it = 0; it < NTT; ++it) {
                 const int st = it & 1, f = it >> 1;
                 if (f > 0 && !bounded_wait(&bars->q_empty[st], (f - 1) & 1, abort, lim)) break;
-                const int i = i_begin + it;
+                const int i = i_begin + it % NT;
+                const int qbh = kvbh * p.kv_group + it / NT;
                 mbar_arrive_expect_tx(&bars->q_full[st], 2 * C::TILE);
                 for (int ch = 0; ch < C::NCH; ++ch) {
                     tma_load_3d(sQ + st * C::TILE + ch * C::CHUNK, &tmQ, &bars->q_full[st],
-                                ch * C::CW, i * 128, bh);
+                                ch * C::CW, i * 128, qbh);
                     tma_load_3d(sdO + st * C::TILE + ch * C::CHUNK, &tmdO, &bars->q_full[st],
-                                ch * C::CW, i * 128, bh);
+                                ch * C::CW, i * 128, qbh);
                 }
                 issued = it + 1;
             }
@@ -324,7 +327,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 issue_dp(0);
                 mma_commit(&bars->dp_full);
             }
-            for (int it = 0; ok && it < NT; ++it) {
+            for (int it = 0; ok && it < NTT; ++it) {
                 const int st = it & 1;
                 if (it > 0) {
                     if (!(ok = bounded_wait(&bars->dq_drained, (it - 1) & 1, abort, lim))) break;
@@ -342,7 +345,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         mma_ts(tmem + COL_DV, tmem + COL_S + (ks >> 2) * 64 + (ks & 3) * 8,
                                sdesc_at(bo, roff(ks)), idKN, 1u);
                 }
-                if (it + 1 < NT) {
+                if (it + 1 < NTT) {
                     if (!(ok = bounded_wait(&bars->q_full[(it + 1) & 1], ((it + 1) >> 1) & 1,
                                             abort, lim)))
                         break;
@@ -405,13 +408,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
         // dQ partial of tile `it` out of TMEM into the fp32 accumulator
         auto drain = [&](int it) -> bool {
-            const int i = i_begin + it;
+            const int i = i_begin + it % NT;
+            const int qbh = kvbh * p.kv_group + it / NT;
             if (!wait_all(&bars->dq_full, it & 1)) return false;
             tc_fence_after();
             if (p.deterministic) {
                 // add this tile's partial only after every lower key tile has added its own
                 // (each CTA contributes two halves, one per warpgroup)
-                volatile int* sem = p.sems + static_cast<size_t>(bh) * p.nq + i;
+                volatile int* sem = p.sems + static_cast<size_t>(qbh) * p.nq + i;
                 const int need = 2 * (p.causal ? j : j);
                 bool got = true;
                 if (t == 0) {
@@ -435,7 +439,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     return false;
                 }
             }
-            float* acc_tile = p.dq_acc + (static_cast<size_t>(bh) * p.n_pad + i * 128) * D;
+            float* acc_tile = p.dq_acc + (static_cast<size_t>(qbh) * p.n_pad + i * 128) * D;
             if constexpr (C::DQT) {
                 // lane r = head-dim index; columns = queries cb .. cb+63
 #pragma unroll 1
@@ -473,21 +477,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (p.deterministic) {
                 __threadfence();
                 wg_bar();
-                if (t == 0) atomicAdd(p.sems + static_cast<size_t>(bh) * p.nq + i, 1);
+                if (t == 0) atomicAdd(p.sems + static_cast<size_t>(qbh) * p.nq + i, 1);
             }
             return true;
         };
 
-        for (int it = 0; it < NT; ++it) {
-            const int i = i_begin + it;
+        for (int it = 0; it < NTT; ++it) {
+            const int i = i_begin + it % NT;
+            const int qbh = kvbh * p.kv_group + it / NT;
             float* sL = sStat + (g * 2 + (it & 1)) * 128;
             float* sD = sL + 64;
             {
                 const int qq = i * 128 + cb + (t & 63);
                 if (t < 64)
-                    sL[t] = (qq < n) ? p.lse[static_cast<size_t>(bh) * n + qq] * kBwdLog2e : INFINITY;
+                    sL[t] = (qq < n) ? p.lse[static_cast<size_t>(qbh) * n + qq] * kBwdLog2e : INFINITY;
                 else
-                    sD[t - 64] = (qq < n) ? p.Dvec[static_cast<size_t>(bh) * p.n_pad + qq] : 0.f;
+                    sD[t - 64] = (qq < n) ? p.Dvec[static_cast<size_t>(qbh) * p.n_pad + qq] : 0.f;
             }
             wg_bar();
             // ---- P^T = exp2(S^T·scale·log2e - LSE·log2e), masked; bf16 copy into TMEM
@@ -547,11 +552,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tc_fence_before();
             mbar_arrive(&bars->ds_full);
         }
-        if (ok && NT > 0) ok = drain(NT - 1);
+        if (ok && NTT > 0) ok = drain(NTT - 1);
         if (ok) ok = wait_all(&bars->dkv_done, 0);
         if (ok) {
             tc_fence_after();
-            const size_t orow = (static_cast<size_t>(bh) * n + kidx) * D + g * (D / 2);
+            const size_t orow = (static_cast<size_t>(kvbh) * n + kidx) * D + g * (D / 2);
 #pragma unroll 1
             for (int which = 0; which < 2; ++which) {
                 const uint32_t tacc = tmem + lane_base + (which == 0 ? COL_DV : COL_DK) + g * (D / 2);
@@ -663,11 +668,12 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
     const int gsize = min(p.group, p.BH - gbase);
     const int r_in = L - gbase * p.nq;
     const int j = r_in / gsize;
-    const int bh = gbase + r_in % gsize;
+    const int kvbh = gbase + r_in % gsize;         // K/V head of this CTA
     const int n = p.n;
     const int nq = p.n_pad / BQ;                   // 64-row query tiles per head (padded)
     const int i_begin = p.causal ? 2 * j : 0;
-    const int NT = nq - i_begin;
+    const int NT = nq - i_begin;                   // query tiles per query head
+    const int NTT = NT * p.kv_group;               // over all query heads sharing this K/V head
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->kv_full, 1);
@@ -712,14 +718,15 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
         if (lane == 0 && !*abort) {
             mbar_arrive_expect_tx(&bars->kv_full, 2 * KTILE);
             for (int ch = 0; ch < 2; ++ch) {
-                tma_load_3d(sK + ch * 16384, &tmK, &bars->kv_full, ch * 64, j * 128, bh);
-                tma_load_3d(sV + ch * 16384, &tmV, &bars->kv_full, ch * 64, j * 128, bh);
+                tma_load_3d(sK + ch * 16384, &tmK, &bars->kv_full, ch * 64, j * 128, kvbh);
+                tma_load_3d(sV + ch * 16384, &tmV, &bars->kv_full, ch * 64, j * 128, kvbh);
             }
             int issued = 0;
-            for (int it = 0; it < NT; ++it) {
+            for (int it = 0; it < NTT; ++it) {
                 const int st = it % STAGES, f = it / STAGES;
                 if (f > 0 && !bounded_wait(&bars->q_empty[st], (f - 1) & 1, abort, lim)) break;
-                const int i = i_begin + it;
+                const int i = i_begin + it % NT;
+                const int bh = kvbh * p.kv_group + it / NT;   // query head
                 mbar_arrive_expect_tx(&bars->q_full[st], 2 * QTILE + 2 * 256);
                 for (int ch = 0; ch < 2; ++ch) {
                     tma_load_3d(sQ + st * QTILE + ch * QCHUNK, &tmQ, &bars->q_full[st], ch * 64,
@@ -775,7 +782,7 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
                 issue_s(0);
                 MMA_COMMIT(&bars->s_full);
             }
-            for (int it = 0; ok && it < NT; ++it) {
+            for (int it = 0; ok && it < NTT; ++it) {
                 const int st = it % STAGES;
                 // dP^T(i): its columns were last read for dS^T(i-1), which ds_full(i-1) covered
                 issue_dp(it);
@@ -790,7 +797,7 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
                         MMA_TS(tmem + COL_DV, tmem + COL_S + (ks >> 1) * 32 + (ks & 1) * 8,
                                sdesc_at(bo, static_cast<uint32_t>((ks * 2048) >> 4)), idKV, 1u);
                 }
-                if (it + 1 < NT) {
+                if (it + 1 < NTT) {
                     const int st1 = (it + 1) % STAGES;
                     if (!(ok = bounded_wait_warp(&bars->q_full[st1], ((it + 1) / STAGES) & 1, abort, lim))) break;
                     tc_fence_after();
@@ -838,7 +845,7 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
             sync_phase[s] ^= 1;
             return okw;
         };
-        for (int it = 0; it < NT; ++it) {
+        for (int it = 0; it < NTT; ++it) {
             const int b2 = it & 1;
             if (!bounded_wait_warp(&bars->dq_full[b2], (it >> 1) & 1, abort, lim)) break;
             tc_fence_after();
@@ -857,9 +864,10 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
             fence_proxy_async_smem();
             if (!wg_sync(1)) break;
             if (leader && lane == 0) {
-                const int i = i_begin + it;
-                float* dst = p.dq_acc + (static_cast<size_t>(bh) * p.n_pad + i * BQ) * D;
-                volatile int* sem = p.deterministic ? p.sems + static_cast<size_t>(bh) * nq + i : nullptr;
+                const int i = i_begin + it % NT;
+                const int qbh = kvbh * p.kv_group + it / NT;
+                float* dst = p.dq_acc + (static_cast<size_t>(qbh) * p.n_pad + i * BQ) * D;
+                volatile int* sem = p.deterministic ? p.sems + static_cast<size_t>(qbh) * nq + i : nullptr;
                 bool got = true;
                 if (sem) {
                     // contributions to one query tile are added in increasing key-tile order
@@ -903,8 +911,8 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
         float pr[32];
         bool ok = true;
 
-        for (int it = 0; it < NT; ++it) {
-            const int i = i_begin + it;
+        for (int it = 0; it < NTT; ++it) {
+            const int i = i_begin + it % NT;
             const int st = it % STAGES;
             const float* L2 = sL2 + st * 64 + cb;
             const float* Dv = sDv + st * 64 + cb;
@@ -971,7 +979,7 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
         if (ok) ok = wait_all(&bars->dkv_done, 0);
         if (ok) {
             tc_fence_after();
-            const size_t orow = (static_cast<size_t>(bh) * n + kidx) * D + g * 64;
+            const size_t orow = (static_cast<size_t>(kvbh) * n + kidx) * D + g * 64;
 #pragma unroll 1
             for (int which = 0; which < 2; ++which) {
                 const uint32_t tacc = tmem + lane_base + (which == 0 ? COL_DV : COL_DK) + g * 64;
@@ -1013,13 +1021,16 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
     const int BH = a.B * a.H;
     const int nq = (a.n + 127) / 128;
     const int n_pad = nq * 128;
-    // heads per group: Q, dO, K, V (bf16) and the fp32 dQ rows of one head take (8 + 4)·n·d
-    // bytes; keep a group's within ~48 MB of L2
+    // Main-kernel CTAs run per K/V head. Heads per group: a K/V head's K and V (4·n·d bytes) and
+    // its g query heads' Q, dO (4·n·d each) and fp32 dQ rows (4·n·d each); keep a group within
+    // ~48 MB of L2
+    const int BHkv = a.B * a.Hkv;
+    const int kvg = a.H / a.Hkv;
     int group;
     {
-        const long long per_head = 12LL * n_pad * D;
+        const long long per_head = (4LL + 8LL * kvg) * n_pad * D;
         long long g = (48LL << 20) / (per_head > 0 ? per_head : 1);
-        group = static_cast<int>(g < 1 ? 1 : (g > BH ? BH : g));
+        group = static_cast<int>(g < 1 ? 1 : (g > BHkv ? BHkv : g));
     }
     cudaError_t e;
     const cudaEvent_t* ev = a.phase_events;
@@ -1041,8 +1052,8 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
     if constexpr (D == 128) {
         CUtensorMap mq, mk, mv, mdo;
         if ((e = make_tmap_bf16(&mq, a.q, BH, a.n, D, q64::BQ)) != cudaSuccess) return e;
-        if ((e = make_tmap_bf16(&mk, a.k, BH, a.n, D)) != cudaSuccess) return e;
-        if ((e = make_tmap_bf16(&mv, a.v, BH, a.n, D)) != cudaSuccess) return e;
+        if ((e = make_tmap_bf16(&mk, a.k, BHkv, a.n, D)) != cudaSuccess) return e;
+        if ((e = make_tmap_bf16(&mv, a.v, BHkv, a.n, D)) != cudaSuccess) return e;
         if ((e = make_tmap_bf16(&mdo, a.dO, BH, a.n, D, q64::BQ)) != cudaSuccess) return e;
         e = cudaFuncSetAttribute(bwd_main_q64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  q64::SMEM);
@@ -1057,7 +1068,8 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
         kp.dv = static_cast<__nv_bfloat16*>(a.dv);
         kp.n = a.n;
         kp.n_pad = n_pad;
-        kp.BH = BH;
+        kp.BH = BHkv;
+        kp.kv_group = kvg;
         kp.nq = nq;
         kp.causal = a.causal;
         kp.deterministic = a.deterministic;
@@ -1065,7 +1077,7 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
         kp.scale = a.scale;
         kp.scale_log2 = a.scale * kBwdLog2e;
         kp.timeout_ns = a.timeout_ns;
-        const long long grid = static_cast<long long>(nq) * BH;
+        const long long grid = static_cast<long long>(nq) * BHkv;
         if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
         if (ev && ev[1] && (e = cudaEventRecord(ev[1], stream)) != cudaSuccess) return e;
         bwd_main_q64_kernel<<<static_cast<unsigned>(grid), q64::kThreads, q64::SMEM, stream>>>(
@@ -1075,8 +1087,8 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
     } else {
         CUtensorMap mq, mk, mv, mdo;
         if ((e = make_tmap_bf16(&mq, a.q, BH, a.n, D)) != cudaSuccess) return e;
-        if ((e = make_tmap_bf16(&mk, a.k, BH, a.n, D)) != cudaSuccess) return e;
-        if ((e = make_tmap_bf16(&mv, a.v, BH, a.n, D)) != cudaSuccess) return e;
+        if ((e = make_tmap_bf16(&mk, a.k, BHkv, a.n, D)) != cudaSuccess) return e;
+        if ((e = make_tmap_bf16(&mv, a.v, BHkv, a.n, D)) != cudaSuccess) return e;
         if ((e = make_tmap_bf16(&mdo, a.dO, BH, a.n, D)) != cudaSuccess) return e;
         e = cudaFuncSetAttribute(bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::SMEM);
@@ -1091,7 +1103,8 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
         kp.dv = static_cast<__nv_bfloat16*>(a.dv);
         kp.n = a.n;
         kp.n_pad = n_pad;
-        kp.BH = BH;
+        kp.BH = BHkv;
+        kp.kv_group = kvg;
         kp.nq = nq;
         kp.causal = a.causal;
         kp.deterministic = a.deterministic;
@@ -1099,7 +1112,7 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
         kp.scale = a.scale;
         kp.scale_log2 = a.scale * kBwdLog2e;
         kp.timeout_ns = a.timeout_ns;
-        const long long grid = static_cast<long long>(nq) * BH;
+        const long long grid = static_cast<long long>(nq) * BHkv;
         if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
         if (ev && ev[1] && (e = cudaEventRecord(ev[1], stream)) != cudaSuccess) return e;
         bwd_main_kernel<D><<<static_cast<unsigned>(grid), kBwdThreads, C::SMEM, stream>>>(

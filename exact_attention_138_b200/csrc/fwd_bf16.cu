@@ -65,6 +65,7 @@ struct FwdKParams {
     void* o;
     float* lse;
     int n, BH, n_pairs, causal, group;
+    int kv_group;     // query heads per K/V head (grouped-query attention); 1 for MHA
     float scale_log2;
     uint64_t timeout_ns;
 };
@@ -108,6 +109,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const int r_in = L - gbase * p.n_pairs;
     const int pair = p.n_pairs - 1 - r_in / gsize;
     const int bh = gbase + r_in % gsize;
+    const int kvbh = bh / p.kv_group;                     // (b, h / g) = (b·H + h) / g
     const int n = p.n;
     const int n_kv = (n + C::BN - 1) / C::BN;
     int T[2];
@@ -173,13 +175,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 mbar_arrive_expect_tx(&bars->k_full[s], C::TILE);
                 for (int ch = 0; ch < C::NCH; ++ch)
                     tma_load_3d(sK + s * C::TILE + ch * C::CHUNK, &tmK, &bars->k_full[s],
-                                ch * C::CW, jj * C::BN, bh);
+                                ch * C::CW, jj * C::BN, kvbh);
                 issued = 2 * jj + 1;
                 if (f > 0 && !bounded_wait(&bars->v_empty[s], (f - 1) & 1, abort, lim)) break;
                 mbar_arrive_expect_tx(&bars->v_full[s], C::TILE);
                 for (int ch = 0; ch < C::NCH; ++ch)
                     tma_load_3d(sV + s * C::TILE + ch * C::CHUNK, &tmV, &bars->v_full[s],
-                                ch * C::CW, jj * C::BN, bh);
+                                ch * C::CW, jj * C::BN, kvbh);
                 issued = 2 * jj + 2;
             }
             if (*abort) {
@@ -453,8 +455,9 @@ cudaError_t launch_fwd_bf16_d(const FwdArgs& a, cudaStream_t stream) {
     const int BH = a.B * a.H;
     cudaError_t e;
     if ((e = make_tmap_bf16(&mq, a.q, BH, a.n, D)) != cudaSuccess) return e;
-    if ((e = make_tmap_bf16(&mk, a.k, BH, a.n, D)) != cudaSuccess) return e;
-    if ((e = make_tmap_bf16(&mv, a.v, BH, a.n, D)) != cudaSuccess) return e;
+    const int BHkv = a.B * a.Hkv;
+    if ((e = make_tmap_bf16(&mk, a.k, BHkv, a.n, D)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16(&mv, a.v, BHkv, a.n, D)) != cudaSuccess) return e;
     e = cudaFuncSetAttribute(fwd_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM);
     if (e != cudaSuccess) return e;
@@ -466,6 +469,7 @@ cudaError_t launch_fwd_bf16_d(const FwdArgs& a, cudaStream_t stream) {
     const int nq = (a.n + 127) / 128;
     kp.n_pairs = (nq + 1) / 2;
     kp.causal = a.causal;
+    kp.kv_group = a.H / a.Hkv;
     // heads per group: K and V of one head take 4·n·d bytes; keep a group's within ~32 MB of L2
     {
         const long long per_head = 4LL * a.n * D;

@@ -29,7 +29,7 @@ __global__ void __launch_bounds__(256) fwd_f32_kernel(const float* __restrict__ 
                                                       const float* __restrict__ V,
                                                       float* __restrict__ O,
                                                       float* __restrict__ lse, int n, int n_qtiles,
-                                                      float scale, int causal) {
+                                                      float scale, int causal, int kv_group) {
     constexpr int DP = D + 1;
     constexpr int PP = kBN + 1;
     constexpr int OC = D / 16;
@@ -43,6 +43,7 @@ __global__ void __launch_bounds__(256) fwd_f32_kernel(const float* __restrict__ 
     const int bh = blockIdx.y;
     const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
     const size_t base = static_cast<size_t>(bh) * n * D;
+    const size_t kvbase = static_cast<size_t>(bh / kv_group) * n * D;   // grouped-query K/V head
     const int q0 = qt * kBM;
 
     for (int idx = tid; idx < kBM * D; idx += 256) {
@@ -67,7 +68,7 @@ __global__ void __launch_bounds__(256) fwd_f32_kernel(const float* __restrict__ 
         for (int idx = tid; idx < kBN * D; idx += 256) {
             const int r = idx / D, c = idx % D;
             const bool in = k0 + r < n;
-            const size_t g = base + static_cast<size_t>(k0 + r) * D + c;
+            const size_t g = kvbase + static_cast<size_t>(k0 + r) * D + c;
             Ks[r * DP + c] = in ? K[g] : 0.f;
             Vs[r * D + c] = in ? V[g] : 0.f;
         }
@@ -168,7 +169,7 @@ cudaError_t launch_fwd_f32_d(const FwdArgs& a, cudaStream_t stream) {
     fwd_f32_kernel<D><<<grid, 256, smem, stream>>>(
         static_cast<const float*>(a.q), static_cast<const float*>(a.k),
         static_cast<const float*>(a.v), static_cast<float*>(a.o), a.lse, a.n, nqt, a.scale,
-        a.causal);
+        a.causal, a.H / a.Hkv);
     return cudaGetLastError();
 }
 

@@ -14,6 +14,7 @@ struct FwdArgs {
     void* o;
     float* lse;
     int B, H, n, d;
+    int Hkv;          // K/V heads; query head h reads K/V head h / (H / Hkv)
     float scale;
     int causal;
     uint64_t timeout_ns;
@@ -30,6 +31,7 @@ struct BwdArgs {
     void* dk;
     void* dv;
     int B, H, n, d;
+    int Hkv;          // K/V heads (dk, dv have Hkv heads)
     float scale;
     int causal;
     int deterministic;

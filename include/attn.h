@@ -68,6 +68,15 @@ int attn_version(void);
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              int B, int H, int n, int d, float scale, int causal, int dtype, void* stream);
 
+/* Grouped-query attention ("Attention Mechanism: Revolusi Representasi Sequence", §12 "GQA vs
+ * MQA — KV Cache Optimization"): k and v have Hkv heads, (B, Hkv, n, d); query head h (of H) uses
+ * K/V head h / (H / Hkv), exactly as if K and V were expanded with repeat_interleave(H/Hkv, dim=1)
+ * (no copy is made). Hkv = H is attn_fwd; Hkv = 1 is multi-query attention. H must be a multiple
+ * of Hkv (else ATTN_ERR_INVALID). Everything else as attn_fwd. */
+int attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int H, int Hkv, int n, int d, float scale, int causal, int dtype,
+                 void* stream);
+
 /* Bytes of device workspace attn_bwd needs for these sizes: the D vector and the LSE·log2(e)
  * vector (B·H·n fp32 each, padded per head to a multiple of 128 rows) and the fp32 dQ accumulator
  * (B·H·n·d fp32, padded the same way), each rounded up to 256 bytes; with deterministic != 0 also
@@ -85,6 +94,15 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
              const float* lse, void* dq, void* dk, void* dv,
              int B, int H, int n, int d, float scale, int causal, int dtype, int deterministic,
              void* workspace, size_t ws_bytes, void* stream);
+
+/* Backward pass of attn_fwd_gqa: k, v, dk, dv have Hkv heads; dk and dv of a K/V head are the sums
+ * over its H/Hkv query heads (the gradient through the expansion). The workspace is
+ * attn_bwd_workspace_bytes(B, H, n, d, deterministic) with the QUERY head count H. Everything
+ * else as attn_bwd. */
+int attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                 const float* lse, void* dq, void* dk, void* dv,
+                 int B, int H, int Hkv, int n, int d, float scale, int causal, int dtype,
+                 int deterministic, void* workspace, size_t ws_bytes, void* stream);
 
 /* Backward pass without a caller workspace, for callers that cannot allocate device memory where
  * they run it (e.g. code inside a host framework that owns all device allocations, or a loop that

@@ -11,7 +11,8 @@ FAKE = 1 << 20          # an aligned, never-dereferenced pointer value (validati
 
 def test_every_declared_function_is_exported():
     names = ea.declared_functions()
-    assert {"attn_fwd", "attn_bwd", "attn_bwd_workspace_bytes", "attn_get_device_status",
+    assert {"attn_fwd", "attn_bwd", "attn_fwd_gqa", "attn_bwd_gqa", "attn_bwd_noalloc",
+            "attn_bwd_workspace_bytes", "attn_get_device_status",
             "attn_error_string", "attn_version", "attn_set_wait_timeout_us",
             "attn_selftest_wait_timeout"} <= set(names)
     lib = ea.library()
@@ -96,3 +97,13 @@ def test_selftest_rejects_bad_limit():
 def test_timeout_setter_roundtrip():
     old = ea.attn_set_wait_timeout_us(5)
     assert ea.attn_set_wait_timeout_us(old) == 100      # raised to the 100 us floor
+
+
+def test_gqa_rejects_head_counts_that_do_not_divide():
+    a = [ctypes.c_void_p(FAKE)] * 5
+    assert ea.attn_fwd_gqa(*a, 1, 6, 4, 128, 64, 0.125, 0, ea.ATTN_BF16, None) == ea.ATTN_ERR_INVALID
+    assert ea.attn_fwd_gqa(*a, 1, 6, 0, 128, 64, 0.125, 0, ea.ATTN_BF16, None) == ea.ATTN_ERR_INVALID
+    need = ea.attn_bwd_workspace_bytes(1, 6, 128, 64, 0)
+    b = [ctypes.c_void_p(FAKE)] * 9
+    assert ea.attn_bwd_gqa(*b, 1, 6, 4, 128, 64, 0.125, 0, ea.ATTN_BF16, 0, ctypes.c_void_p(FAKE),
+                           need, None) == ea.ATTN_ERR_INVALID

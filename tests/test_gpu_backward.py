@@ -94,3 +94,26 @@ def test_backward_full_size_invariants(full_run):
     assert (torch.linalg.norm(sdk) / torch.linalg.norm(scale_ref)).item() <= TOL_GRAD_REL
     for t in (dq, dk, dv):
         assert torch.isfinite(t).all()
+
+
+@pytest.mark.parametrize("shape,Hkv,causal,det", [((1, 4, 300, 128), 2, True, False),
+                                                  ((2, 8, 256, 128), 1, True, False),
+                                                  ((1, 6, 200, 64), 3, False, False),
+                                                  ((1, 4, 383, 128), 2, True, True),
+                                                  ((1, 4, 129, 32), 4, True, False)])
+def test_gqa_forward_backward(cuda_device, shape, Hkv, causal, det):
+    # grouped-query attention ("Attention Mechanism ...", §12): K/V with Hkv heads, no copy
+    B, H, n, d = shape
+    q, do = attn_inputs.random_draws(shape, seed=31, count=2)
+    k, v = attn_inputs.random_draws((B, Hkv, n, d), seed=32, count=2)
+    scale = 1.0 / math.sqrt(d)
+    o, lse, dev = cuda_forward(q, k, v, causal, scale)
+    ro, rlse = oracle.fwd_gqa(q, k, v, scale, causal)
+    assert np.abs(to_np(o) - ro).max() <= 1e-2
+    assert np.abs(to_np(lse) - rlse).max() <= 1e-3
+    dq, dk, dv = cuda_backward(dev, o, lse, do, causal, scale, deterministic=det)
+    assert tuple(dk.shape) == (B, Hkv, n, d) and tuple(dv.shape) == (B, Hkv, n, d)
+    rq, rk, rv, _ = oracle.bwd_gqa(q, k, v, do, scale, causal)
+    assert grad_close(to_np(dq), rq)
+    assert grad_close(to_np(dk), rk)
+    assert grad_close(to_np(dv), rv)

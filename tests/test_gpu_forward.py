@@ -93,3 +93,13 @@ def test_forward_repeatable(cuda_device):
     o1, l1, _ = cuda_forward(q, k, v, True, 0.1)
     o2, l2, _ = cuda_forward(q, k, v, True, 0.1)
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("Hkv", [1, 2])
+def test_gqa_forward_fp32(cuda_device, Hkv):
+    q = attn_inputs.random_draws((1, 4, 200, 64), dtype="fp32", seed=41, count=1)[0]
+    k, v = attn_inputs.random_draws((1, Hkv, 200, 64), dtype="fp32", seed=42, count=2)
+    o, lse, _ = cuda_forward(q, k, v, True, 0.125)
+    ro, rlse = oracle.fwd_gqa(q, k, v, 0.125, True)
+    assert np.abs(to_np(o) - ro).max() <= TOL_O["fp32"]
+    assert np.abs(to_np(lse) - rlse).max() <= TOL_LSE["fp32"]
