@@ -73,12 +73,16 @@ def _load():
                                               f64p, f64p]
         lib.oracle_bwd_key_rows.argtypes = [f32p, f32p, f32p, f32p, I, I, I, I, D, I,
                                             ctypes.c_long, i32p, I, f64p, f64p]
+        lib.oracle_fwd_ex.argtypes = [f32p, f32p, f32p, I, I, I, I, I, D, I, I, f64p, f64p]
+        lib.oracle_bwd_ex.argtypes = [f32p, f32p, f32p, f32p, I, I, I, I, I, D, I, I, f64p, f64p,
+                                      f64p]
         lib.oracle_score_matrix_bytes.argtypes = [D, D, D, D]
         lib.oracle_score_matrix_bytes.restype = D
         lib.oracle_num_threads.restype = I
         lib.oracle_set_num_threads.argtypes = [I]
         for name in ("oracle_fwd", "oracle_fwd_rowtiled", "oracle_fwd_online", "oracle_fwd_rows",
-                     "oracle_bwd", "oracle_bwd_query_rows", "oracle_bwd_key_rows"):
+                     "oracle_bwd", "oracle_bwd_query_rows", "oracle_bwd_key_rows", "oracle_fwd_ex",
+                     "oracle_bwd_ex"):
             getattr(lib, name).restype = I
         _lib = lib
         return lib
@@ -228,3 +232,38 @@ def bwd_gqa(q, k, v, do, scale, causal=False):
     dk = dk.reshape(B, Hkv, g, n, d).sum(axis=2)
     dv = dv.reshape(B, Hkv, g, n, d).sum(axis=2)
     return dq, dk, dv, D
+
+
+# ---------------------------------------------------------------------------------------------
+# Mask and shape variants ("Attention Mechanism ...", §4.5 sliding window ±w; §4.2 cross-attention
+# with different query / key lengths). Query i is aligned with key i + (nk - nq); key j is visible
+# iff (i + off) - wl <= j <= (i + off) + wr, negative = unbounded. Rows that see no key: O = 0,
+# LSE = -inf. Optional kv heads (grouped-query) follow the repeat_interleave recipe.
+# ---------------------------------------------------------------------------------------------
+def fwd_ex(q, k, v, scale, window_left=-1, window_right=-1):
+    q = _f32(q)
+    H = q.shape[1]
+    k, v = _expand_kv(k, H), _expand_kv(v, H)
+    B, _, nq, d = q.shape
+    nk = k.shape[2]
+    o = np.empty(q.shape, np.float64)
+    lse = np.empty(q.shape[:-1], np.float64)
+    _check(_load().oracle_fwd_ex(q, k, v, B, H, nq, nk, d, float(scale), int(window_left),
+                                 int(window_right), o, lse), "oracle_fwd_ex")
+    return o, lse
+
+
+def bwd_ex(q, k, v, do, scale, window_left=-1, window_right=-1):
+    """(dQ, dK, dV): dK, dV with k's head count (summed over grouped query heads)."""
+    q, do = _f32(q), _f32(do)
+    B, H, nq, d = q.shape
+    Hkv = _f32(k).shape[1]
+    ke, ve = _expand_kv(k, H), _expand_kv(v, H)
+    nk = ke.shape[2]
+    dq = np.empty(q.shape, np.float64)
+    dk = np.empty(ke.shape, np.float64)
+    dv = np.empty(ke.shape, np.float64)
+    _check(_load().oracle_bwd_ex(q, ke, ve, do, B, H, nq, nk, d, float(scale), int(window_left),
+                                 int(window_right), dq, dk, dv), "oracle_bwd_ex")
+    g = H // Hkv
+    return dq, dk.reshape(B, Hkv, g, nk, d).sum(2), dv.reshape(B, Hkv, g, nk, d).sum(2)

@@ -40,6 +40,9 @@
  *                       dP = dO·V^T, D_i = sum_j P_ij dP_ij, dS = P∘(dP - D), the gradients are
  *                       dV = P^T·dO, dQ = scale·dS·K, dK = scale·dS^T·Q.
  *   oracle_bwd_query_rows / oracle_bwd_key_rows   the same derivative for sampled rows.
+ *   oracle_fwd_ex / oracle_bwd_ex   the definition and its derivative with a generalized mask
+ *                       (sliding window of §4.5 "Sparse Attention", causal, none) and different
+ *                       query / key lengths (cross-attention, §4.2); see the block before them.
  *   oracle_score_matrix_bytes   the score-matrix size B·H·n²·e of "Calculateur de mémoire
  *                       d'attention", section "La formule".
  *
@@ -477,4 +480,151 @@ int oracle_bwd_key_rows(const float* Q, const float* K, const float* V, const fl
     }
     free(KT); free(Psel); free(dSsel);
     return fail ? ORC_ERR_MEM : ORC_OK;
+}
+
+/* ------------------------------------------------------------------------------------------
+ * Mask and shape variants: sliding-window attention ("Attention Mechanism ...", §4.5 Sparse
+ * Attention, "Sliding Window: only neighbours ±w") and cross-attention with different query and
+ * key lengths (§4.2: Q from the decoder, K and V from the encoder).
+ * Query i (of nq) is aligned with key i + (nk - nq) (the last query with the last key); key j is
+ * visible iff  (i + off) - wl <= j <= (i + off) + wr, where a negative wl or wr means unbounded.
+ * (wl, wr) = (-1, 0) is the causal mask of §4.4 when nq = nk; (-1, -1) is no mask; (w, w) is the
+ * page's ±w window. A row that sees no key gets O = 0 and LSE = -inf.
+ * Q is (B,H,nq,d); K and V are (B,H,nk,d).
+ * ------------------------------------------------------------------------------------------ */
+static int visible(long i, long j, long off, long wl, long wr) {
+    const long c = i + off;
+    if (wl >= 0 && j < c - wl) return 0;
+    if (wr >= 0 && j > c + wr) return 0;
+    return 1;
+}
+
+/* Definition for one query row over nk keys with the generalized mask. */
+static void attend_row_ex(const float* qi, const double* KT, const float* V, int nk, int d,
+                          double scale, long i, long off, long wl, long wr, double* s, double* o,
+                          double* lse) {
+    for (int j = 0; j < nk; ++j) s[j] = 0.0;
+    for (int c = 0; c < d; ++c) {
+        const double qc = (double)qi[c];
+        const double* kc = KT + (size_t)c * nk;
+        for (int j = 0; j < nk; ++j) s[j] += qc * kc[j];
+    }
+    int any = 0;
+    for (int j = 0; j < nk; ++j) {
+        if (visible(i, j, off, wl, wr)) { s[j] *= scale; any = 1; }
+        else s[j] = -INFINITY;
+    }
+    if (!any) {
+        for (int c = 0; c < d; ++c) o[c] = 0.0;
+        *lse = -INFINITY;
+        return;
+    }
+    double m, l;
+    softmax_row(s, nk, &m, &l);
+    pv_row(s, V, nk, d, o);
+    *lse = m + log(l);
+}
+
+int oracle_fwd_ex(const float* Q, const float* K, const float* V, int B, int H, int nq, int nk,
+                  int d, double scale, int wl, int wr, double* O, double* lse) {
+    if (B < 1 || H < 1 || nq < 1 || nk < 1 || d < 1) return ORC_ERR_ARG;
+    const long off = (long)nk - (long)nq;
+    int fail = 0;
+    for (long bh = 0; bh < (long)B * H; ++bh) {
+        double* KT = transpose_keys(K + (size_t)bh * nk * d, nk, d);
+        if (!KT) return ORC_ERR_MEM;
+#pragma omp parallel
+        {
+            double* s = (double*)malloc((size_t)nk * sizeof(double));
+            if (!s) {
+#pragma omp atomic write
+                fail = 1;
+            } else {
+#pragma omp for schedule(static)
+                for (int i = 0; i < nq; ++i)
+                    attend_row_ex(Q + ((size_t)bh * nq + i) * d, KT, V + (size_t)bh * nk * d, nk, d,
+                                  scale, i, off, wl, wr, s, O + ((size_t)bh * nq + i) * d,
+                                  lse + (size_t)bh * nq + i);
+            }
+            free(s);
+        }
+        free(KT);
+        if (fail) return ORC_ERR_MEM;
+    }
+    return ORC_OK;
+}
+
+/* Exact derivative with the generalized mask; P and dS of each (b,h) materialised (nq x nk). */
+int oracle_bwd_ex(const float* Q, const float* K, const float* V, const float* dO, int B, int H,
+                  int nq, int nk, int d, double scale, int wl, int wr, double* dQ, double* dK,
+                  double* dV) {
+    if (B < 1 || H < 1 || nq < 1 || nk < 1 || d < 1) return ORC_ERR_ARG;
+    const long off = (long)nk - (long)nq;
+    for (long bh = 0; bh < (long)B * H; ++bh) {
+        const float* Qh = Q + (size_t)bh * nq * d;
+        const float* dOh = dO + (size_t)bh * nq * d;
+        const float* Kh = K + (size_t)bh * nk * d;
+        const float* Vh = V + (size_t)bh * nk * d;
+        double* KT = transpose_keys(Kh, nk, d);
+        double* P = (double*)malloc((size_t)nq * nk * sizeof(double));
+        double* dS = (double*)malloc((size_t)nq * nk * sizeof(double));
+        if (!KT || !P || !dS) { free(KT); free(P); free(dS); return ORC_ERR_MEM; }
+#pragma omp parallel for schedule(static)
+        for (int i = 0; i < nq; ++i) {
+            double* p = P + (size_t)i * nk;
+            double* ds = dS + (size_t)i * nk;
+            /* P row: the softmax of the masked scores (all zero for a row with no key) */
+            for (int j = 0; j < nk; ++j) p[j] = 0.0;
+            for (int c = 0; c < d; ++c) {
+                const double qc = (double)Qh[(size_t)i * d + c];
+                const double* kc = KT + (size_t)c * nk;
+                for (int j = 0; j < nk; ++j) p[j] += qc * kc[j];
+            }
+            int any = 0;
+            for (int j = 0; j < nk; ++j) {
+                if (visible(i, j, off, wl, wr)) { p[j] *= scale; any = 1; }
+                else p[j] = -INFINITY;
+            }
+            if (any) {
+                double m, l;
+                softmax_row(p, nk, &m, &l);
+            } else {
+                for (int j = 0; j < nk; ++j) p[j] = 0.0;
+            }
+            double D = 0.0;
+            for (int j = 0; j < nk; ++j) {
+                double dp = 0.0;
+                for (int c = 0; c < d; ++c) dp += (double)dOh[(size_t)i * d + c] * (double)Vh[(size_t)j * d + c];
+                ds[j] = dp;
+                D += p[j] * dp;
+            }
+            for (int j = 0; j < nk; ++j) ds[j] = p[j] * (ds[j] - D);
+        }
+#pragma omp parallel for schedule(static)
+        for (int i = 0; i < nq; ++i) {
+            double* g = dQ + ((size_t)bh * nq + i) * d;
+            for (int c = 0; c < d; ++c) g[c] = 0.0;
+            for (int j = 0; j < nk; ++j) {
+                const double w = dS[(size_t)i * nk + j];
+                for (int c = 0; c < d; ++c) g[c] += w * (double)Kh[(size_t)j * d + c];
+            }
+            for (int c = 0; c < d; ++c) g[c] *= scale;
+        }
+#pragma omp parallel for schedule(static)
+        for (int j = 0; j < nk; ++j) {
+            double* gk = dK + ((size_t)bh * nk + j) * d;
+            double* gv = dV + ((size_t)bh * nk + j) * d;
+            for (int c = 0; c < d; ++c) { gk[c] = 0.0; gv[c] = 0.0; }
+            for (int i = 0; i < nq; ++i) {
+                const double ws = dS[(size_t)i * nk + j], wp = P[(size_t)i * nk + j];
+                for (int c = 0; c < d; ++c) {
+                    gk[c] += ws * (double)Qh[(size_t)i * d + c];
+                    gv[c] += wp * (double)dOh[(size_t)i * d + c];
+                }
+            }
+            for (int c = 0; c < d; ++c) gk[c] *= scale;
+        }
+        free(KT); free(P); free(dS);
+    }
+    return ORC_OK;
 }

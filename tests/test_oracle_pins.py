@@ -387,3 +387,67 @@ def test_mqa_heads_with_equal_queries_agree():
     _, dk1, dv1, _ = oracle.bwd(qh, k, v, doh, 0.35, True)
     np.testing.assert_allclose(dv, 3 * dv1, rtol=0, atol=1e-13)
     np.testing.assert_allclose(dk, 3 * dk1, rtol=0, atol=1e-13)
+
+
+# --------------------------------------------------------------------------------------------
+# Mask and shape variants (§4.5 sliding window, §4.2 cross-attention)
+# --------------------------------------------------------------------------------------------
+def _torch_masked(q, k, v, do, scale, wl, wr):
+    Q, K, V = (torch.from_numpy(x.astype(np.float64)).requires_grad_() for x in (q, k, v))
+    nq, nk = q.shape[2], k.shape[2]
+    i = torch.arange(nq)[:, None] + (nk - nq)
+    j = torch.arange(nk)[None, :]
+    vis = torch.ones(nq, nk, dtype=torch.bool)
+    if wl >= 0:
+        vis &= j >= i - wl
+    if wr >= 0:
+        vis &= j <= i + wr
+    S = (Q @ K.transpose(-1, -2) * scale).masked_fill(~vis, float("-inf"))
+    rows = vis.any(-1)
+    P = torch.softmax(S.masked_fill(~rows[:, None], 0.0), -1) * rows[:, None]
+    O = P @ V
+    O.backward(torch.from_numpy(do.astype(np.float64)))
+    lse = torch.logsumexp(S, -1)
+    return O.detach().numpy(), lse.detach().numpy(), Q.grad.numpy(), K.grad.numpy(), V.grad.numpy()
+
+
+def test_ex_reduces_to_causal_and_full_bitwise():
+    q, k, v, do = (_rand((1, 2, 70, 16), s) for s in (80, 81, 82, 83))
+    for causal, (wl, wr) in ((True, (-1, 0)), (False, (-1, -1))):
+        o, lse = oracle.fwd(q, k, v, 0.2, causal)
+        oe, lsee = oracle.fwd_ex(q, k, v, 0.2, wl, wr)
+        assert np.array_equal(o, oe) and np.array_equal(lse, lsee)
+        rq, rk, rv, _ = oracle.bwd(q, k, v, do, 0.2, causal)
+        eq, ek, ev = oracle.bwd_ex(q, k, v, do, 0.2, wl, wr)
+        np.testing.assert_allclose(eq, rq, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(ek, rk, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(ev, rv, rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("nq,nk,wl,wr", [(40, 40, 5, 5), (40, 40, 7, 0), (30, 50, -1, -1),
+                                         (50, 30, -1, 0), (30, 50, 4, 2), (45, 20, 3, 0)])
+def test_ex_matches_torch_with_explicit_mask(nq, nk, wl, wr):
+    q, do = _rand((1, 2, nq, 8), 84), _rand((1, 2, nq, 8), 85)
+    k, v = _rand((1, 2, nk, 8), 86), _rand((1, 2, nk, 8), 87)
+    o, lse = oracle.fwd_ex(q, k, v, 0.3, wl, wr)
+    dq, dk, dv = oracle.bwd_ex(q, k, v, do, 0.3, wl, wr)
+    ro, rlse, rq, rk, rv = _torch_masked(q, k, v, do, 0.3, wl, wr)
+    np.testing.assert_allclose(o, ro, rtol=0, atol=1e-13)
+    np.testing.assert_array_equal(np.isneginf(lse), np.isneginf(rlse))
+    fin = np.isfinite(rlse)
+    np.testing.assert_allclose(lse[fin], rlse[fin], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dq, rq, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dk, rk, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dv, rv, rtol=0, atol=1e-12)
+
+
+def test_zero_window_returns_own_value_and_empty_rows_are_zero():
+    q, k, v = (_rand((1, 1, 20, 8), s) for s in (88, 89, 90))
+    o, lse = oracle.fwd_ex(q, k, v, 0.5, 0, 0)          # each query sees only its own key
+    np.testing.assert_array_equal(o, v.astype(np.float64))
+    np.testing.assert_allclose(lse, 0.5 * (q.astype(np.float64) * k).sum(-1), rtol=0, atol=1e-14)
+    # 20 queries on 8 keys, bottom-right aligned causal: the first 12 queries see nothing
+    q2 = _rand((1, 1, 20, 8), 91)
+    o2, lse2 = oracle.fwd_ex(q2, k[:, :, :8], v[:, :, :8], 0.5, -1, 0)
+    assert np.all(o2[0, 0, :12] == 0) and np.all(np.isneginf(lse2[0, 0, :12]))
+    assert np.all(np.isfinite(lse2[0, 0, 12:]))
