@@ -6,9 +6,11 @@ memory and streams come from PyTorch, every step of the computation runs in the 
 CUDA kernels. There is no CPU fallback: if the library is missing the import fails.
 
     O = softmax(scale · Q·K^T + M) · V      ("Attention Mechanism: Revolusi Representasi
-    Sequence", §3 Steps 1-4; causal mask M of §4.4)
+    Sequence", §3 Steps 1-4; causal mask M of §4.4, sliding window of §4.5, cross-attention
+    with different query / key lengths of §4.2)
 
-Raw entry points keep the C names (``attn_fwd``, ``attn_bwd``, ``attn_bwd_workspace_bytes``,
+Raw entry points keep the C names (``attn_fwd``, ``attn_fwd_gqa``, ``attn_fwd_ex``, ``attn_bwd``,
+``attn_bwd_gqa``, ``attn_bwd_ex``, ``attn_bwd_workspace_bytes``,
 ``attn_get_device_status``, ``attn_set_wait_timeout_us``, ``attn_selftest_wait_timeout``,
 ``attn_error_string``, ``attn_version``); ``forward`` / ``backward`` wrap them for torch tensors.
 """
@@ -46,6 +48,11 @@ _lib.attn_fwd_gqa.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _
 _lib.attn_bwd_gqa.restype = _i
 _lib.attn_bwd_gqa.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f,
                               _i, _i, _i, _vp, _sz, _vp]
+_lib.attn_fwd_ex.restype = _i
+_lib.attn_fwd_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i, _i, _vp]
+_lib.attn_bwd_ex.restype = _i
+_lib.attn_bwd_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                             _f, _i, _i, _i, _i, _vp, _sz, _vp]
 _lib.attn_bwd_workspace_bytes.restype = _sz
 _lib.attn_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
 _lib.attn_bwd.restype = _i
@@ -100,6 +107,19 @@ def attn_bwd_gqa(q, k, v, o, dO, lse, dq, dk, dv, B, H, Hkv, n, d, scale, causal
                  deterministic, workspace, ws_bytes, stream) -> int:
     return _lib.attn_bwd_gqa(q, k, v, o, dO, lse, dq, dk, dv, B, H, Hkv, n, d, scale, causal,
                              dtype, deterministic, workspace, ws_bytes, stream)
+
+
+def attn_fwd_ex(q, k, v, o, lse, B, H, Hkv, nq, nk, d, scale, window_left, window_right, dtype,
+                stream) -> int:
+    return _lib.attn_fwd_ex(q, k, v, o, lse, B, H, Hkv, nq, nk, d, scale, window_left,
+                            window_right, dtype, stream)
+
+
+def attn_bwd_ex(q, k, v, o, dO, lse, dq, dk, dv, B, H, Hkv, nq, nk, d, scale, window_left,
+                window_right, dtype, deterministic, workspace, ws_bytes, stream) -> int:
+    return _lib.attn_bwd_ex(q, k, v, o, dO, lse, dq, dk, dv, B, H, Hkv, nq, nk, d, scale,
+                            window_left, window_right, dtype, deterministic, workspace, ws_bytes,
+                            stream)
 
 
 def attn_bwd_workspace_bytes(B, H, n, d, deterministic) -> int:
@@ -167,31 +187,51 @@ def _check(rc, where):
 
 
 def _kv_heads(q, k, v):
-    """K/V head count: equal to q's (multi-head) or a divisor of it (grouped-query, k and v of
-    shape (B, Hkv, n, d))."""
+    """(K/V head count, key length): heads equal to q's (multi-head) or a divisor of it
+    (grouped-query); k and v of shape (B, Hkv, nk, d)."""
     B, H, n, d = _dims(q)
     kd = _dims(k)
     if k.dim() != q.dim() or v.shape != k.shape or k.dtype != q.dtype or v.dtype != q.dtype:
         raise ValueError("k and v must match each other and q's dtype")
-    if kd[0] != B or kd[2] != n or kd[3] != d or H % kd[1] != 0:
-        raise ValueError("k, v must be (B, Hkv, n, d) with H a multiple of Hkv")
-    return kd[1]
+    if kd[0] != B or kd[3] != d or H % kd[1] != 0:
+        raise ValueError("k, v must be (B, Hkv, nk, d) with H a multiple of Hkv")
+    return kd[1], kd[2]
 
 
-def forward(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None):
+def _window(causal, window):
+    """(window_left, window_right): None -> causal (-1, 0) or none (-1, -1); causal=True with a
+    window caps the right side at 0. Negative = unbounded."""
+    if window is None:
+        return (-1, 0) if causal else (-1, -1)
+    wl, wr = (int(window[0]), int(window[1]))
+    wl = -1 if wl < 0 else wl
+    wr = -1 if wr < 0 else wr
+    if causal:
+        wr = 0
+    return wl, wr
+
+
+def forward(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None, window=None):
     """O, LSE = attention(q, k, v). q: contiguous CUDA tensor (B,H,n,d) or (n,d), bf16 or fp32;
-    k, v: same shape, or (B,Hkv,n,d) for grouped-query attention. Returns O (same dtype/shape as
-    q) and LSE (fp32, (B,H,n))."""
+    k, v: same shape, or (B,Hkv,nk,d) for grouped-query attention and / or another key length
+    (cross-attention). window=(left, right): key j visible to query i iff
+    i+nk-nq-left <= j <= i+nk-nq+right (negative = unbounded); causal=True is (-1, 0).
+    Returns O (same dtype/shape as q) and LSE (fp32, (B,H,nq)); a query that sees no key gets
+    O = 0 and LSE = -inf."""
     import torch
     B, H, n, d = _dims(q)
-    Hkv = _kv_heads(q, k, v)
+    Hkv, nk = _kv_heads(q, k, v)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, n), dtype=torch.float32, device=q.device)
-    if Hkv == H:
+    if nk != n or window is not None:
+        wl, wr = _window(causal, window)
+        rc = attn_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Hkv, n, nk, d,
+                         float(scale), wl, wr, _dtype_code(q), _stream_handle(stream))
+    elif Hkv == H:
         rc = attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, n, d, float(scale),
                       int(bool(causal)), _dtype_code(q), _stream_handle(stream))
     else:
@@ -202,12 +242,13 @@ def forward(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None):
 
 
 def backward(q, k, v, o, do, lse, causal=False, scale=None, deterministic=False, dq=None,
-             dk=None, dv=None, workspace=None, stream=None):
-    """dQ, dK, dV of attention given dO (bf16 tensors, lse from `forward`). For grouped-query
-    inputs dK, dV have k's (B, Hkv, n, d) shape and sum over each group's query heads."""
+             dk=None, dv=None, workspace=None, stream=None, window=None):
+    """dQ, dK, dV of attention given dO (bf16 tensors, lse from `forward` with the same causal /
+    window arguments). dK, dV have k's (B, Hkv, nk, d) shape and, for grouped-query inputs, sum
+    over each group's query heads."""
     import torch
     B, H, n, d = _dims(q)
-    Hkv = _kv_heads(q, k, v)
+    Hkv, nk = _kv_heads(q, k, v)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     dq = torch.empty_like(q) if dq is None else dq
@@ -217,7 +258,13 @@ def backward(q, k, v, o, do, lse, causal=False, scale=None, deterministic=False,
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = workspace.numel() * workspace.element_size()
-    if Hkv == H:
+    if nk != n or window is not None:
+        wl, wr = _window(causal, window)
+        rc = attn_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
+                         _ptr(dk), _ptr(dv), B, H, Hkv, n, nk, d, float(scale), wl, wr,
+                         _dtype_code(q), int(bool(deterministic)), _ptr(workspace), ws_bytes,
+                         _stream_handle(stream))
+    elif Hkv == H:
         rc = attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk),
                       _ptr(dv), B, H, n, d, float(scale), int(bool(causal)), _dtype_code(q),
                       int(bool(deterministic)), _ptr(workspace), ws_bytes, _stream_handle(stream))

@@ -132,18 +132,21 @@ unsigned attn_set_wait_timeout_us(unsigned us) {
 }
 
 static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                    int H, int Hkv, int n, int d, float scale, int causal, int dtype, void* stream) {
+                    int H, int Hkv, int nq, int nk, int d, float scale, int wl, int wr, int dtype,
+                    void* stream) {
     if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID;
-    int rc = validate_common(B, H, n, d, scale, dtype);
+    int rc = validate_common(B, H, nq, d, scale, dtype);
     if (rc) return rc;
+    if (nk < 1) return ATTN_ERR_INVALID;
     if (Hkv < 1 || H % Hkv != 0) return ATTN_ERR_INVALID;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
         return ATTN_ERR_INVALID;
     FwdArgs a;
     a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
-    a.B = B; a.H = H; a.n = n; a.d = d; a.Hkv = Hkv;
+    a.B = B; a.H = H; a.nq = nq; a.nk = nk; a.d = d; a.Hkv = Hkv;
     a.scale = scale;
-    a.causal = causal ? 1 : 0;
+    a.wl = wl < 0 ? -1 : wl;
+    a.wr = wr < 0 ? -1 : wr;
     a.timeout_ns = static_cast<uint64_t>(g_timeout_us.load()) * 1000ull;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = (dtype == ATTN_BF16) ? launch_fwd_bf16(a, s) : launch_fwd_f32(a, s);
@@ -152,12 +155,20 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
              int n, int d, float scale, int causal, int dtype, void* stream) {
-    return fwd_impl(q, k, v, o, lse, B, H, H, n, d, scale, causal, dtype, stream);
+    return fwd_impl(q, k, v, o, lse, B, H, H, n, n, d, scale, -1, causal ? 0 : -1, dtype, stream);
 }
 
 int attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                  int Hkv, int n, int d, float scale, int causal, int dtype, void* stream) {
-    return fwd_impl(q, k, v, o, lse, B, H, Hkv, n, d, scale, causal, dtype, stream);
+    return fwd_impl(q, k, v, o, lse, B, H, Hkv, n, n, d, scale, -1, causal ? 0 : -1, dtype,
+                    stream);
+}
+
+int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                int Hkv, int nq, int nk, int d, float scale, int window_left, int window_right,
+                int dtype, void* stream) {
+    return fwd_impl(q, k, v, o, lse, B, H, Hkv, nq, nk, d, scale, window_left, window_right, dtype,
+                    stream);
 }
 
 size_t attn_bwd_workspace_bytes(int B, int H, int n, int d, int deterministic) {
@@ -166,27 +177,29 @@ size_t attn_bwd_workspace_bytes(int B, int H, int n, int d, int deterministic) {
 }
 
 static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dO,
-                    const float* lse, void* dq, void* dk, void* dv, int B, int H, int Hkv, int n,
-                    int d, float scale, int causal, int dtype, int deterministic, void* workspace,
-                    size_t ws_bytes, void* stream) {
+                    const float* lse, void* dq, void* dk, void* dv, int B, int H, int Hkv, int nq,
+                    int nk, int d, float scale, int wl, int wr, int dtype, int deterministic,
+                    void* workspace, size_t ws_bytes, void* stream) {
     if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return ATTN_ERR_INVALID;
-    int rc = validate_common(B, H, n, d, scale, dtype);
+    int rc = validate_common(B, H, nq, d, scale, dtype);
     if (rc) return rc;
+    if (nk < 1) return ATTN_ERR_INVALID;
     if (Hkv < 1 || H % Hkv != 0) return ATTN_ERR_INVALID;
     if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
     const void* ptrs[] = {q, k, v, o, dO, lse, dq, dk, dv};
     for (const void* p : ptrs)
         if (!aligned16(p)) return ATTN_ERR_INVALID;
-    WsLayout w = ws_layout(B, H, n, d, deterministic);
+    WsLayout w = ws_layout(B, H, nq, d, deterministic);
     if (!workspace) return ATTN_ERR_INVALID;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_INVALID;
     if (ws_bytes < w.total) return ATTN_ERR_WORKSPACE;
     BwdArgs a;
     a.q = q; a.k = k; a.v = v; a.o = o; a.dO = dO; a.lse = lse;
     a.dq = dq; a.dk = dk; a.dv = dv;
-    a.B = B; a.H = H; a.n = n; a.d = d; a.Hkv = Hkv;
+    a.B = B; a.H = H; a.nq = nq; a.nk = nk; a.d = d; a.Hkv = Hkv;
     a.scale = scale;
-    a.causal = causal ? 1 : 0;
+    a.wl = wl < 0 ? -1 : wl;
+    a.wr = wr < 0 ? -1 : wr;
     a.deterministic = deterministic ? 1 : 0;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     a.Dvec = reinterpret_cast<float*>(ws + w.d_off);
@@ -202,16 +215,24 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const v
              const float* lse, void* dq, void* dk, void* dv, int B, int H, int n, int d,
              float scale, int causal, int dtype, int deterministic, void* workspace,
              size_t ws_bytes, void* stream) {
-    return bwd_impl(q, k, v, o, dO, lse, dq, dk, dv, B, H, H, n, d, scale, causal, dtype,
-                    deterministic, workspace, ws_bytes, stream);
+    return bwd_impl(q, k, v, o, dO, lse, dq, dk, dv, B, H, H, n, n, d, scale, -1, causal ? 0 : -1,
+                    dtype, deterministic, workspace, ws_bytes, stream);
 }
 
 int attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const void* dO,
                  const float* lse, void* dq, void* dk, void* dv, int B, int H, int Hkv, int n,
                  int d, float scale, int causal, int dtype, int deterministic, void* workspace,
                  size_t ws_bytes, void* stream) {
-    return bwd_impl(q, k, v, o, dO, lse, dq, dk, dv, B, H, Hkv, n, d, scale, causal, dtype,
-                    deterministic, workspace, ws_bytes, stream);
+    return bwd_impl(q, k, v, o, dO, lse, dq, dk, dv, B, H, Hkv, n, n, d, scale, -1,
+                    causal ? 0 : -1, dtype, deterministic, workspace, ws_bytes, stream);
+}
+
+int attn_bwd_ex(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                const float* lse, void* dq, void* dk, void* dv, int B, int H, int Hkv, int nq,
+                int nk, int d, float scale, int window_left, int window_right, int dtype,
+                int deterministic, void* workspace, size_t ws_bytes, void* stream) {
+    return bwd_impl(q, k, v, o, dO, lse, dq, dk, dv, B, H, Hkv, nq, nk, d, scale, window_left,
+                    window_right, dtype, deterministic, workspace, ws_bytes, stream);
 }
 
 void attn_set_bwd_phase_events(void* const* events) {

@@ -20,7 +20,9 @@
 //                   TMEM (512 columns): dV | dK | S^T (P^T as bf16) | dP^T, and the dQ tile reuses
 //                   the dP^T columns once dS^T is formed.
 //   bwd_dq_convert  dQ = scale·acc -> bf16.                                    HBM-bound
-// Causal: key tile j only meets query tiles i >= j.
+// Masks (causal, sliding window, query/key lengths that differ; see MaskSpec): key tile j only
+// meets the query tiles that hold a query which sees one of its keys; a key tile that no query
+// sees gets dK = dV = 0.
 #include "kernels.h"
 #include "sm100_ptx.cuh"
 
@@ -61,8 +63,12 @@ struct BwdKParams {
     int* sems;
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
-    int n, n_pad, BH, nq, causal, deterministic, group;
-    int kv_group;     // query heads per K/V head; BH counts K/V heads (one CTA row per K/V head)
+    int n_pad;        // query rows per head in the workspace arrays (multiple of 128)
+    int BH;           // K/V heads (one CTA row per K/V head)
+    int nkt;          // key tiles of 128 per head
+    int deterministic, group;
+    int kv_group;     // query heads per K/V head
+    MaskSpec mask;
     float scale, scale_log2;
     uint64_t timeout_ns;
 };
@@ -129,8 +135,10 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __nv_bfloat16
             acc += __shfl_xor_sync(0xffffffffu, acc, off, LPR);
         if (row < rows && part == 0) {
             Dvec[row] = valid ? acc : 0.f;
-            // LSE in log2 units; +inf on padding rows makes their P exactly 0 downstream
-            L2vec[row] = valid ? lse[src / D] * 1.44269504088896340736f : INFINITY;
+            // LSE in log2 units; +inf on padding rows and on rows that see no key (LSE = -inf)
+            // makes their P exactly 0 downstream
+            const float l = valid ? lse[src / D] : INFINITY;
+            L2vec[row] = l == -INFINITY ? INFINITY : l * 1.44269504088896340736f;
         }
     }
     if (sems) {
@@ -204,14 +212,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // Heads in groups of p.group (a group's Q, dO, K, V and dQ rows stay in L2); within a group,
     // key tiles go from small j (most causal work) to large j across the group's heads.
     const int L = blockIdx.x;
-    const int gbase = (L / (p.group * p.nq)) * p.group;
+    const int gbase = (L / (p.group * p.nkt)) * p.group;
     const int gsize = min(p.group, p.BH - gbase);
-    const int r_in = L - gbase * p.nq;
+    const int r_in = L - gbase * p.nkt;
     const int j = r_in / gsize;
     const int kvbh = gbase + r_in % gsize;        // K/V head of this CTA
-    const int n = p.n;
-    const int i_begin = p.causal ? j : 0;
-    const int NT = p.nq - i_begin;                // query tiles per query head
+    const MaskSpec& mk = p.mask;
+    const int nk = mk.nk;
+    const int qt128 = p.n_pad / 128;              // semaphore stride per query head
+    int i_begin, i_end;                           // query tiles that meet this key tile
+    visible_query_tiles(mk, j * 128LL, min(j * 128LL + 127, nk - 1LL), 128, i_begin, i_end);
+    const int NT = i_end - i_begin;               // query tiles per query head
     const int NTT = NT * p.kv_group;              // over all query heads sharing this K/V head
 
     if (threadIdx.x == 0) {
@@ -250,7 +261,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
     if (warp == 8) {
         // ---------------------------------------------------------------- TMA producer
-        if (lane == 0 && !*abort) {
+        if (lane == 0 && !*abort && NTT > 0) {
             mbar_arrive_expect_tx(&bars->kv_full, 2 * C::TILE);
             for (int ch = 0; ch < C::NCH; ++ch) {
                 tma_load_3d(sK + ch * C::CHUNK, &tmK, &bars->kv_full, ch * C::CW, j * 128, kvbh);
@@ -318,7 +329,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     mma_ss(tmem + COL_DP, sdesc_at(V_k, koff(ks)), sdesc_at(bo, koff(ks)), idSS,
                            ks > 0 ? 1u : 0u);
             };
-            bool ok = bounded_wait(&bars->kv_full, 0, abort, lim);
+            bool ok = NTT > 0 && bounded_wait(&bars->kv_full, 0, abort, lim);
             if (ok) ok = bounded_wait(&bars->q_full[0], 0, abort, lim);
             tc_fence_after();
             if (ok) {
@@ -390,6 +401,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int r = (warp & 3) * 32 + lane;              // key row within the tile = TMEM lane
         const int kidx = j * 128 + r;
         const int cb = g * 64;
+        // queries that see key kidx: [qmin, qmax] (empty for a key past the end)
+        int qmin = 1, qmax = 0;
+        if (kidx < nk) {
+            qmin = mk.wr < 0 ? -0x7fffffff : clamp_int(kidx - mk.off - mk.wr);
+            qmax = mk.wl < 0 ? 0x7fffffff : clamp_int(kidx - mk.off + mk.wl);
+        }
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + lane_base + COL_S;
         const uint32_t tDP = tmem + lane_base + COL_DP;
@@ -415,8 +432,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (p.deterministic) {
                 // add this tile's partial only after every lower key tile has added its own
                 // (each CTA contributes two halves, one per warpgroup)
-                volatile int* sem = p.sems + static_cast<size_t>(qbh) * p.nq + i;
-                const int need = 2 * (p.causal ? j : j);
+                volatile int* sem = p.sems + static_cast<size_t>(qbh) * qt128 + i;
+                const int need = 2 * (j - first_key_tile(mk, i * 128LL, 128));
                 bool got = true;
                 if (t == 0) {
                     const uint64_t t0 = globaltimer_ns();
@@ -477,7 +494,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (p.deterministic) {
                 __threadfence();
                 wg_bar();
-                if (t == 0) atomicAdd(p.sems + static_cast<size_t>(qbh) * p.nq + i, 1);
+                if (t == 0) atomicAdd(p.sems + static_cast<size_t>(qbh) * qt128 + i, 1);
             }
             return true;
         };
@@ -488,17 +505,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             float* sL = sStat + (g * 2 + (it & 1)) * 128;
             float* sD = sL + 64;
             {
-                const int qq = i * 128 + cb + (t & 63);
+                const size_t qq = static_cast<size_t>(qbh) * p.n_pad + i * 128 + cb + (t & 63);
                 if (t < 64)
-                    sL[t] = (qq < n) ? p.lse[static_cast<size_t>(qbh) * n + qq] * kBwdLog2e : INFINITY;
+                    sL[t] = p.L2vec[qq];
                 else
-                    sD[t - 64] = (qq < n) ? p.Dvec[static_cast<size_t>(qbh) * p.n_pad + qq] : 0.f;
+                    sD[t - 64] = p.Dvec[qq];
             }
             wg_bar();
             // ---- P^T = exp2(S^T·scale·log2e - LSE·log2e), masked; bf16 copy into TMEM
             if (!(ok = wait_all(&bars->s_full, it & 1))) break;
             tc_fence_after();
-            const bool edge = (p.causal && i == j) || (kidx >= n);
+            bool edge;
+            {   // every key of the tile visible to every query of the tile: no mask needed
+                long long flo, fhi;
+                visible_keys(mk, i * 128LL + 127, i * 128LL, flo, fhi);
+                edge = !(flo <= j * 128LL && j * 128LL + 127 <= fhi);
+            }
+            const int q0 = i * 128 + cb;
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 uint32_t u[32];
@@ -508,7 +531,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 for (int x = 0; x < 32; ++x) {
                     const int col = c * 32 + x;
                     float v = ex2_approx(fmaf(__uint_as_float(u[x]), sl2, -sL[col]));
-                    if (edge && (kidx >= n || (p.causal && i * 128 + cb + col < kidx))) v = 0.f;
+                    if (edge && (q0 + col < qmin || q0 + col > qmax)) v = 0.f;
                     pr[col] = v;
                 }
             }
@@ -553,10 +576,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_arrive(&bars->ds_full);
         }
         if (ok && NTT > 0) ok = drain(NTT - 1);
+        if (ok && NTT == 0) {
+            // no query sees these keys: dK = dV = 0
+            if (kidx < nk) {
+                const size_t orow = (static_cast<size_t>(kvbh) * nk + kidx) * D + g * (D / 2);
+#pragma unroll
+                for (int x = 0; x < D / 16; ++x) {
+                    reinterpret_cast<uint4*>(p.dk + orow)[x] = make_uint4(0u, 0u, 0u, 0u);
+                    reinterpret_cast<uint4*>(p.dv + orow)[x] = make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+            ok = false;
+        }
         if (ok) ok = wait_all(&bars->dkv_done, 0);
         if (ok) {
             tc_fence_after();
-            const size_t orow = (static_cast<size_t>(kvbh) * n + kidx) * D + g * (D / 2);
+            const size_t orow = (static_cast<size_t>(kvbh) * nk + kidx) * D + g * (D / 2);
 #pragma unroll 1
             for (int which = 0; which < 2; ++which) {
                 const uint32_t tacc = tmem + lane_base + (which == 0 ? COL_DV : COL_DK) + g * (D / 2);
@@ -572,7 +607,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     for (int x = 0; x < 8; ++x)
                         w[x] = pack_bf16x2(__uint_as_float(u[2 * x]) * mul,
                                            __uint_as_float(u[2 * x + 1]) * mul);
-                    if (kidx < n) {
+                    if (kidx < nk) {
                         uint4* o = reinterpret_cast<uint4*>(dst + cc);
                         o[0] = make_uint4(w[0], w[1], w[2], w[3]);
                         o[1] = make_uint4(w[4], w[5], w[6], w[7]);
@@ -664,15 +699,17 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
     const int lane = threadIdx.x & 31;
     // Heads in groups of p.group (see bwd_main_kernel); key tiles of 128 keys, small j first.
     const int L = blockIdx.x;
-    const int gbase = (L / (p.group * p.nq)) * p.group;
+    const int gbase = (L / (p.group * p.nkt)) * p.group;
     const int gsize = min(p.group, p.BH - gbase);
-    const int r_in = L - gbase * p.nq;
+    const int r_in = L - gbase * p.nkt;
     const int j = r_in / gsize;
     const int kvbh = gbase + r_in % gsize;         // K/V head of this CTA
-    const int n = p.n;
-    const int nq = p.n_pad / BQ;                   // 64-row query tiles per head (padded)
-    const int i_begin = p.causal ? 2 * j : 0;
-    const int NT = nq - i_begin;                   // query tiles per query head
+    const MaskSpec& mk = p.mask;
+    const int nk = mk.nk;
+    const int qt64 = p.n_pad / BQ;                 // semaphore stride per query head
+    int i_begin, i_end;                            // 64-row query tiles that meet this key tile
+    visible_query_tiles(mk, j * 128LL, min(j * 128LL + 127, nk - 1LL), BQ, i_begin, i_end);
+    const int NT = i_end - i_begin;                // query tiles per query head
     const int NTT = NT * p.kv_group;               // over all query heads sharing this K/V head
 
     if (threadIdx.x == 0) {
@@ -715,7 +752,7 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
 
     if (warp == 8) {
         // ---------------------------------------------------------------- TMA producer
-        if (lane == 0 && !*abort) {
+        if (lane == 0 && !*abort && NTT > 0) {
             mbar_arrive_expect_tx(&bars->kv_full, 2 * KTILE);
             for (int ch = 0; ch < 2; ++ch) {
                 tma_load_3d(sK + ch * 16384, &tmK, &bars->kv_full, ch * 64, j * 128, kvbh);
@@ -775,7 +812,7 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
                 for (int ks = 0; ks < 8; ++ks)
                     MMA_SS(tmem + COL_DP, sdesc_at(V_k, k128(ks)), sdesc_at(bo, k64(ks)), idS, ks > 0 ? 1u : 0u);
             };
-            bool ok = bounded_wait_warp(&bars->kv_full, 0, abort, lim);
+            bool ok = NTT > 0 && bounded_wait_warp(&bars->kv_full, 0, abort, lim);
             if (ok) ok = bounded_wait_warp(&bars->q_full[0], 0, abort, lim);
             tc_fence_after();
             if (ok) {
@@ -867,12 +904,14 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
                 const int i = i_begin + it % NT;
                 const int qbh = kvbh * p.kv_group + it / NT;
                 float* dst = p.dq_acc + (static_cast<size_t>(qbh) * p.n_pad + i * BQ) * D;
-                volatile int* sem = p.deterministic ? p.sems + static_cast<size_t>(qbh) * nq + i : nullptr;
+                volatile int* sem = p.deterministic ? p.sems + static_cast<size_t>(qbh) * qt64 + i : nullptr;
                 bool got = true;
                 if (sem) {
-                    // contributions to one query tile are added in increasing key-tile order
+                    // contributions to one query tile are added in increasing key-tile order,
+                    // starting from the first key tile that this query tile meets
+                    const int need = j - first_key_tile(mk, static_cast<long long>(i) * BQ, 128);
                     const uint64_t t0 = globaltimer_ns();
-                    while (*sem < j) {
+                    while (*sem < need) {
                         if (*abort || globaltimer_ns() - t0 > lim) {
                             *abort = 1;
                             report_error(4);
@@ -903,6 +942,12 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
         const int r = (warp & 3) * 32 + lane;              // key row = TMEM lane
         const int kidx = j * 128 + r;
         const int cb = g * 32;
+        // queries that see key kidx: [qmin, qmax] (empty for a key past the end)
+        int qmin = 1, qmax = 0;
+        if (kidx < nk) {
+            qmin = mk.wr < 0 ? -0x7fffffff : clamp_int(kidx - mk.off - mk.wr);
+            qmax = mk.wl < 0 ? 0x7fffffff : clamp_int(kidx - mk.off + mk.wl);
+        }
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const float sl2 = p.scale_log2;
         auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
@@ -924,7 +969,13 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
                 tmem_ld32(tmem + lane_base + COL_S + cb, u);
                 tmem_ld_wait();
                 reg_fence<32>(u);
-                const bool edge = (p.causal && i * BQ < (j + 1) * 128) || (kidx >= n);
+                bool edge;
+                {   // every key of the tile visible to every query of the tile: no mask needed
+                    long long flo, fhi;
+                    visible_keys(mk, static_cast<long long>(i) * BQ + BQ - 1,
+                                 static_cast<long long>(i) * BQ, flo, fhi);
+                    edge = !(flo <= j * 128LL && j * 128LL + 127 <= fhi);
+                }
 #pragma unroll
                 for (int x = 0; x < 32; x += 4) {
                     const float4 l4 = *reinterpret_cast<const float4*>(L2 + x);
@@ -934,9 +985,10 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
                     pr[x + 3] = ex2_approx(fmaf(__uint_as_float(u[x + 3]), sl2, -l4.w));
                 }
                 if (edge) {
+                    const int q0 = i * BQ + cb;
 #pragma unroll
                     for (int x = 0; x < 32; ++x)
-                        if (kidx >= n || (p.causal && i * BQ + cb + x < kidx)) pr[x] = 0.f;
+                        if (q0 + x < qmin || q0 + x > qmax) pr[x] = 0.f;
                 }
                 uint32_t w[16];
 #pragma unroll
@@ -976,10 +1028,22 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
             tc_fence_before();
             mbar_arrive(&bars->ds_full);
         }
+        if (ok && NTT == 0) {
+            // no query sees these keys: dK = dV = 0
+            if (kidx < nk) {
+                const size_t orow = (static_cast<size_t>(kvbh) * nk + kidx) * D + g * 64;
+#pragma unroll
+                for (int x = 0; x < 8; ++x) {
+                    reinterpret_cast<uint4*>(p.dk + orow)[x] = make_uint4(0u, 0u, 0u, 0u);
+                    reinterpret_cast<uint4*>(p.dv + orow)[x] = make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+            ok = false;
+        }
         if (ok) ok = wait_all(&bars->dkv_done, 0);
         if (ok) {
             tc_fence_after();
-            const size_t orow = (static_cast<size_t>(kvbh) * n + kidx) * D + g * 64;
+            const size_t orow = (static_cast<size_t>(kvbh) * nk + kidx) * D + g * 64;
 #pragma unroll 1
             for (int which = 0; which < 2; ++which) {
                 const uint32_t tacc = tmem + lane_base + (which == 0 ? COL_DV : COL_DK) + g * 64;
@@ -996,7 +1060,7 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
                     for (int x = 0; x < 16; ++x)
                         w[x] = pack_bf16x2(__uint_as_float(u[2 * x]) * mul,
                                            __uint_as_float(u[2 * x + 1]) * mul);
-                    if (kidx < n) {
+                    if (kidx < nk) {
                         uint4* o = reinterpret_cast<uint4*>(dst + cc);
 #pragma unroll
                         for (int x = 0; x < 4; ++x)
@@ -1019,16 +1083,17 @@ template <int D>
 cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
     using C = BwdCfg<D>;
     const int BH = a.B * a.H;
-    const int nq = (a.n + 127) / 128;
-    const int n_pad = nq * 128;
-    // Main-kernel CTAs run per K/V head. Heads per group: a K/V head's K and V (4·n·d bytes) and
-    // its g query heads' Q, dO (4·n·d each) and fp32 dQ rows (4·n·d each); keep a group within
+    const int n_pad = (a.nq + 127) / 128 * 128;
+    const int nkt = (a.nk + 127) / 128;
+    const int nk_pad = nkt * 128;
+    // Main-kernel CTAs run per K/V head. Heads per group: a K/V head's K and V (4·nk·d bytes) and
+    // its g query heads' Q, dO (4·nq·d each) and fp32 dQ rows (4·nq·d each); keep a group within
     // ~48 MB of L2
     const int BHkv = a.B * a.Hkv;
     const int kvg = a.H / a.Hkv;
     int group;
     {
-        const long long per_head = (4LL + 8LL * kvg) * n_pad * D;
+        const long long per_head = (4LL * nk_pad + 8LL * kvg * n_pad) * D;
         long long g = (48LL << 20) / (per_head > 0 ? per_head : 1);
         group = static_cast<int>(g < 1 ? 1 : (g > BHkv ? BHkv : g));
     }
@@ -1044,89 +1109,61 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
         const int n_sems = a.deterministic ? BH * (n_pad / 64) : 0;
         bwd_preprocess_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
             static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dO), a.lse,
-            a.L2vec, a.Dvec, a.dq_acc, a.deterministic ? a.sems : nullptr, a.n, n_pad, rows,
+            a.L2vec, a.Dvec, a.dq_acc, a.deterministic ? a.sems : nullptr, a.nq, n_pad, rows,
             n_sems);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     // 2. main
+    BwdKParams kp;
+    kp.lse = a.lse;
+    kp.Dvec = a.Dvec;
+    kp.L2vec = a.L2vec;
+    kp.dq_acc = a.dq_acc;
+    kp.sems = a.sems;
+    kp.dk = static_cast<__nv_bfloat16*>(a.dk);
+    kp.dv = static_cast<__nv_bfloat16*>(a.dv);
+    kp.n_pad = n_pad;
+    kp.BH = BHkv;
+    kp.nkt = nkt;
+    kp.kv_group = kvg;
+    kp.deterministic = a.deterministic;
+    kp.group = group;
+    kp.mask = MaskSpec{a.nq, a.nk, a.wl, a.wr, static_cast<long long>(a.nk) - a.nq};
+    kp.scale = a.scale;
+    kp.scale_log2 = a.scale * kBwdLog2e;
+    kp.timeout_ns = a.timeout_ns;
+    const long long grid = static_cast<long long>(nkt) * BHkv;
+    if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    const int qbox = D == 128 ? q64::BQ : 128;
+    CUtensorMap mq, mk, mv, mdo;
+    if ((e = make_tmap_bf16(&mq, a.q, BH, a.nq, D, qbox)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16(&mk, a.k, BHkv, a.nk, D)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16(&mv, a.v, BHkv, a.nk, D)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16(&mdo, a.dO, BH, a.nq, D, qbox)) != cudaSuccess) return e;
     if constexpr (D == 128) {
-        CUtensorMap mq, mk, mv, mdo;
-        if ((e = make_tmap_bf16(&mq, a.q, BH, a.n, D, q64::BQ)) != cudaSuccess) return e;
-        if ((e = make_tmap_bf16(&mk, a.k, BHkv, a.n, D)) != cudaSuccess) return e;
-        if ((e = make_tmap_bf16(&mv, a.v, BHkv, a.n, D)) != cudaSuccess) return e;
-        if ((e = make_tmap_bf16(&mdo, a.dO, BH, a.n, D, q64::BQ)) != cudaSuccess) return e;
         e = cudaFuncSetAttribute(bwd_main_q64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  q64::SMEM);
         if (e != cudaSuccess) return e;
-        BwdKParams kp;
-        kp.lse = a.lse;
-        kp.Dvec = a.Dvec;
-        kp.L2vec = a.L2vec;
-        kp.dq_acc = a.dq_acc;
-        kp.sems = a.sems;
-        kp.dk = static_cast<__nv_bfloat16*>(a.dk);
-        kp.dv = static_cast<__nv_bfloat16*>(a.dv);
-        kp.n = a.n;
-        kp.n_pad = n_pad;
-        kp.BH = BHkv;
-        kp.kv_group = kvg;
-        kp.nq = nq;
-        kp.causal = a.causal;
-        kp.deterministic = a.deterministic;
-        kp.group = group;
-        kp.scale = a.scale;
-        kp.scale_log2 = a.scale * kBwdLog2e;
-        kp.timeout_ns = a.timeout_ns;
-        const long long grid = static_cast<long long>(nq) * BHkv;
-        if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
         if (ev && ev[1] && (e = cudaEventRecord(ev[1], stream)) != cudaSuccess) return e;
         bwd_main_q64_kernel<<<static_cast<unsigned>(grid), q64::kThreads, q64::SMEM, stream>>>(
             mq, mk, mv, mdo, kp);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        if (ev && ev[2] && (e = cudaEventRecord(ev[2], stream)) != cudaSuccess) return e;
     } else {
-        CUtensorMap mq, mk, mv, mdo;
-        if ((e = make_tmap_bf16(&mq, a.q, BH, a.n, D)) != cudaSuccess) return e;
-        if ((e = make_tmap_bf16(&mk, a.k, BHkv, a.n, D)) != cudaSuccess) return e;
-        if ((e = make_tmap_bf16(&mv, a.v, BHkv, a.n, D)) != cudaSuccess) return e;
-        if ((e = make_tmap_bf16(&mdo, a.dO, BH, a.n, D)) != cudaSuccess) return e;
         e = cudaFuncSetAttribute(bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::SMEM);
         if (e != cudaSuccess) return e;
-        BwdKParams kp;
-        kp.lse = a.lse;
-        kp.Dvec = a.Dvec;
-        kp.L2vec = a.L2vec;
-        kp.dq_acc = a.dq_acc;
-        kp.sems = a.sems;
-        kp.dk = static_cast<__nv_bfloat16*>(a.dk);
-        kp.dv = static_cast<__nv_bfloat16*>(a.dv);
-        kp.n = a.n;
-        kp.n_pad = n_pad;
-        kp.BH = BHkv;
-        kp.kv_group = kvg;
-        kp.nq = nq;
-        kp.causal = a.causal;
-        kp.deterministic = a.deterministic;
-        kp.group = group;
-        kp.scale = a.scale;
-        kp.scale_log2 = a.scale * kBwdLog2e;
-        kp.timeout_ns = a.timeout_ns;
-        const long long grid = static_cast<long long>(nq) * BHkv;
-        if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
         if (ev && ev[1] && (e = cudaEventRecord(ev[1], stream)) != cudaSuccess) return e;
         bwd_main_kernel<D><<<static_cast<unsigned>(grid), kBwdThreads, C::SMEM, stream>>>(
             mq, mk, mv, mdo, kp);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        if (ev && ev[2] && (e = cudaEventRecord(ev[2], stream)) != cudaSuccess) return e;
     }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (ev && ev[2] && (e = cudaEventRecord(ev[2], stream)) != cudaSuccess) return e;
     // 3. dQ convert
     {
-        const long long total8 = static_cast<long long>(BH) * a.n * (D / 8);
+        const long long total8 = static_cast<long long>(BH) * a.nq * (D / 8);
         long long blocks = (total8 + 255) / 256;
         if (blocks > 148 * 16) blocks = 148 * 16;
         bwd_dq_convert_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-            a.dq_acc, static_cast<__nv_bfloat16*>(a.dq), a.n, n_pad, total8, a.scale);
+            a.dq_acc, static_cast<__nv_bfloat16*>(a.dq), a.nq, n_pad, total8, a.scale);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         if (ev && ev[3] && (e = cudaEventRecord(ev[3], stream)) != cudaSuccess) return e;
     }

@@ -13,11 +13,14 @@
 //   warp 9      one thread issues every tcgen05.mma:  S_g = Q_g·K_j^T (SMEM x SMEM -> TMEM) and
 //               O_g += P_g·V_j (P from TMEM, V from SMEM), and signals through tcgen05.commit.
 //   warps 0-3   softmax of query tile 0, warps 4-7 softmax of query tile 1: one thread per row
-//               (= one TMEM lane). They read S from TMEM, apply the causal mask on the diagonal
-//               tile, update m/l, rescale O in TMEM when m grows, and write P (bf16) back over S.
+//               (= one TMEM lane). They read S from TMEM, apply the mask on tiles that straddle
+//               its boundary, update m/l, rescale O in TMEM when m grows, and write P (bf16)
+//               back over S.
 //   The two query tiles alternate, so the tensor cores run one tile's MMAs while the other tile's
 //   softmax runs. TMEM (512 columns): O_0 | O_1 | S_0 (P_0) | S_1 (P_1), 128 columns each.
-//   Causal: query tile q only visits key tiles 0..q (tiles above the diagonal are skipped).
+//   Masks (causal, sliding window, query/key lengths that differ; see MaskSpec): each query tile
+//   visits only the key tiles that hold a key it can see; the two tiles of a pair stream the
+//   union of their ranges once. A row that sees no key gets O = 0 and LSE = -inf.
 #include "kernels.h"
 #include "sm100_ptx.cuh"
 
@@ -31,12 +34,8 @@ constexpr float kLog2e = 1.44269504088896340736f;
 #ifndef ATTN_FWD_EXP_FMA_PER8
 #define ATTN_FWD_EXP_FMA_PER8 0
 #endif
-#ifndef ATTN_FWD_PINGPONG
-#define ATTN_FWD_PINGPONG 0
-#endif
 constexpr int kExpFmaPer8 = ATTN_FWD_EXP_FMA_PER8;   // column pairs (of every 8) whose exp2 runs
                                                      // on the FMA pipe
-constexpr bool kPingPong = ATTN_FWD_PINGPONG != 0;   // softmax warpgroups take turns
 
 template <int D>
 struct FwdCfg {
@@ -55,7 +54,7 @@ struct FwdCfg {
 struct FwdBars {
     uint64_t q_full;
     uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
-    uint64_t s_full[2], p_full[2], o_done[2], sm_done[2];
+    uint64_t s_full[2], p_full[2], o_done[2];
     uint64_t teardown;
     uint32_t tmem_base;
     int abort;
@@ -64,8 +63,9 @@ struct FwdBars {
 struct FwdKParams {
     void* o;
     float* lse;
-    int n, BH, n_pairs, causal, group;
+    int BH, n_pairs, group;
     int kv_group;     // query heads per K/V head (grouped-query attention); 1 for MHA
+    MaskSpec mask;
     float scale_log2;
     uint64_t timeout_ns;
 };
@@ -102,7 +102,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     // Heads are processed in groups of p.group (sized so that a group's K and V stay in L2);
-    // within a group, tile pairs go longest-first (causal) across the group's heads.
+    // within a group, tile pairs go from the last to the first (longest first under a causal
+    // mask) across the group's heads.
     const int L = blockIdx.x;
     const int gbase = (L / (p.group * p.n_pairs)) * p.group;
     const int gsize = min(p.group, p.BH - gbase);
@@ -110,15 +111,28 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const int pair = p.n_pairs - 1 - r_in / gsize;
     const int bh = gbase + r_in % gsize;
     const int kvbh = bh / p.kv_group;                     // (b, h / g) = (b·H + h) / g
-    const int n = p.n;
-    const int n_kv = (n + C::BN - 1) / C::BN;
-    int T[2];
+    const MaskSpec& mk = p.mask;
+    const int nq = mk.nq;
+    // key tiles [J0[g], J0[g] + T[g]) of query tile g; the pair streams [Jmin, Jmin + U) once
+    int J0[2], T[2];
 #pragma unroll
     for (int g = 0; g < 2; ++g) {
-        const int qt = 2 * pair + g;
-        T[g] = (qt * C::BM >= n) ? 0 : (p.causal ? min(n_kv, qt + 1) : n_kv);
+        const long long a = static_cast<long long>(2 * pair + g) * C::BM;
+        J0[g] = 0;
+        T[g] = 0;
+        if (a < nq) {
+            long long lo, hi;
+            visible_keys(mk, a, min(a + C::BM - 1, static_cast<long long>(nq - 1)), lo, hi);
+            if (lo <= hi) {
+                J0[g] = static_cast<int>(lo / C::BN);
+                T[g] = static_cast<int>(hi / C::BN) + 1 - J0[g];
+            }
+        }
     }
-    const int Tmax = max(T[0], T[1]);
+    const int Jmin = T[0] > 0 ? (T[1] > 0 ? min(J0[0], J0[1]) : J0[0]) : J0[1];
+    const int U = (T[0] > 0 || T[1] > 0)
+                      ? max(T[0] > 0 ? J0[0] + T[0] : 0, T[1] > 0 ? J0[1] + T[1] : 0) - Jmin
+                      : 0;
 
     if (threadIdx.x == 0) {
         if ((smem_addr(smem) & 1023u) != 0) report_error(3);
@@ -133,7 +147,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             mbar_init(&bars->s_full[g], 1);
             mbar_init(&bars->p_full[g], 128);
             mbar_init(&bars->o_done[g], 1);
-            mbar_init(&bars->sm_done[g], 128);
         }
         mbar_init(&bars->teardown, 1);
         bars->abort = ((smem_addr(smem) & 1023u) != 0) ? 1 : 0;
@@ -159,7 +172,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 80;");
     if (warp == 8) {
         // ---------------------------------------------------------------- TMA producer
-        if (lane == 0 && !*abort) {
+        if (lane == 0 && !*abort && U > 0) {
             uint32_t qbytes = (T[0] > 0 ? C::TILE : 0) + (T[1] > 0 ? C::TILE : 0);
             mbar_arrive_expect_tx(&bars->q_full, qbytes);
             for (int g = 0; g < 2; ++g)
@@ -168,30 +181,31 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                         tma_load_3d(sQ + g * C::TILE + ch * C::CHUNK, &tmQ, &bars->q_full,
                                     ch * C::CW, (2 * pair + g) * C::BM, bh);
             int issued = 0;
-            for (int jj = 0; jj < Tmax; ++jj) {
-                const int s = jj % C::STAGES;
-                const int f = jj / C::STAGES;
+            for (int u = 0; u < U; ++u) {
+                const int s = u % C::STAGES;
+                const int f = u / C::STAGES;
+                const int krow = (Jmin + u) * C::BN;
                 if (f > 0 && !bounded_wait(&bars->k_empty[s], (f - 1) & 1, abort, lim)) break;
                 mbar_arrive_expect_tx(&bars->k_full[s], C::TILE);
                 for (int ch = 0; ch < C::NCH; ++ch)
                     tma_load_3d(sK + s * C::TILE + ch * C::CHUNK, &tmK, &bars->k_full[s],
-                                ch * C::CW, jj * C::BN, kvbh);
-                issued = 2 * jj + 1;
+                                ch * C::CW, krow, kvbh);
+                issued = 2 * u + 1;
                 if (f > 0 && !bounded_wait(&bars->v_empty[s], (f - 1) & 1, abort, lim)) break;
                 mbar_arrive_expect_tx(&bars->v_full[s], C::TILE);
                 for (int ch = 0; ch < C::NCH; ++ch)
                     tma_load_3d(sV + s * C::TILE + ch * C::CHUNK, &tmV, &bars->v_full[s],
-                                ch * C::CW, jj * C::BN, kvbh);
-                issued = 2 * jj + 2;
+                                ch * C::CW, krow, kvbh);
+                issued = 2 * u + 2;
             }
             if (*abort) {
                 // let every copy issued so far land before the CTA can exit
                 drain_wait_fwd(&bars->q_full, 0, 100000000ull);
                 for (int x = 0; x < issued; ++x) {
-                    const int jj = x >> 1;
-                    const int s = jj % C::STAGES;
+                    const int u = x >> 1;
+                    const int s = u % C::STAGES;
                     drain_wait_fwd((x & 1) ? &bars->v_full[s] : &bars->k_full[s],
-                               (jj / C::STAGES) & 1, 100000000ull);
+                               (u / C::STAGES) & 1, 100000000ull);
                 }
             }
         }
@@ -202,16 +216,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             constexpr uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);
             constexpr uint32_t idPV = idesc_bf16_f32(128, D, 0, 1);
             const uint32_t sQa = smem_addr(sQ), sKa = smem_addr(sK), sVa = smem_addr(sV);
-            bool ok = bounded_wait_warp(&bars->q_full, 0, abort, lim);
+            bool ok = U > 0 && bounded_wait_warp(&bars->q_full, 0, abort, lim);
             tc_fence_after();
             int k_ready = -1;
-            auto wait_k = [&](int jj) -> bool {
-                if (k_ready >= jj) return true;
-                if (!bounded_wait_warp(&bars->k_full[jj % C::STAGES], (jj / C::STAGES) & 1, abort,
+            auto wait_k = [&](int u) -> bool {     // u: index in the pair's key-tile stream
+                if (k_ready >= u) return true;
+                if (!bounded_wait_warp(&bars->k_full[u % C::STAGES], (u / C::STAGES) & 1, abort,
                                   lim))
                     return false;
                 tc_fence_after();
-                k_ready = jj;
+                k_ready = u;
                 return true;
             };
             // Lean issue path: descriptors per operand tile computed once, each k-step adds a
@@ -225,8 +239,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 dK[st] = sdesc(sKa + st * C::TILE, 16, 8 * C::SWB, C::SWZ);
                 dV[st] = sdesc(sVa + st * C::TILE, C::CHUNK, 8 * C::SWB, C::SWZ);
             }
-            auto issue_s = [&](int g, int jj) {
-                const SDesc a = dQ[g], b = dK[jj % C::STAGES];
+            auto issue_s = [&](int g, int u) {
+                const SDesc a = dQ[g], b = dK[u % C::STAGES];
                 const uint32_t d = tmem + 256 + g * 128;
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
@@ -235,48 +249,69 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     FMMA_SS(d, sdesc_at(a, off), sdesc_at(b, off), idS, ks > 0 ? 1u : 0u);
                 }
             };
-            auto issue_pv = [&](int g, int jj) {
-                const SDesc b = dV[jj % C::STAGES];
+            auto issue_pv = [&](int g, int u, bool accumulate) {
+                const SDesc b = dV[u % C::STAGES];
                 const uint32_t d = tmem + g * 128, a = tmem + 256 + g * 128;
-                FMMA_TS(d, a, sdesc_at(b, 0), idPV, jj > 0 ? 1u : 0u);
+                FMMA_TS(d, a, sdesc_at(b, 0), idPV, accumulate ? 1u : 0u);
 #pragma unroll
                 for (int ks = 1; ks < C::BN / 16; ++ks)
                     FMMA_TS(d, a + ks * 8, sdesc_at(b, static_cast<uint32_t>((ks * 16 * C::SWB) >> 4)),
                            idPV, 1u);
             };
+            // Stream step u holds key tile Jmin + u. Query tile g uses steps [J0[g] - Jmin,
+            // J0[g] - Jmin + T[g]); its S for step u+1 is issued during step u (or, for its first
+            // tile, before the loop / at the end of step u), so every S reading K tile u+1 is
+            // issued before k_empty of that tile is committed.
+            const int s0[2] = {J0[0] - Jmin, J0[1] - Jmin};
+            auto active = [&](int g, int u) { return T[g] > 0 && u >= s0[g] && u < s0[g] + T[g]; };
             if (ok) ok = wait_k(0);
             if (ok) {
                 for (int g = 0; g < 2; ++g)
-                    if (T[g] > 0) {
+                    if (T[g] > 0 && s0[g] == 0) {
                         issue_s(g, 0);
                         FMMA_COMMIT(&bars->s_full[g]);
                     }
                 FMMA_COMMIT(&bars->k_empty[0]);
             }
-            for (int jj = 0; ok && jj < Tmax; ++jj) {
+            for (int u = 0; ok && u < U; ++u) {
                 bool v_ready = false;
-                for (int g = 0; g < 2 && ok; ++g) {
-                    if (jj >= T[g]) continue;
-                    if (!bounded_wait_warp(&bars->p_full[g], jj & 1, abort, lim)) { ok = false; break; }
+                auto wait_v = [&]() -> bool {
+                    if (v_ready) return true;
+                    if (!bounded_wait_warp(&bars->v_full[u % C::STAGES], (u / C::STAGES) & 1,
+                                           abort, lim))
+                        return false;
                     tc_fence_after();
-                    if (!v_ready) {
-                        if (!bounded_wait_warp(&bars->v_full[jj % C::STAGES], (jj / C::STAGES) & 1,
-                                          abort, lim)) { ok = false; break; }
-                        tc_fence_after();
-                        v_ready = true;
-                    }
-                    issue_pv(g, jj);
-                    if (jj + 1 < T[g]) {
-                        if (!wait_k(jj + 1)) { ok = false; break; }
-                        issue_s(g, jj + 1);
+                    v_ready = true;
+                    return true;
+                };
+                for (int g = 0; g < 2 && ok; ++g) {
+                    if (!active(g, u)) continue;
+                    const int t = u - s0[g];
+                    if (!bounded_wait_warp(&bars->p_full[g], t & 1, abort, lim)) { ok = false; break; }
+                    tc_fence_after();
+                    if (!wait_v()) { ok = false; break; }
+                    issue_pv(g, u, t > 0);
+                    if (t + 1 < T[g]) {
+                        if (!wait_k(u + 1)) { ok = false; break; }
+                        issue_s(g, u + 1);
                         FMMA_COMMIT(&bars->s_full[g]);
                     } else {
                         FMMA_COMMIT(&bars->o_done[g]);
                     }
                 }
                 if (!ok) break;
-                FMMA_COMMIT(&bars->v_empty[jj % C::STAGES]);
-                if (jj + 1 < Tmax) FMMA_COMMIT(&bars->k_empty[(jj + 1) % C::STAGES]);
+                if (u + 1 < U) {
+                    for (int g = 0; g < 2 && ok; ++g)
+                        if (T[g] > 0 && s0[g] == u + 1) {      // first tile of g is the next one
+                            if (!wait_k(u + 1)) { ok = false; break; }
+                            issue_s(g, u + 1);
+                            FMMA_COMMIT(&bars->s_full[g]);
+                        }
+                    if (!ok || !(ok = wait_k(u + 1))) break;
+                }
+                if (!(ok = wait_v())) break;     // every loaded V tile is consumed before reuse
+                FMMA_COMMIT(&bars->v_empty[u % C::STAGES]);
+                if (u + 1 < U) FMMA_COMMIT(&bars->k_empty[(u + 1) % C::STAGES]);
             }
             // all MMAs of this CTA complete before TMEM is released
             FMMA_COMMIT(&bars->teardown);
@@ -292,6 +327,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const int r = wq * 32 + lane;                     // row within the tile = TMEM lane
         const int qt = 2 * pair + g;
         const int qidx = qt * C::BM + r;
+        const long long a = static_cast<long long>(qt) * C::BM;
+        // visible keys of this row: [klo, khi]
+        long long klo_l, khi_l;
+        visible_keys(mk, qidx, qidx, klo_l, khi_l);
+        const int klo = clamp_int(klo_l), khi = clamp_int(khi_l);
+        // keys seen by every row of the tile: [flo, fhi] (the last row's lower bound, the first
+        // row's upper bound); a key tile starting at kb needs no mask iff flo <= kb, kb+127 <= fhi
+        long long flo, fhi;
+        visible_keys(mk, a + C::BM - 1, a, flo, fhi);
+        const int full_lo = clamp_int(flo);
+        const int full_hi = clamp_int(fhi - (C::BN - 1));
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
         const uint32_t tS = tmem + lane_base + 256 + g * 128;
         const uint32_t tO = tmem + lane_base + g * 128;
@@ -299,17 +345,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         float m = -INFINITY;   // running max of scale*log2(e)*s
         float l = 0.f;         // running sum of exp2(.. - m)
         bool ok = true;
-        for (int jj = 0; jj < T[g]; ++jj) {
-            // Ping-pong: the two softmax warpgroups take turns (tile 0 of step jj, tile 1 of step
-            // jj, tile 0 of step jj+1, ...), so each has the exp units to itself while the tensor
-            // cores run the other tile's MMAs.
-            ok = true;
-            if (!kPingPong) {
-            } else if (g == 0 && jj > 0 && T[1] > 0)
-                ok = bounded_wait(&bars->sm_done[1], (jj - 1) & 1, abort, lim);
-            else if (g == 1 && jj < T[0])
-                ok = bounded_wait(&bars->sm_done[0], jj & 1, abort, lim);
-            ok = ok && bounded_wait(&bars->s_full[g], jj & 1, abort, lim);
+        for (int t = 0; t < T[g]; ++t) {
+            const int jj = J0[g] + t;
+            ok = bounded_wait(&bars->s_full[g], t & 1, abort, lim);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
@@ -321,12 +359,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             tmem_ld_wait();
             reg_fence<128>(u);
             const int kbase = jj * C::BN;
-            const bool edge = (p.causal && jj == qt) || kbase + C::BN > n;
+            const bool edge = kbase < full_lo || kbase > full_hi;
             if (edge) {
 #pragma unroll
                 for (int c = 0; c < 128; ++c) {
                     const int kidx = kbase + c;
-                    if (kidx >= n || (p.causal && kidx > qidx)) u[c] = __float_as_uint(-INFINITY);
+                    if (kidx < klo || kidx > khi) u[c] = __float_as_uint(-INFINITY);
                 }
             }
             float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
@@ -341,7 +379,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             // Lazy rescaling: the reference max m only moves when the tile max exceeds it by more
             // than 8 (a factor 2^8 on P); otherwise P = exp2(s·c - m) is simply allowed to exceed
             // 1. The final O/l and LSE = m + log2 l use the same m, so the result is unchanged.
-            if (jj == 0) {
+            if (t == 0) {
                 m = m_tile;
             } else if (__any_sync(0xffffffffu, m_tile > m + 8.f)) {
                 float alpha = 1.f;
@@ -407,16 +445,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&bars->p_full[g]);
-            mbar_arrive(&bars->sm_done[g]);
         }
         if (ok && T[g] > 0) {
             ok = bounded_wait(&bars->o_done[g], 0, abort, lim);
             ok = __all_sync(0xffffffffu, ok);
             if (ok) {
                 tc_fence_after();
-                const float inv_l = 1.f / l;
+                // a row that saw no key has l = 0 and an all-zero accumulator
+                const float inv_l = l > 0.f ? 1.f / l : 0.f;
                 __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) +
-                                      (static_cast<size_t>(bh) * n + qidx) * D;
+                                      (static_cast<size_t>(bh) * nq + qidx) * D;
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t u[32];
@@ -427,16 +465,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     for (int x = 0; x < 16; ++x)
                         w[x] = pack_bf16x2(__uint_as_float(u[2 * x]) * inv_l,
                                            __uint_as_float(u[2 * x + 1]) * inv_l);
-                    if (qidx < n) {
+                    if (qidx < nq) {
                         uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
                         for (int x = 0; x < 4; ++x)
                             dst[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
                     }
                 }
-                if (qidx < n)
-                    p.lse[static_cast<size_t>(bh) * n + qidx] = (m + __log2f(l)) * kLn2;
+                if (qidx < nq)
+                    p.lse[static_cast<size_t>(bh) * nq + qidx] =
+                        l > 0.f ? (m + __log2f(l)) * kLn2 : -INFINITY;
             }
+        } else if (ok && T[g] == 0 && qidx < nq) {
+            // the whole tile sees no key: O = 0, LSE = -inf
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.o) +
+                                                  (static_cast<size_t>(bh) * nq + qidx) * D);
+#pragma unroll
+            for (int x = 0; x < D / 8; ++x) dst[x] = make_uint4(0u, 0u, 0u, 0u);
+            p.lse[static_cast<size_t>(bh) * nq + qidx] = -INFINITY;
         }
     }
 
@@ -454,25 +500,24 @@ cudaError_t launch_fwd_bf16_d(const FwdArgs& a, cudaStream_t stream) {
     CUtensorMap mq, mk, mv;
     const int BH = a.B * a.H;
     cudaError_t e;
-    if ((e = make_tmap_bf16(&mq, a.q, BH, a.n, D)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16(&mq, a.q, BH, a.nq, D)) != cudaSuccess) return e;
     const int BHkv = a.B * a.Hkv;
-    if ((e = make_tmap_bf16(&mk, a.k, BHkv, a.n, D)) != cudaSuccess) return e;
-    if ((e = make_tmap_bf16(&mv, a.v, BHkv, a.n, D)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16(&mk, a.k, BHkv, a.nk, D)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16(&mv, a.v, BHkv, a.nk, D)) != cudaSuccess) return e;
     e = cudaFuncSetAttribute(fwd_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM);
     if (e != cudaSuccess) return e;
     FwdKParams kp;
     kp.o = a.o;
     kp.lse = a.lse;
-    kp.n = a.n;
     kp.BH = BH;
-    const int nq = (a.n + 127) / 128;
-    kp.n_pairs = (nq + 1) / 2;
-    kp.causal = a.causal;
+    const int qtiles = (a.nq + 127) / 128;
+    kp.n_pairs = (qtiles + 1) / 2;
+    kp.mask = MaskSpec{a.nq, a.nk, a.wl, a.wr, static_cast<long long>(a.nk) - a.nq};
     kp.kv_group = a.H / a.Hkv;
-    // heads per group: K and V of one head take 4·n·d bytes; keep a group's within ~32 MB of L2
+    // heads per group: K and V of one head take 4·nk·d bytes; keep a group's within ~32 MB of L2
     {
-        const long long per_head = 4LL * a.n * D;
+        const long long per_head = 4LL * a.nk * D;
         long long g = (32LL << 20) / (per_head > 0 ? per_head : 1);
         kp.group = static_cast<int>(g < 1 ? 1 : (g > BH ? BH : g));
     }

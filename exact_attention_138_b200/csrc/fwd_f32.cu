@@ -28,8 +28,8 @@ __global__ void __launch_bounds__(256) fwd_f32_kernel(const float* __restrict__ 
                                                       const float* __restrict__ K,
                                                       const float* __restrict__ V,
                                                       float* __restrict__ O,
-                                                      float* __restrict__ lse, int n, int n_qtiles,
-                                                      float scale, int causal, int kv_group) {
+                                                      float* __restrict__ lse, MaskSpec mk,
+                                                      int n_qtiles, float scale, int kv_group) {
     constexpr int DP = D + 1;
     constexpr int PP = kBN + 1;
     constexpr int OC = D / 16;
@@ -42,13 +42,23 @@ __global__ void __launch_bounds__(256) fwd_f32_kernel(const float* __restrict__ 
     const int qt = n_qtiles - 1 - static_cast<int>(blockIdx.x);   // longest causal rows first
     const int bh = blockIdx.y;
     const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-    const size_t base = static_cast<size_t>(bh) * n * D;
-    const size_t kvbase = static_cast<size_t>(bh / kv_group) * n * D;   // grouped-query K/V head
+    const int nq = mk.nq, nk = mk.nk;
+    const size_t base = static_cast<size_t>(bh) * nq * D;
+    const size_t kvbase = static_cast<size_t>(bh / kv_group) * nk * D;   // grouped-query K/V head
     const int q0 = qt * kBM;
 
     for (int idx = tid; idx < kBM * D; idx += 256) {
         const int r = idx / D, c = idx % D;
-        Qs[r * DP + c] = (q0 + r < n) ? Q[base + static_cast<size_t>(q0 + r) * D + c] : 0.f;
+        Qs[r * DP + c] = (q0 + r < nq) ? Q[base + static_cast<size_t>(q0 + r) * D + c] : 0.f;
+    }
+    // visible keys [klo[i], khi[i]] of this thread's 4 rows
+    int klo[4], khi[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        long long lo, hi;
+        visible_keys(mk, q0 + ty * 4 + i, q0 + ty * 4 + i, lo, hi);
+        klo[i] = clamp_int(lo);
+        khi[i] = clamp_int(hi);
     }
 
     float m[4], l[4], acc[4][OC];
@@ -60,14 +70,17 @@ __global__ void __launch_bounds__(256) fwd_f32_kernel(const float* __restrict__ 
         for (int c = 0; c < OC; ++c) acc[i][c] = 0.f;
     }
 
-    const int n_kv = (n + kBN - 1) / kBN;
-    const int kv_end = causal ? min(n_kv, (min(q0 + kBM, n) - 1) / kBN + 1) : n_kv;
-    for (int kt = 0; kt < kv_end; ++kt) {
+    // key tiles that hold a key some row of this tile sees
+    long long tlo, thi;
+    visible_keys(mk, q0, min(q0 + kBM, nq) - 1, tlo, thi);
+    const int kv_begin = tlo <= thi ? static_cast<int>(tlo / kBN) : 0;
+    const int kv_end = tlo <= thi ? static_cast<int>(thi / kBN) + 1 : 0;
+    for (int kt = kv_begin; kt < kv_end; ++kt) {
         const int k0 = kt * kBN;
         __syncthreads();
         for (int idx = tid; idx < kBN * D; idx += 256) {
             const int r = idx / D, c = idx % D;
-            const bool in = k0 + r < n;
+            const bool in = k0 + r < nk;
             const size_t g = kvbase + static_cast<size_t>(k0 + r) * D + c;
             Ks[r * DP + c] = in ? K[g] : 0.f;
             Vs[r * D + c] = in ? V[g] : 0.f;
@@ -94,12 +107,11 @@ __global__ void __launch_bounds__(256) fwd_f32_kernel(const float* __restrict__ 
 
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const int qidx = q0 + ty * 4 + i;
             float mx = -INFINITY;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const int kidx = k0 + tx + 16 * c;
-                s[i][c] = (kidx >= n || (causal && kidx > qidx)) ? -INFINITY : s[i][c] * scale;
+                s[i][c] = (kidx < klo[i] || kidx > khi[i]) ? -INFINITY : s[i][c] * scale;
                 mx = fmaxf(mx, s[i][c]);
             }
 #pragma unroll
@@ -147,12 +159,14 @@ __global__ void __launch_bounds__(256) fwd_f32_kernel(const float* __restrict__ 
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int qidx = q0 + ty * 4 + i;
-        if (qidx >= n) continue;
-        const float inv = 1.f / l[i];
+        if (qidx >= nq) continue;
+        // a row that sees no key: l = 0, accumulator 0 -> O = 0, LSE = -inf
+        const float inv = l[i] > 0.f ? 1.f / l[i] : 0.f;
 #pragma unroll
         for (int c = 0; c < OC; ++c)
             O[base + static_cast<size_t>(qidx) * D + tx + 16 * c] = acc[i][c] * inv;
-        if (tx == 0) lse[static_cast<size_t>(bh) * n + qidx] = m[i] + logf(l[i]);
+        if (tx == 0)
+            lse[static_cast<size_t>(bh) * nq + qidx] = l[i] > 0.f ? m[i] + logf(l[i]) : -INFINITY;
     }
 }
 
@@ -162,14 +176,15 @@ cudaError_t launch_fwd_f32_d(const FwdArgs& a, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(fwd_f32_kernel<D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    const int nqt = (a.n + kBM - 1) / kBM;
+    const int nqt = (a.nq + kBM - 1) / kBM;
     const long long bh = static_cast<long long>(a.B) * a.H;
     if (bh > 65535) return cudaErrorInvalidConfiguration;
     dim3 grid(nqt, static_cast<unsigned>(bh));
     fwd_f32_kernel<D><<<grid, 256, smem, stream>>>(
         static_cast<const float*>(a.q), static_cast<const float*>(a.k),
-        static_cast<const float*>(a.v), static_cast<float*>(a.o), a.lse, a.n, nqt, a.scale,
-        a.causal, a.H / a.Hkv);
+        static_cast<const float*>(a.v), static_cast<float*>(a.o), a.lse,
+        MaskSpec{a.nq, a.nk, a.wl, a.wr, static_cast<long long>(a.nk) - a.nq}, nqt, a.scale,
+        a.H / a.Hkv);
     return cudaGetLastError();
 }
 

@@ -7,16 +7,73 @@
 
 namespace attn {
 
+// Which keys each query sees. Query i (of nq) is aligned with key i + off, off = nk - nq (the last
+// query with the last key); key j is visible iff  i + off - wl <= j <= i + off + wr, a negative
+// wl or wr meaning unbounded on that side. (wl, wr) = (-1, 0) with nq = nk is the causal mask,
+// (-1, -1) no mask, (w, w) the sliding window of "Attention Mechanism ...", §4.5.
+// Because both bounds grow with i, the keys seen by a block of consecutive queries form one
+// contiguous range, and the queries that see a block of keys do too; host and device derive the
+// tile ranges of both passes from the functions below, so the passes agree on which (query tile,
+// key tile) pairs meet.
+struct MaskSpec {
+    int nq, nk;
+    int wl, wr;
+    long long off;
+};
+
+__host__ __device__ inline long long floor_div(long long a, long long b) {
+    return a >= 0 ? a / b : -((-a + b - 1) / b);
+}
+
+// Keys [lo, hi] (clipped to [0, nk)) seen by some query in rows [a, b] (b < nq); lo > hi if none.
+__host__ __device__ inline void visible_keys(const MaskSpec& m, long long a, long long b,
+                                             long long& lo, long long& hi) {
+    lo = m.wl < 0 ? 0 : a + m.off - m.wl;
+    hi = m.wr < 0 ? m.nk - 1 : b + m.off + m.wr;
+    if (lo < 0) lo = 0;
+    if (hi > m.nk - 1) hi = m.nk - 1;
+}
+
+// Query tiles [i0, i1) of `bq` rows that meet keys [c, e] (e < nk); i0 >= i1 if none.
+__host__ __device__ inline void visible_query_tiles(const MaskSpec& m, long long c, long long e,
+                                                    int bq, int& i0, int& i1) {
+    const long long ntiles = (m.nq + bq - 1) / bq;
+    long long t0 = 0, t1 = ntiles;
+    if (m.wr >= 0) {
+        const long long x = c - m.off - m.wr;   // first query whose window reaches key c
+        if (x > m.nq - 1) t0 = ntiles;
+        else if (x > 0) t0 = x / bq;
+    }
+    if (m.wl >= 0) {
+        const long long y = e - m.off + m.wl;   // last query whose window reaches back to key e
+        if (y < 0) t1 = 0;
+        else if (y / bq + 1 < t1) t1 = y / bq + 1;
+    }
+    i0 = static_cast<int>(t0);
+    i1 = static_cast<int>(t1 > t0 ? t1 : t0);
+}
+
+// First key tile of `bk` keys met by the query tile starting at row a.
+__host__ __device__ inline int first_key_tile(const MaskSpec& m, long long a, int bk) {
+    if (m.wl < 0) return 0;
+    const long long lo = a + m.off - m.wl;
+    return lo <= 0 ? 0 : static_cast<int>(lo / bk);
+}
+
+__host__ __device__ inline int clamp_int(long long x) {
+    return x < -0x7fffffffLL ? -0x7fffffff : (x > 0x7fffffffLL ? 0x7fffffff : static_cast<int>(x));
+}
+
 struct FwdArgs {
     const void* q;
     const void* k;
     const void* v;
     void* o;
     float* lse;
-    int B, H, n, d;
+    int B, H, nq, nk, d;  // query rows, key rows
     int Hkv;          // K/V heads; query head h reads K/V head h / (H / Hkv)
     float scale;
-    int causal;
+    int wl, wr;       // visible window (see MaskSpec)
     uint64_t timeout_ns;
 };
 
@@ -30,13 +87,15 @@ struct BwdArgs {
     void* dq;
     void* dk;
     void* dv;
-    int B, H, n, d;
+    int B, H, nq, nk, d;  // query rows, key rows
     int Hkv;          // K/V heads (dk, dv have Hkv heads)
     float scale;
-    int causal;
+    int wl, wr;       // visible window (see MaskSpec)
     int deterministic;
+    // n_pad = nq rounded up to a multiple of 128
     float* Dvec;      // workspace: B*H*n_pad, D_i = rowsum(dO∘O) (0 on padding rows)
-    float* L2vec;     // workspace: B*H*n_pad, LSE_i·log2(e) (+inf on padding rows)
+    float* L2vec;     // workspace: B*H*n_pad, LSE_i·log2(e) (+inf on padding rows and on rows
+                      // that see no key)
     float* dq_acc;    // workspace: B*H*n_pad*d
     int* sems;        // workspace: B*H*(n_pad/64), deterministic mode only
     uint64_t timeout_ns;

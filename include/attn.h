@@ -83,6 +83,23 @@ int attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* ls
  * one int semaphore per 64 query rows. */
 size_t attn_bwd_workspace_bytes(int B, int H, int n, int d, int deterministic);
 
+/* Masked and cross-length attention. Sliding window: "Attention Mechanism: Revolusi
+ * Representasi Sequence", §4.5 "Sparse Attention" (each token attends only to neighbours within
+ * ±w); cross-attention: same page, §4.2 (queries from one sequence, keys and values from another,
+ * so nq and nk differ).
+ *   q, o: (B, H, nq, d); k, v: (B, Hkv, nk, d); lse: (B, H, nq); layouts and dtypes as attn_fwd.
+ *   Query i is aligned with key i + (nk - nq) (the last query with the last key). Key j is
+ *   visible to query i iff  i + (nk - nq) - window_left <= j <= i + (nk - nq) + window_right;
+ *   a negative window_left / window_right means unbounded on that side. So (-1, 0) with nq == nk
+ *   is attn_fwd's causal mask, (-1, -1) no mask, (w, w) the page's ±w window, (w, 0) a causal
+ *   window of w + 1 keys.
+ *   A query that sees no key (possible when nq > nk or with a window that falls outside the keys)
+ *   gets o = 0 and lse = -inf.
+ * Errors as attn_fwd; nk < 1 is ATTN_ERR_INVALID. */
+int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
+                int B, int H, int Hkv, int nq, int nk, int d, float scale,
+                int window_left, int window_right, int dtype, void* stream);
+
 /* Backward pass (bf16 only). Inputs q, k, v, o, dO (bf16) and lse (fp32, from attn_fwd with the
  * same scale and causal flag). Writes dq, dk, dv (bf16). The workspace (caller-owned device
  * memory of at least attn_bwd_workspace_bytes() bytes, 256-byte aligned) is overwritten.
@@ -103,6 +120,17 @@ int attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, con
                  const float* lse, void* dq, void* dk, void* dv,
                  int B, int H, int Hkv, int n, int d, float scale, int causal, int dtype,
                  int deterministic, void* workspace, size_t ws_bytes, void* stream);
+
+/* Backward pass of attn_fwd_ex (bf16 only): dq (B, H, nq, d); dk, dv (B, Hkv, nk, d), summed over
+ * the query heads of each K/V head. Keys that no query sees get dk = dv = 0. The workspace is
+ * attn_bwd_workspace_bytes(B, H, nq, d, deterministic) (query rows). Everything else as attn_bwd;
+ * the deterministic mode adds the dQ partials of a query tile in increasing key-tile order,
+ * starting from the first key tile that the tile meets. */
+int attn_bwd_ex(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                const float* lse, void* dq, void* dk, void* dv,
+                int B, int H, int Hkv, int nq, int nk, int d, float scale,
+                int window_left, int window_right, int dtype, int deterministic,
+                void* workspace, size_t ws_bytes, void* stream);
 
 /* Backward pass without a caller workspace, for callers that cannot allocate device memory where
  * they run it (e.g. code inside a host framework that owns all device allocations, or a loop that

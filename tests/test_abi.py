@@ -12,6 +12,7 @@ FAKE = 1 << 20          # an aligned, never-dereferenced pointer value (validati
 def test_every_declared_function_is_exported():
     names = ea.declared_functions()
     assert {"attn_fwd", "attn_bwd", "attn_fwd_gqa", "attn_bwd_gqa", "attn_bwd_noalloc",
+            "attn_fwd_ex", "attn_bwd_ex",
             "attn_bwd_workspace_bytes", "attn_get_device_status",
             "attn_error_string", "attn_version", "attn_set_wait_timeout_us",
             "attn_selftest_wait_timeout"} <= set(names)
@@ -107,3 +108,21 @@ def test_gqa_rejects_head_counts_that_do_not_divide():
     b = [ctypes.c_void_p(FAKE)] * 9
     assert ea.attn_bwd_gqa(*b, 1, 6, 4, 128, 64, 0.125, 0, ea.ATTN_BF16, 0, ctypes.c_void_p(FAKE),
                            need, None) == ea.ATTN_ERR_INVALID
+
+
+def test_ex_rejects_bad_lengths_and_heads():
+    a = [ctypes.c_void_p(FAKE)] * 5
+    f = lambda B, H, Hkv, nq, nk, d=64: ea.attn_fwd_ex(*a, B, H, Hkv, nq, nk, d, 0.125, 4, 4,
+                                                       ea.ATTN_BF16, None)
+    assert f(1, 2, 2, 128, 0) == ea.ATTN_ERR_INVALID
+    assert f(1, 2, 2, 0, 128) == ea.ATTN_ERR_INVALID
+    assert f(1, 6, 4, 128, 128) == ea.ATTN_ERR_INVALID
+    assert f(1, 2, 2, 128, 64, d=80) == ea.ATTN_ERR_UNSUPPORTED
+    b = [ctypes.c_void_p(FAKE)] * 9
+    need = ea.attn_bwd_workspace_bytes(1, 2, 128, 64, 0)
+    g = lambda nq, nk, ws_bytes=need, dtype=ea.ATTN_BF16: ea.attn_bwd_ex(
+        *b, 1, 2, 2, nq, nk, 64, 0.125, -1, 0, dtype, 0, ctypes.c_void_p(FAKE), ws_bytes, None)
+    assert g(128, 0) == ea.ATTN_ERR_INVALID
+    assert g(128, 64, dtype=ea.ATTN_FP32) == ea.ATTN_ERR_UNSUPPORTED
+    # the workspace follows the query length
+    assert g(300, 64) == ea.ATTN_ERR_WORKSPACE
