@@ -70,10 +70,19 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def csrc_digest():
+# Sources that determine each profiled kernel: its own file plus the shared headers.
+KERNEL_SOURCES = {
+    "bwd_main_q64_kernel": ("bwd_bf16.cu", "kernels.h", "sm100_ptx.cuh"),
+    "fwd_bf16_kernel": ("fwd_bf16.cu", "kernels.h", "sm100_ptx.cuh"),
+}
+
+
+def csrc_digest(kernel=None):
+    """Hash of the CUDA sources of `kernel` (all of csrc/ when None)."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "exact_attention_138_b200", "csrc")
-    for name in sorted(os.listdir(d)):
+    names = KERNEL_SOURCES.get(kernel) or sorted(os.listdir(d))
+    for name in sorted(names):
         with open(os.path.join(d, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -90,7 +99,8 @@ def recorded_traffic(kernel, workload):
     except (OSError, ValueError):
         return None
     entry = rec.get(kernel)
-    if not entry or entry.get("csrc_sha") != csrc_digest() or entry.get("workload") != workload:
+    if (not entry or entry.get("csrc_sha") != csrc_digest(kernel)
+            or entry.get("workload") != workload):
         return None
     return entry.get("bytes_per_launch")
 

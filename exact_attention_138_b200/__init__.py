@@ -53,6 +53,11 @@ _lib.attn_fwd_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f
 _lib.attn_bwd_ex.restype = _i
 _lib.attn_bwd_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
                              _f, _i, _i, _i, _i, _vp, _sz, _vp]
+_ll = ctypes.c_longlong
+_lib.attn_ring_merge.restype = _i
+_lib.attn_ring_merge.argtypes = [_vp, _vp, _vp, _vp, _ll, _i, _i, _i, _vp, _i, _vp]
+_lib.attn_ring_accumulate.restype = _i
+_lib.attn_ring_accumulate.argtypes = [_vp, _vp, _ll, _i, _i, _vp, _i, _vp]
 _lib.attn_bwd_workspace_bytes.restype = _sz
 _lib.attn_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
 _lib.attn_bwd.restype = _i
@@ -120,6 +125,16 @@ def attn_bwd_ex(q, k, v, o, dO, lse, dq, dk, dv, B, H, Hkv, nq, nk, d, scale, wi
     return _lib.attn_bwd_ex(q, k, v, o, dO, lse, dq, dk, dv, B, H, Hkv, nq, nk, d, scale,
                             window_left, window_right, dtype, deterministic, workspace, ws_bytes,
                             stream)
+
+
+def attn_ring_merge(o_acc, lse_acc, o_part, lse_part, rows, d, part_dtype, first, o_out,
+                    out_dtype, stream) -> int:
+    return _lib.attn_ring_merge(o_acc, lse_acc, o_part, lse_part, rows, d, part_dtype, first,
+                                o_out, out_dtype, stream)
+
+
+def attn_ring_accumulate(acc, part, count, part_dtype, first, out, out_dtype, stream) -> int:
+    return _lib.attn_ring_accumulate(acc, part, count, part_dtype, first, out, out_dtype, stream)
 
 
 def attn_bwd_workspace_bytes(B, H, n, d, deterministic) -> int:
@@ -280,3 +295,26 @@ def backward(q, k, v, o, do, lse, causal=False, scale=None, deterministic=False,
 def device_status(stream=None) -> int:
     """Synchronise and return/clear the device status word (ATTN_OK or ATTN_ERR_TIMEOUT)."""
     return attn_get_device_status(_stream_handle(stream))
+
+
+def ring_merge(o_acc, lse_acc, o_part, lse_part, first=False, out=None, stream=None):
+    """Fold a partial (o_part, lse_part) into the running fp32 (o_acc, lse_acc) in place; with
+    `out` also write the merged output there (see attn_ring_merge)."""
+    d = o_acc.shape[-1]
+    rows = lse_acc.numel()
+    rc = attn_ring_merge(_ptr(o_acc), _ptr(lse_acc), _ptr(o_part), _ptr(lse_part), rows, d,
+                         _dtype_code(o_part), int(bool(first)),
+                         _ptr(out) if out is not None else None,
+                         _dtype_code(out) if out is not None else ATTN_BF16,
+                         _stream_handle(stream))
+    _check(rc, "attn_ring_merge")
+
+
+def ring_accumulate(acc, part=None, first=False, out=None, stream=None):
+    """acc (fp32) = (0 if first else acc) + part; with `out` also write the sum there."""
+    rc = attn_ring_accumulate(_ptr(acc), _ptr(part) if part is not None else None, acc.numel(),
+                              _dtype_code(part) if part is not None else ATTN_BF16,
+                              int(bool(first)), _ptr(out) if out is not None else None,
+                              _dtype_code(out) if out is not None else ATTN_BF16,
+                              _stream_handle(stream))
+    _check(rc, "attn_ring_accumulate")

@@ -8,6 +8,7 @@
 
 #include "../../include/attn.h"
 #include "kernels.h"
+#include "ring.h"
 #include "sm100_ptx.cuh"
 
 namespace attn {
@@ -233,6 +234,34 @@ int attn_bwd_ex(const void* q, const void* k, const void* v, const void* o, cons
                 int deterministic, void* workspace, size_t ws_bytes, void* stream) {
     return bwd_impl(q, k, v, o, dO, lse, dq, dk, dv, B, H, Hkv, nq, nk, d, scale, window_left,
                     window_right, dtype, deterministic, workspace, ws_bytes, stream);
+}
+
+int attn_ring_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
+                    long long rows, int d, int part_dtype, int first, void* o_out, int out_dtype,
+                    void* stream) {
+    if (!o_acc || !lse_acc || !o_part || !lse_part || rows < 1) return ATTN_ERR_INVALID;
+    if (d != 32 && d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if ((part_dtype != ATTN_BF16 && part_dtype != ATTN_FP32) ||
+        (o_out && out_dtype != ATTN_BF16 && out_dtype != ATTN_FP32))
+        return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(o_acc) || !aligned16(o_part) || (o_out && !aligned16(o_out)))
+        return ATTN_ERR_INVALID;
+    return to_code(launch_ring_merge(o_acc, lse_acc, o_part, lse_part, rows, d,
+                                     part_dtype == ATTN_BF16, first ? 1 : 0, o_out,
+                                     out_dtype == ATTN_BF16, static_cast<cudaStream_t>(stream)));
+}
+
+int attn_ring_accumulate(float* acc, const void* part, long long count, int part_dtype, int first,
+                         void* out, int out_dtype, void* stream) {
+    if (!acc || count < 1 || count % 8 != 0) return ATTN_ERR_INVALID;
+    if ((part && part_dtype != ATTN_BF16 && part_dtype != ATTN_FP32) ||
+        (out && out_dtype != ATTN_BF16 && out_dtype != ATTN_FP32))
+        return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(acc) || (part && !aligned16(part)) || (out && !aligned16(out)))
+        return ATTN_ERR_INVALID;
+    return to_code(launch_ring_accumulate(acc, part, count, part_dtype == ATTN_BF16,
+                                          first ? 1 : 0, out, out_dtype == ATTN_BF16,
+                                          static_cast<cudaStream_t>(stream)));
 }
 
 void attn_set_bwd_phase_events(void* const* events) {

@@ -5,3 +5,4 @@
 #include "fwd_f32.cu"
 #include "bwd_bf16.cu"
 #include "bwd_noalloc.cu"
+#include "ring.cu"

@@ -164,6 +164,36 @@ unsigned attn_set_wait_timeout_us(unsigned us);
  * attn_get_device_status(). Never faults or hangs the device. */
 int attn_selftest_wait_timeout(unsigned timeout_us, void* stream);
 
+/* Ring attention building blocks ("Attention Mechanism: Revolusi Representasi Sequence", §16 "Long
+ * Context Training", Ring Attention: the sequence is split across GPUs and attention over all
+ * chunks is computed by passing K/V chunks around a ring). Each hop attends the local queries to
+ * one K/V chunk (attn_fwd_ex / attn_bwd_ex); these two calls combine the hops. Both are
+ * elementwise, asynchronous on `stream`, and validate before launching.
+ *
+ * attn_ring_merge: folds one hop's partial result into a running one, row by row:
+ *     LSE = log(exp(lse_acc) + exp(lse_part)),
+ *     o_acc = exp(lse_acc - LSE)·o_acc + exp(lse_part - LSE)·o_part,   lse_acc = LSE,
+ *   which is exact because each partial output is normalised by its own exp(LSE). A row with
+ *   lse = -inf (no visible key in that chunk) has weight 0; rows with no key anywhere stay o = 0,
+ *   lse = -inf.
+ *   o_acc: rows x d fp32 (caller-owned device memory, 16-byte aligned); lse_acc: rows fp32;
+ *   o_part: rows x d in part_dtype (ATTN_BF16 or ATTN_FP32); lse_part: rows fp32 (natural log).
+ *   first != 0: o_acc / lse_acc are not read (they are initialised from the partial).
+ *   o_out != NULL: the merged rows are also written there in out_dtype (the final hop's output).
+ *   Errors: null pointer or rows < 1 -> ATTN_ERR_INVALID; d not in {32, 64, 128} or an unknown
+ *   dtype -> ATTN_ERR_UNSUPPORTED; misaligned pointer -> ATTN_ERR_INVALID. */
+int attn_ring_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
+                    long long rows, int d, int part_dtype, int first, void* o_out, int out_dtype,
+                    void* stream);
+
+/* attn_ring_accumulate: acc (count fp32) = (first ? 0 : acc) + part, where part (count elements
+ * in part_dtype) may be NULL (no addition); with out != NULL the sum is also written there in
+ * out_dtype. Used for the gradients of ring attention: dQ accumulates over the hops of the local
+ * queries, dK / dV accumulate while travelling with their K / V chunk.
+ *   count must be a positive multiple of 8; pointers 16-byte aligned (else ATTN_ERR_INVALID). */
+int attn_ring_accumulate(float* acc, const void* part, long long count, int part_dtype, int first,
+                         void* out, int out_dtype, void* stream);
+
 /* Measurement hook. `events` is NULL (recording off, the default) or an array of 4 cudaEvent_t
  * created by the caller. While set, every attn_bwd call records, on its stream, events[0] before
  * its preprocess kernel (D = rowsum(dO∘O)), events[1] before its main kernel, events[2] after

@@ -1,0 +1,70 @@
+"""CPU stand-ins (fp64 numpy) for the four per-hop operations of the ring schedule, so that the
+multi-rank schedule and its point-to-point exchanges can run as gloo ranks on the CPU. The hop
+forward is the oracle's masked definition; the hop backward uses the global LSE and O (as the
+CUDA hop kernel does): P = exp(scale·q·k - LSE), D = rowsum(dO∘O), dS = P∘(dP - D)."""
+import numpy as np
+import torch
+
+import oracle
+
+
+def _np(t):
+    return t.detach().cpu().numpy().astype(np.float64)
+
+
+def _visible(nq, nk, wl, wr):
+    i = np.arange(nq)[:, None] + (nk - nq)
+    j = np.arange(nk)[None, :]
+    vis = np.ones((nq, nk), bool)
+    if wl >= 0:
+        vis &= j >= i - wl
+    if wr >= 0:
+        vis &= j <= i + wr
+    return vis
+
+
+class CpuOps:
+    def fwd(self, q, k, v, scale, window):
+        o, lse = oracle.fwd_ex(q.float().numpy(), k.float().numpy(), v.float().numpy(), scale,
+                               window[0], window[1])
+        return torch.from_numpy(o), torch.from_numpy(lse)
+
+    def bwd(self, q, k, v, o, do, lse, scale, window, deterministic):
+        Q, K, V, O, dO, L = (_np(x) for x in (q, k, v, o, do, lse))
+        H, Hkv = Q.shape[1], K.shape[1]
+        K, V = np.repeat(K, H // Hkv, axis=1), np.repeat(V, H // Hkv, axis=1)
+        vis = _visible(Q.shape[2], K.shape[2], *window)
+        S = np.einsum("bhid,bhjd->bhij", Q, K) * scale
+        P = np.where(vis, np.exp(S - L[..., None]), 0.0)
+        dP = np.einsum("bhid,bhjd->bhij", dO, V)
+        D = (dO * O).sum(-1)
+        dS = P * (dP - D[..., None])
+        dq = scale * np.einsum("bhij,bhjd->bhid", dS, K)
+        dk = scale * np.einsum("bhij,bhid->bhjd", dS, Q)
+        dv = np.einsum("bhij,bhid->bhjd", P, dO)
+        B, _, n, d = dk.shape
+        dk = dk.reshape(B, Hkv, H // Hkv, n, d).sum(2)
+        dv = dv.reshape(B, Hkv, H // Hkv, n, d).sum(2)
+        return tuple(torch.from_numpy(x) for x in (dq, dk, dv))
+
+    def merge(self, o_acc, lse_acc, o_part, lse_part, first, out):
+        la = np.full(lse_part.shape, -np.inf) if first else _np(lse_acc)
+        lb = _np(lse_part)
+        L = np.logaddexp(la, lb)
+        with np.errstate(invalid="ignore"):
+            wa = np.where(np.isneginf(la), 0.0, np.exp(la - L))
+            wb = np.where(np.isneginf(lb), 0.0, np.exp(lb - L))
+        oa = np.zeros(o_acc.shape) if first else _np(o_acc)
+        o = wa[..., None] * oa + wb[..., None] * _np(o_part)
+        o_acc.copy_(torch.from_numpy(o))
+        lse_acc.copy_(torch.from_numpy(L))
+        if out is not None:
+            out.copy_(torch.from_numpy(o))
+
+    def accumulate(self, acc, part, first, out):
+        a = np.zeros(acc.shape) if first else _np(acc)
+        if part is not None:
+            a = a + _np(part)
+        acc.copy_(torch.from_numpy(a))
+        if out is not None:
+            out.copy_(torch.from_numpy(a))

@@ -1,0 +1,83 @@
+"""Ring attention's multi-rank schedule on CPU ranks (gloo, point-to-point isend/irecv): each
+rank holds one chunk of the sequence, K/V chunks travel around the ring, partial results are
+merged and the dK/dV accumulators travel back to their owners. The per-hop arithmetic is the CPU
+stand-in of tests/ring_cpu_ops.py; the gathered results must equal the oracle's attention over
+the whole sequence ("Attention Mechanism ...", §16 Ring Attention)."""
+import math
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _inputs(world, n_chunk, H, Hkv, d):
+    g = torch.Generator().manual_seed(41)
+    n = world * n_chunk
+    q = torch.randn(1, H, n, d, generator=g).double()
+    k = torch.randn(1, Hkv, n, d, generator=g).double()
+    v = torch.randn(1, Hkv, n, d, generator=g).double()
+    do = torch.randn(1, H, n, d, generator=g).double()
+    return q, k, v, do
+
+
+def _worker(rank, world, port, causal, n_chunk, H, Hkv, d, out):
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from exact_attention_138_b200 import ring
+    from ring_cpu_ops import CpuOps
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        q, k, v, do = _inputs(world, n_chunk, H, Hkv, d)
+        sl = slice(rank * n_chunk, (rank + 1) * n_chunk)
+        mine = [x[:, :, sl].contiguous() for x in (q, k, v, do)]
+        scale = 1.0 / math.sqrt(d)
+        ops = CpuOps()
+        o, lse = ring.ring_forward(mine[0], mine[1], mine[2], causal=causal, scale=scale, ops=ops)
+        dq, dk, dv = ring.ring_backward(mine[0], mine[1], mine[2], o, mine[3], lse, causal=causal,
+                                        scale=scale, ops=ops)
+        out[rank] = tuple(x.numpy() for x in (o, lse, dq, dk, dv))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,causal,H,Hkv", [(2, True, 2, 2), (2, False, 2, 1), (3, True, 4, 2)])
+def test_ring_schedule_on_cpu_ranks_equals_full_attention(world, causal, H, Hkv):
+    import oracle
+    n_chunk, d = 24, 8
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_worker, args=(world, _free_port(), causal, n_chunk, H, Hkv, d, out),
+                       nprocs=world, join=True, start_method="spawn")
+    q, k, v, do = _inputs(world, n_chunk, H, Hkv, d)
+    scale = 1.0 / math.sqrt(d)
+    qf, kf, vf, dof = (x.float().numpy() for x in (q, k, v, do))
+    ro, rlse = oracle.fwd_ex(qf, kf, vf, scale, -1, 0 if causal else -1)
+    rq, rk, rv = oracle.bwd_ex(qf, kf, vf, dof, scale, -1, 0 if causal else -1)
+    got = [np.concatenate([out[r][i] for r in range(world)], axis=2) for i in range(5)]
+    np.testing.assert_allclose(got[0], ro, rtol=0, atol=1e-5)
+    np.testing.assert_allclose(got[1], rlse, rtol=0, atol=1e-5)
+    for g, want in zip(got[2:], (rq, rk, rv)):
+        np.testing.assert_allclose(g, want, rtol=0, atol=1e-5)
+
+
+def test_hop_windows():
+    from exact_attention_138_b200 import ring
+    assert ring.hop_window(3, 1, True) == (-1, -1)
+    assert ring.hop_window(2, 2, True) == (-1, 0)
+    assert ring.hop_window(1, 2, True) is None
+    assert all(ring.hop_window(p, s, False) == (-1, -1) for p in range(3) for s in range(3))
