@@ -54,6 +54,9 @@ _lib.attn_bwd_ex.restype = _i
 _lib.attn_bwd_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
                              _f, _i, _i, _i, _i, _vp, _sz, _vp]
 _ll = ctypes.c_longlong
+_lib.attn_fwd_fp8.restype = _i
+_lib.attn_fwd_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i, _f, _f,
+                              _f, _vp]
 _lib.attn_ring_merge.restype = _i
 _lib.attn_ring_merge.argtypes = [_vp, _vp, _vp, _vp, _ll, _i, _i, _i, _vp, _i, _vp]
 _lib.attn_ring_accumulate.restype = _i
@@ -125,6 +128,12 @@ def attn_bwd_ex(q, k, v, o, dO, lse, dq, dk, dv, B, H, Hkv, nq, nk, d, scale, wi
     return _lib.attn_bwd_ex(q, k, v, o, dO, lse, dq, dk, dv, B, H, Hkv, nq, nk, d, scale,
                             window_left, window_right, dtype, deterministic, workspace, ws_bytes,
                             stream)
+
+
+def attn_fwd_fp8(q, k, v, o, lse, B, H, Hkv, nq, nk, d, scale, window_left, window_right,
+                 q_descale, k_descale, v_descale, stream) -> int:
+    return _lib.attn_fwd_fp8(q, k, v, o, lse, B, H, Hkv, nq, nk, d, scale, window_left,
+                             window_right, q_descale, k_descale, v_descale, stream)
 
 
 def attn_ring_merge(o_acc, lse_acc, o_part, lse_part, rows, d, part_dtype, first, o_out,
@@ -318,3 +327,31 @@ def ring_accumulate(acc, part=None, first=False, out=None, stream=None):
                               _dtype_code(out) if out is not None else ATTN_BF16,
                               _stream_handle(stream))
     _check(rc, "attn_ring_accumulate")
+
+
+def forward_fp8(q, k, v, q_descale=1.0, k_descale=1.0, v_descale=1.0, causal=False, scale=None,
+                out=None, lse=None, stream=None, window=None):
+    """O (bf16), LSE of attention with E4M3 inputs: q, k, v are torch.float8_e4m3fn (or uint8
+    holding E4M3 bytes) CUDA tensors (B,H,nq,d) / (B,Hkv,nk,d), d in {64, 128}; the real inputs
+    are q·q_descale, k·k_descale, v·v_descale. Masks as `forward`."""
+    import torch
+    for t in (q, k, v):
+        if t.dtype not in (torch.float8_e4m3fn, torch.uint8):
+            raise ValueError("forward_fp8 expects float8_e4m3fn (or uint8) tensors")
+    B, H, n, d = _dims(q)
+    kd = _dims(k)
+    if v.shape != k.shape or kd[0] != B or kd[3] != d or H % kd[1] != 0:
+        raise ValueError("k, v must be (B, Hkv, nk, d) with H a multiple of Hkv")
+    Hkv, nk = kd[1], kd[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H, n), dtype=torch.float32, device=q.device)
+    wl, wr = _window(causal, window)
+    rc = attn_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Hkv, n, nk, d,
+                      float(scale), wl, wr, float(q_descale), float(k_descale), float(v_descale),
+                      _stream_handle(stream))
+    _check(rc, "attn_fwd_fp8")
+    return out, lse

@@ -83,22 +83,26 @@ int validate_common(int B, int H, int n, int d, float scale, int dtype) {
 
 }  // namespace
 
-cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int BH, int n, int d,
-                           int box_rows) {
+cudaError_t make_tmap(CUtensorMap* map, const void* base, int esize, int BH, int n, int d,
+                      int box_rows) {
     auto fn = encode_fn();
     if (!fn) return cudaErrorNotSupported;
-    const int chunk = d >= 64 ? 64 : d;
+    const int chunk = d * esize >= 128 ? 128 / esize : d;
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n),
                           static_cast<cuuint64_t>(BH)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
-                             static_cast<cuuint64_t>(d) * 2 * static_cast<cuuint64_t>(n)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * esize,
+                             static_cast<cuuint64_t>(d) * esize * static_cast<cuuint64_t>(n)};
     cuuint32_t box[3] = {static_cast<cuuint32_t>(chunk), static_cast<cuuint32_t>(box_rows), 1u};
     cuuint32_t estr[3] = {1u, 1u, 1u};
+    const int chunk_bytes = chunk * esize;
+    if (chunk_bytes != 128 && chunk_bytes != 64) return cudaErrorInvalidValue;
     const CUtensorMapSwizzle swz =
-        chunk == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
-                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        chunk_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    const CUtensorMapDataType dt =
+        esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    CUresult r = fn(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
@@ -148,6 +152,7 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
     a.scale = scale;
     a.wl = wl < 0 ? -1 : wl;
     a.wr = wr < 0 ? -1 : wr;
+    a.q_descale = a.k_descale = a.v_descale = 1.f;
     a.timeout_ns = static_cast<uint64_t>(g_timeout_us.load()) * 1000ull;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = (dtype == ATTN_BF16) ? launch_fwd_bf16(a, s) : launch_fwd_f32(a, s);
@@ -170,6 +175,32 @@ int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse
                 int dtype, void* stream) {
     return fwd_impl(q, k, v, o, lse, B, H, Hkv, nq, nk, d, scale, window_left, window_right, dtype,
                     stream);
+}
+
+int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int Hkv, int nq, int nk, int d, float scale, int window_left, int window_right,
+                 float q_descale, float k_descale, float v_descale, void* stream) {
+    if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID;
+    int rc = validate_common(B, H, nq, d, scale, ATTN_BF16);
+    if (rc) return rc;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (nk < 1 || Hkv < 1 || H % Hkv != 0) return ATTN_ERR_INVALID;
+    const float ds[3] = {q_descale, k_descale, v_descale};
+    for (float x : ds)
+        if (!(x > 0.f) || !isfinite(x)) return ATTN_ERR_INVALID;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return ATTN_ERR_INVALID;
+    FwdArgs a;
+    a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
+    a.B = B; a.H = H; a.nq = nq; a.nk = nk; a.d = d; a.Hkv = Hkv;
+    a.scale = scale;
+    a.wl = window_left < 0 ? -1 : window_left;
+    a.wr = window_right < 0 ? -1 : window_right;
+    a.q_descale = q_descale;
+    a.k_descale = k_descale;
+    a.v_descale = v_descale;
+    a.timeout_ns = static_cast<uint64_t>(g_timeout_us.load()) * 1000ull;
+    return to_code(launch_fwd_fp8(a, static_cast<cudaStream_t>(stream)));
 }
 
 size_t attn_bwd_workspace_bytes(int B, int H, int n, int d, int deterministic) {

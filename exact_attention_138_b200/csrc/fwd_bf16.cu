@@ -1,4 +1,5 @@
-// Forward pass, bf16 in / bf16 out, fp32 accumulation, on the sm_100a tensor cores.
+// Forward pass on the sm_100a tensor cores: bf16 in / bf16 out, or E4M3 (fp8) in / bf16 out, with
+// fp32 accumulation.
 //
 // The method is the tiled forward pass with online softmax: Q, K and V are split into tiles held
 // on chip, each tile updates a running row max m and row sum l, and the running output is
@@ -18,6 +19,12 @@
 //               back over S.
 //   The two query tiles alternate, so the tensor cores run one tile's MMAs while the other tile's
 //   softmax runs. TMEM (512 columns): O_0 | O_1 | S_0 (P_0) | S_1 (P_1), 128 columns each.
+//   FP8 variant ("Flash Attention Nedir?" and "Apa itu FlashAttention": FlashAttention-3 runs the
+//   same method in FP8 on Hopper): Q, K, V are E4M3 with one dequantisation factor per tensor;
+//   both products run as kind::f8f6f4 MMAs (32 keys or features per instruction), S is scaled by
+//   scale·q_descale·k_descale, P is rounded to E4M3 (values up to 2^8 under the lazy rescale,
+//   within E4M3's range of 448) and O is multiplied by v_descale in the epilogue. An E4M3 tile with
+//   d = 128 has the byte layout of a bf16 tile with d = 64 (rows of 128 bytes).
 //   Masks (causal, sliding window, query/key lengths that differ; see MaskSpec): each query tile
 //   visits only the key tiles that hold a key it can see; the two tiles of a pair stream the
 //   union of their ranges once. A row that sees no key gets O = 0 and LSE = -inf.
@@ -37,18 +44,21 @@ constexpr float kLog2e = 1.44269504088896340736f;
 constexpr int kExpFmaPer8 = ATTN_FWD_EXP_FMA_PER8;   // column pairs (of every 8) whose exp2 runs
                                                      // on the FMA pipe
 
-template <int D>
+template <int D, bool F8>
 struct FwdCfg {
+    static constexpr int EB = F8 ? 1 : 2;                // bytes per element
     static constexpr int BM = 128;                       // query rows per tile
     static constexpr int BN = 128;                       // keys per tile
-    static constexpr int CW = D >= 64 ? 64 : D;          // elements per swizzle row
+    static constexpr int CW = D * EB >= 128 ? 128 / EB : D;   // elements per swizzle row
     static constexpr int NCH = D / CW;                   // swizzle chunks per tile row
-    static constexpr int SWB = CW * 2;                   // swizzle width in bytes
+    static constexpr int SWB = CW * EB;                  // swizzle width in bytes (128 or 64)
     static constexpr uint32_t SWZ = SWB == 128 ? 2u : 4u;
+    static constexpr int KSTEP = 32 / EB;                // K elements per MMA instruction
     static constexpr int CHUNK = 128 * SWB;              // bytes of one [128 rows x CW] chunk
     static constexpr int TILE = NCH * CHUNK;             // bytes of one 128 x D tile
-    static constexpr int STAGES = D == 128 ? 2 : 3;
+    static constexpr int STAGES = TILE >= 32768 ? 2 : 3;
     static constexpr int SMEM = (2 + 2 * STAGES) * TILE + 512;
+    static_assert(SWB == 128 || SWB == 64, "tile rows of 64 or 128 bytes");
 };
 
 struct FwdBars {
@@ -67,6 +77,7 @@ struct FwdKParams {
     int kv_group;     // query heads per K/V head (grouped-query attention); 1 for MHA
     MaskSpec mask;
     float scale_log2;
+    float o_scale;    // output multiplier (v_descale for E4M3 inputs, 1 for bf16)
     uint64_t timeout_ns;
 };
 
@@ -82,17 +93,30 @@ __device__ __forceinline__ void drain_wait_fwd(uint64_t* bar, uint32_t parity, u
         }
 }
 
-// Single-lane issue helpers for a converged warp (see elect_one).
-#define FMMA_SS(...) do { if (elect_one()) mma_ss(__VA_ARGS__); } while (0)
-#define FMMA_TS(...) do { if (elect_one()) mma_ts(__VA_ARGS__); } while (0)
+// Single-lane commit for a converged warp (see elect_one).
 #define FMMA_COMMIT(bar) do { if (elect_one()) mma_commit(bar); } while (0)
 
-template <int D>
-__global__ void __launch_bounds__(kFwdThreads, 1)
-    fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
-                    const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const FwdKParams p) {
-    using C = FwdCfg<D>;
+// Writes P of columns c, c+1 over the raw scores in u (c even, loop unrolled): bf16 pairs fill
+// u[c/2]; E4M3 quadruples fill u[c/4] (columns c, c+1 in the low half when c % 4 == 0). Only
+// entries at or below c/2 are written, all already consumed.
+template <bool F8>
+__device__ __forceinline__ void store_p(uint32_t* u, int c, float p0, float p1) {
+    if constexpr (F8) {
+        const uint32_t h = pack_e4m3x2(p0, p1);
+        if ((c & 2) == 0) u[c / 4] = h;
+        else u[c / 4] |= h << 16;
+    } else {
+        u[c / 2] = pack_bf16x2(p0, p1);
+    }
+}
+
+template <int D, bool F8>
+__device__ __forceinline__ void fwd_body(const CUtensorMap* tmQ_, const CUtensorMap* tmK_,
+                                         const CUtensorMap* tmV_, const FwdKParams& p) {
+    using C = FwdCfg<D, F8>;
+    const CUtensorMap& tmQ = *tmQ_;
+    const CUtensorMap& tmK = *tmK_;
+    const CUtensorMap& tmV = *tmV_;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t* sQ = smem;                                   // 2 tiles
     uint8_t* sK = smem + 2 * C::TILE;                     // STAGES tiles
@@ -213,8 +237,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // ---------------------------------------------------------------- MMA issuer
         // The whole warp runs this loop (warp-uniform state); one elected lane issues.
         {
-            constexpr uint32_t idS = idesc_bf16_f32(128, 128, 0, 0);
-            constexpr uint32_t idPV = idesc_bf16_f32(128, D, 0, 1);
+            constexpr uint32_t idS = F8 ? idesc_e4m3_f32(128, 128, 0, 0) : idesc_bf16_f32(128, 128, 0, 0);
+            constexpr uint32_t idPV = F8 ? idesc_e4m3_f32(128, D, 0, 1) : idesc_bf16_f32(128, D, 0, 1);
+            auto mss = [](uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+                if (elect_one()) {
+                    if constexpr (F8) mma_ss_f8(d, a, b, id, acc);
+                    else mma_ss(d, a, b, id, acc);
+                }
+            };
+            auto mts = [](uint32_t d, uint32_t a, uint64_t b, uint32_t id, uint32_t acc) {
+                if (elect_one()) {
+                    if constexpr (F8) mma_ts_f8(d, a, b, id, acc);
+                    else mma_ts(d, a, b, id, acc);
+                }
+            };
             const uint32_t sQa = smem_addr(sQ), sKa = smem_addr(sK), sVa = smem_addr(sV);
             bool ok = U > 0 && bounded_wait_warp(&bars->q_full, 0, abort, lim);
             tc_fence_after();
@@ -243,20 +279,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 const SDesc a = dQ[g], b = dK[u % C::STAGES];
                 const uint32_t d = tmem + 256 + g * 128;
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t off =
-                        static_cast<uint32_t>((((ks * 16) / C::CW) * C::CHUNK + ((ks * 16) % C::CW) * 2) >> 4);
-                    FMMA_SS(d, sdesc_at(a, off), sdesc_at(b, off), idS, ks > 0 ? 1u : 0u);
+                for (int ks = 0; ks < D / C::KSTEP; ++ks) {
+                    const uint32_t off = static_cast<uint32_t>(
+                        (((ks * C::KSTEP) / C::CW) * C::CHUNK + ((ks * C::KSTEP) % C::CW) * C::EB) >> 4);
+                    mss(d, sdesc_at(a, off), sdesc_at(b, off), idS, ks > 0 ? 1u : 0u);
                 }
             };
             auto issue_pv = [&](int g, int u, bool accumulate) {
                 const SDesc b = dV[u % C::STAGES];
                 const uint32_t d = tmem + g * 128, a = tmem + 256 + g * 128;
-                FMMA_TS(d, a, sdesc_at(b, 0), idPV, accumulate ? 1u : 0u);
+                // one instruction takes KSTEP keys: 8 TMEM columns of P, KSTEP rows of V
+                mts(d, a, sdesc_at(b, 0), idPV, accumulate ? 1u : 0u);
 #pragma unroll
-                for (int ks = 1; ks < C::BN / 16; ++ks)
-                    FMMA_TS(d, a + ks * 8, sdesc_at(b, static_cast<uint32_t>((ks * 16 * C::SWB) >> 4)),
-                           idPV, 1u);
+                for (int ks = 1; ks < C::BN / C::KSTEP; ++ks)
+                    mts(d, a + ks * 8,
+                        sdesc_at(b, static_cast<uint32_t>((ks * C::KSTEP * C::SWB) >> 4)), idPV, 1u);
             };
             // Stream step u holds key tile Jmin + u. Query tile g uses steps [J0[g] - Jmin,
             // J0[g] - Jmin + T[g]); its S for step u+1 is issued during step u (or, for its first
@@ -414,7 +451,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
                     if (c & 2) rsb = f2_add(rsb, f2_pack(p0, p1));
                     else rsa = f2_add(rsa, f2_pack(p0, p1));
-                    u[c / 2] = pack_bf16x2(p0, p1);
+                    store_p<F8>(u, c, p0, p1);
                 }
             } else {
                 // kExpFmaPer8 of every 8 column pairs use the FMA-pipe exp2, the rest the MUFU
@@ -431,7 +468,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     }
                     if (c & 2) rsb = f2_add(rsb, f2_pack(p0, p1));
                     else rsa = f2_add(rsa, f2_pack(p0, p1));
-                    u[c / 2] = pack_bf16x2(p0, p1);
+                    store_p<F8>(u, c, p0, p1);
                 }
             }
             float ra0, ra1, rb0, rb1;
@@ -439,8 +476,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             f2_unpack(rsb, rb0, rb1);
             const float rs0 = ra0 + rb0, rs1 = ra1 + rb1;
             l += rs0 + rs1;
+            // P: 64 columns of bf16 pairs, or 32 columns of E4M3 quadruples
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
+            for (int h = 0; h < (F8 ? 1 : 2); ++h)
                 tmem_st32(tS + h * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[h * 32]));
             tmem_st_wait();
             tc_fence_before();
@@ -452,7 +490,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if (ok) {
                 tc_fence_after();
                 // a row that saw no key has l = 0 and an all-zero accumulator
-                const float inv_l = l > 0.f ? 1.f / l : 0.f;
+                const float inv_l = l > 0.f ? p.o_scale / l : 0.f;
                 __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) +
                                       (static_cast<size_t>(bh) * nq + qidx) * D;
 #pragma unroll
@@ -495,17 +533,36 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 }
 
 template <int D>
-cudaError_t launch_fwd_bf16_d(const FwdArgs& a, cudaStream_t stream) {
-    using C = FwdCfg<D>;
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
+                    const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const FwdKParams p) {
+    fwd_body<D, false>(&tmQ, &tmK, &tmV, p);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ,
+                   const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const FwdKParams p) {
+    fwd_body<D, true>(&tmQ, &tmK, &tmV, p);
+}
+
+template <int D, bool F8>
+cudaError_t launch_fwd_d(const FwdArgs& a, cudaStream_t stream) {
+    using C = FwdCfg<D, F8>;
     CUtensorMap mq, mk, mv;
     const int BH = a.B * a.H;
+    const int esize = F8 ? 1 : 2;
     cudaError_t e;
-    if ((e = make_tmap_bf16(&mq, a.q, BH, a.nq, D)) != cudaSuccess) return e;
+    if ((e = make_tmap(&mq, a.q, esize, BH, a.nq, D)) != cudaSuccess) return e;
     const int BHkv = a.B * a.Hkv;
-    if ((e = make_tmap_bf16(&mk, a.k, BHkv, a.nk, D)) != cudaSuccess) return e;
-    if ((e = make_tmap_bf16(&mv, a.v, BHkv, a.nk, D)) != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(fwd_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM);
+    if ((e = make_tmap(&mk, a.k, esize, BHkv, a.nk, D)) != cudaSuccess) return e;
+    if ((e = make_tmap(&mv, a.v, esize, BHkv, a.nk, D)) != cudaSuccess) return e;
+    void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const FwdKParams);
+    if constexpr (F8) kern = fwd_fp8_kernel<D>;
+    else kern = fwd_bf16_kernel<D>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     FwdKParams kp;
     kp.o = a.o;
@@ -521,11 +578,12 @@ cudaError_t launch_fwd_bf16_d(const FwdArgs& a, cudaStream_t stream) {
         long long g = (32LL << 20) / (per_head > 0 ? per_head : 1);
         kp.group = static_cast<int>(g < 1 ? 1 : (g > BH ? BH : g));
     }
-    kp.scale_log2 = a.scale * kLog2e;
+    kp.scale_log2 = a.scale * kLog2e * (F8 ? a.q_descale * a.k_descale : 1.f);
+    kp.o_scale = F8 ? a.v_descale : 1.f;
     kp.timeout_ns = a.timeout_ns;
     const long long grid = static_cast<long long>(kp.n_pairs) * BH;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    fwd_bf16_kernel<D><<<static_cast<unsigned>(grid), kFwdThreads, C::SMEM, stream>>>(mq, mk, mv, kp);
+    kern<<<static_cast<unsigned>(grid), kFwdThreads, C::SMEM, stream>>>(mq, mk, mv, kp);
     return cudaGetLastError();
 }
 
@@ -533,9 +591,17 @@ cudaError_t launch_fwd_bf16_d(const FwdArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_fwd_bf16(const FwdArgs& a, cudaStream_t stream) {
     switch (a.d) {
-        case 32: return launch_fwd_bf16_d<32>(a, stream);
-        case 64: return launch_fwd_bf16_d<64>(a, stream);
-        case 128: return launch_fwd_bf16_d<128>(a, stream);
+        case 32: return launch_fwd_d<32, false>(a, stream);
+        case 64: return launch_fwd_d<64, false>(a, stream);
+        case 128: return launch_fwd_d<128, false>(a, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_fwd_fp8(const FwdArgs& a, cudaStream_t stream) {
+    switch (a.d) {
+        case 64: return launch_fwd_d<64, true>(a, stream);
+        case 128: return launch_fwd_d<128, true>(a, stream);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -74,6 +74,7 @@ struct FwdArgs {
     int Hkv;          // K/V heads; query head h reads K/V head h / (H / Hkv)
     float scale;
     int wl, wr;       // visible window (see MaskSpec)
+    float q_descale, k_descale, v_descale;   // E4M3 inputs only: real value = stored · descale
     uint64_t timeout_ns;
 };
 
@@ -102,13 +103,19 @@ struct BwdArgs {
     const cudaEvent_t* phase_events;   // 4 events or nullptr (measurement hook)
 };
 
-// Encodes a 3-D bf16 tensor map over a (B*H, n, d) tensor with a box of (chunk, box_rows, 1) and
-// the swizzle that matches `chunk` (64 elements: 128-byte, 32 elements: 64-byte).
-cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int BH, int n, int d,
-                           int box_rows = 128);
+// Encodes a 3-D tensor map over a (B*H, n, d) tensor of `esize`-byte elements (2: bf16, 1: 8-bit)
+// with a box of (chunk, box_rows, 1), chunk = min(d, 128 / esize) elements, and the swizzle that
+// matches the chunk's bytes (128: 128-byte, 64: 64-byte).
+cudaError_t make_tmap(CUtensorMap* map, const void* base, int esize, int BH, int n, int d,
+                      int box_rows = 128);
+inline cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int BH, int n, int d,
+                                  int box_rows = 128) {
+    return make_tmap(map, base, 2, BH, n, d, box_rows);
+}
 
 cudaError_t launch_fwd_bf16(const FwdArgs& a, cudaStream_t stream);
 cudaError_t launch_fwd_f32(const FwdArgs& a, cudaStream_t stream);
+cudaError_t launch_fwd_fp8(const FwdArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_bf16(const BwdArgs& a, cudaStream_t stream);
 cudaError_t launch_wait_selftest(uint64_t timeout_ns, cudaStream_t stream);
 

@@ -77,6 +77,25 @@ int attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* ls
                  int B, int H, int Hkv, int n, int d, float scale, int causal, int dtype,
                  void* stream);
 
+/* FP8 forward pass ("Flash Attention Nedir?" and "Apa itu FlashAttention": FlashAttention-3 runs
+ * the method in FP8 on Hopper). q, k, v hold E4M3 bytes (OCP FP8 E4M3: 1 sign, 4 exponent bits
+ * with bias 7, 3 mantissa bits, no infinities, max 448) in the layouts of attn_fwd_ex; the real
+ * inputs are q·q_descale, k·k_descale and v·v_descale (one positive, finite factor per tensor).
+ * o receives bf16 (B, H, nq, d); lse (B, H, nq) fp32 is the natural-log row statistic of
+ * scale·Q·K^T over the visible keys, as for attn_fwd. Masks (window_left, window_right), query /
+ * key lengths and K/V head counts as attn_fwd_ex.
+ * Both products run on the tensor cores with E4M3 operands and fp32 accumulation; the softmax
+ * weights P are rounded to E4M3 before P·V (relative rounding error up to 2^-4 per weight), so the
+ * result is not within the bf16 path's tolerance: it differs from the exact attention of the
+ * dequantised inputs by at most 2^-4·max|V| per element from that rounding, plus bf16 output
+ * rounding.
+ * d must be 64 or 128 (else ATTN_ERR_UNSUPPORTED); other errors as attn_fwd_ex, and a descale that
+ * is not positive and finite is ATTN_ERR_INVALID. */
+int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int H, int Hkv, int nq, int nk, int d, float scale,
+                 int window_left, int window_right,
+                 float q_descale, float k_descale, float v_descale, void* stream);
+
 /* Bytes of device workspace attn_bwd needs for these sizes: the D vector and the LSE·log2(e)
  * vector (B·H·n fp32 each, padded per head to a multiple of 128 rows) and the fp32 dQ accumulator
  * (B·H·n·d fp32, padded the same way), each rounded up to 256 bytes; with deterministic != 0 also

@@ -12,7 +12,8 @@ FAKE = 1 << 20          # an aligned, never-dereferenced pointer value (validati
 def test_every_declared_function_is_exported():
     names = ea.declared_functions()
     assert {"attn_fwd", "attn_bwd", "attn_fwd_gqa", "attn_bwd_gqa", "attn_bwd_noalloc",
-            "attn_fwd_ex", "attn_bwd_ex",
+            "attn_fwd_ex", "attn_bwd_ex", "attn_fwd_fp8", "attn_ring_merge",
+            "attn_ring_accumulate",
             "attn_bwd_workspace_bytes", "attn_get_device_status",
             "attn_error_string", "attn_version", "attn_set_wait_timeout_us",
             "attn_selftest_wait_timeout"} <= set(names)
@@ -126,3 +127,20 @@ def test_ex_rejects_bad_lengths_and_heads():
     assert g(128, 64, dtype=ea.ATTN_FP32) == ea.ATTN_ERR_UNSUPPORTED
     # the workspace follows the query length
     assert g(300, 64) == ea.ATTN_ERR_WORKSPACE
+
+
+def test_fp8_and_ring_entry_points_validate_before_launch():
+    a = [ctypes.c_void_p(FAKE)] * 5
+    fp8 = lambda d=128, qs=1.0, nk=128: ea.attn_fwd_fp8(*a, 1, 2, 2, 128, nk, d, 0.1, -1, 0, qs,
+                                                        1.0, 1.0, None)
+    assert fp8(d=32) == ea.ATTN_ERR_UNSUPPORTED
+    assert fp8(qs=0.0) == ea.ATTN_ERR_INVALID
+    assert fp8(qs=float("nan")) == ea.ATTN_ERR_INVALID
+    assert fp8(nk=0) == ea.ATTN_ERR_INVALID
+    f = ctypes.c_void_p(FAKE)
+    assert ea.attn_ring_merge(f, f, f, f, 0, 64, ea.ATTN_BF16, 1, None, 0, None) == ea.ATTN_ERR_INVALID
+    assert ea.attn_ring_merge(f, f, f, f, 8, 48, ea.ATTN_BF16, 1, None, 0, None) == ea.ATTN_ERR_UNSUPPORTED
+    assert ea.attn_ring_merge(f, f, f, f, 8, 64, 9, 1, None, 0, None) == ea.ATTN_ERR_UNSUPPORTED
+    assert ea.attn_ring_accumulate(f, f, 12, ea.ATTN_BF16, 0, None, 0, None) == ea.ATTN_ERR_INVALID
+    assert ea.attn_ring_accumulate(ctypes.c_void_p(FAKE + 4), None, 16, 0, 0, None, 0, None) == \
+        ea.ATTN_ERR_INVALID
