@@ -239,6 +239,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-fp8", action="store_true",
+                    help="skip the extra timing of the FP8 (E4M3) forward pass")
     ap.add_argument("--workload", default=WORKLOAD,
                     help="named workload of attn_inputs.WORKLOADS (profiling runs use a smaller "
                          "one; the headline is the default)")
@@ -339,6 +341,39 @@ def main():
     bwd_tf = bwd_flops / (statistics.mean(bwd_ms) * 1e-3) / 1e12
     main_tf = bwd_flops / (statistics.mean(main_ms) * 1e-3) / 1e12
 
+    # --- extra: the FP8 (E4M3) forward pass on the same inputs, quantised with descale 2^-4
+    fp8 = None
+    if w.d in (64, 128) and not args.no_fp8:
+        desc = 2.0 ** -4
+        q8, k8, v8 = ((t.float() / desc).clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
+                      for t in (q, k, v))
+
+        def fwd8():
+            ea.forward_fp8(q8, k8, v8, desc, desc, desc, causal=True, scale=w.scale, out=o,
+                           lse=lse, stream=stream)
+
+        for _ in range(args.warmup):
+            fwd8()
+        torch.cuda.synchronize()
+        barrier()
+        a8 = torch.cuda.Event(enable_timing=True)
+        b8 = torch.cuda.Event(enable_timing=True)
+        a8.record(stream)
+        for _ in range(args.steps):
+            fwd8()
+        b8.record(stream)
+        torch.cuda.synchronize()
+        if ea.device_status() != ea.ATTN_OK:
+            raise SystemExit("device status not OK after the FP8 forward")
+        ms8 = max_over_ranks(a8.elapsed_time(b8) / args.steps, dist, dev)
+        tf8 = fwd_flops / (ms8 * 1e-3) / 1e12
+        fp8 = {"ms": ms8, "tflops": tf8, "peak": 2 * burst,
+               "peak_kind": "bf16_tflops x 2 (nominal fp8 / bf16 dense ratio)",
+               "pct_of_peak": 100 * tf8 / (2 * burst),
+               "inputs": "the workload's q, k, v quantised to E4M3 with descale 2^-4",
+               "steps": args.steps}
+        del q8, k8, v8
+
     # --- end to end through the public API with host buffers (pinned), copies inside the timing
     pin = [t.pin_memory() for t in (q_h, k_h, v_h, do_h)]
     outs_h = [torch.empty(w.shape, dtype=torch.bfloat16).pin_memory() for _ in range(4)]
@@ -397,6 +432,8 @@ def main():
         "gpu_launches": 4 * args.steps,
         "clocks": clk,
     }
+    if fp8 is not None:
+        line["fp8_fwd"] = fp8
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, dt, rows_n, threads = oracle_sample(args.cpu_seconds, q_h, k_h, v_h, do_h, w)
         line["cpu_baseline"] = {

@@ -85,10 +85,11 @@ int attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* ls
  * scale·Q·K^T over the visible keys, as for attn_fwd. Masks (window_left, window_right), query /
  * key lengths and K/V head counts as attn_fwd_ex.
  * Both products run on the tensor cores with E4M3 operands and fp32 accumulation; the softmax
- * weights P are rounded to E4M3 before P·V (relative rounding error up to 2^-4 per weight), so the
- * result is not within the bf16 path's tolerance: it differs from the exact attention of the
- * dequantised inputs by at most 2^-4·max|V| per element from that rounding, plus bf16 output
- * rounding.
+ * weights P are rounded to E4M3 before P·V (relative error up to 2^-4 for weights >= 2^-6,
+ * absolute error up to 2^-10 below), so the result is not within the bf16 path's tolerance: an
+ * element differs from the exact attention of the dequantised inputs by up to 2^-4·max|V| from the
+ * normal-range weights, plus 2^-10·max|V|/l per subnormal weight (l >= 1 is the row's sum of
+ * weights), plus bf16 output rounding.
  * d must be 64 or 128 (else ATTN_ERR_UNSUPPORTED); other errors as attn_fwd_ex, and a descale that
  * is not positive and finite is ATTN_ERR_INVALID. */
 int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
