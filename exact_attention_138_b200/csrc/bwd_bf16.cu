@@ -639,9 +639,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 //   warp 9          MMA issuer, per tile:  dP^T(i) -> [P^T(i)] dV += P^T dO -> S^T(i+1) ->
 //                   [dS^T(i)] dK += dS^T Q -> dQ^T(i) = K^T dS^T (into buffer i mod 2).
 //   warps 12-15     dQ drain warpgroup: copies dQ^T(i) out of TMEM (one head-dim row per thread)
-//                   into a shared-memory staging tile laid out like the accumulator rows (64 x 128
-//                   fp32, 32 KB contiguous in global memory); one elected lane then adds it with
-//                   a single bulk reduction. This work never sits on the compute warps' path.
+//                   into shared-memory staging laid out like the accumulator rows, one half tile
+//                   (32 queries x 128 fp32, 16 KB contiguous in global memory) per slot of a
+//                   3-slot ring, and one elected lane adds each half with a bulk reduction. The
+//                   reductions are limited by L2's read-modify-write rate, so two of them stay in
+//                   flight while the next half is staged. This work never sits on the compute
+//                   warps' path.
 // ------------------------------------------------------------------------------------------
 // Single-lane issue helpers for a converged warp (see elect_one).
 #define MMA_SS(...) do { if (elect_one()) mma_ss(__VA_ARGS__); } while (0)
@@ -657,12 +660,15 @@ constexpr int QTILE = 64 * 128 * 2;        // Q_i or dO_i: 2 chunks [64 rows][64
 constexpr int QCHUNK = 64 * 128;           // bytes of one [64 rows][64 d] chunk
 constexpr int STAGES = 3;
 constexpr int DS_BYTES = 128 * 64 * 2;     // dS^T [128 keys][64 queries], one SW128 chunk
-constexpr int STG_BYTES = 64 * 128 * 4;    // dQ staging [64 queries][128 d] fp32
+constexpr int STG_SLOT = 32 * 128 * 4;     // dQ staging slot: [32 queries][128 d] fp32
+constexpr int STG_SLOTS = 3;
+constexpr int STG_BYTES = STG_SLOTS * STG_SLOT;
 constexpr int OFF_K = 0, OFF_V = KTILE, OFF_Q = 2 * KTILE, OFF_DO = OFF_Q + STAGES * QTILE;
 constexpr int OFF_DS = OFF_DO + STAGES * QTILE, OFF_STG = OFF_DS + DS_BYTES;
 constexpr int OFF_L2 = OFF_STG + STG_BYTES, OFF_DV = OFF_L2 + STAGES * 256;
 constexpr int OFF_BARS = OFF_DV + STAGES * 256;
 constexpr int SMEM = OFF_BARS + 256;
+static_assert(SMEM <= 232448, "dynamic shared memory per block");
 
 struct Bars {
     uint64_t kv_full;
@@ -882,7 +888,9 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
             sync_phase[s] ^= 1;
             return okw;
         };
-        for (int it = 0; it < NTT; ++it) {
+        int half = 0;                                      // half tiles staged so far
+        bool run = true;
+        for (int it = 0; run && it < NTT; ++it) {
             const int b2 = it & 1;
             if (!bounded_wait_warp(&bars->dq_full[b2], (it >> 1) & 1, abort, lim)) break;
             tc_fence_after();
@@ -893,44 +901,46 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
             reg_fence<64>(u);
             tc_fence_before();
             mbar_arrive(&bars->dq_drained[b2]);
-            // the previous tile's bulk reduction must have read the staging tile
-            if (leader && lane == 0) bulk_wait_read_all();
-            if (!wg_sync(0)) break;
+            const int i = i_begin + it % NT;
+            const int qbh = kvbh * p.kv_group + it / NT;
+            float* dst = p.dq_acc + (static_cast<size_t>(qbh) * p.n_pad + i * BQ) * D;
+            volatile int* sem = p.deterministic ? p.sems + static_cast<size_t>(qbh) * qt64 + i : nullptr;
+            bool got = true;
+            if (sem && leader && lane == 0) {
+                // contributions to one query tile are added in increasing key-tile order,
+                // starting from the first key tile that this query tile meets
+                const int need = j - first_key_tile(mk, static_cast<long long>(i) * BQ, 128);
+                const uint64_t t0 = globaltimer_ns();
+                while (*sem < need) {
+                    if (*abort || globaltimer_ns() - t0 > lim) {
+                        *abort = 1;
+                        report_error(4);
+                        got = false;
+                        break;
+                    }
+                    __nanosleep(64);
+                }
+                __threadfence();
+            }
 #pragma unroll
-            for (int x = 0; x < 64; ++x) sStg[x * D + r] = __uint_as_float(u[x]);
-            fence_proxy_async_smem();
-            if (!wg_sync(1)) break;
-            if (leader && lane == 0) {
-                const int i = i_begin + it % NT;
-                const int qbh = kvbh * p.kv_group + it / NT;
-                float* dst = p.dq_acc + (static_cast<size_t>(qbh) * p.n_pad + i * BQ) * D;
-                volatile int* sem = p.deterministic ? p.sems + static_cast<size_t>(qbh) * qt64 + i : nullptr;
-                bool got = true;
-                if (sem) {
-                    // contributions to one query tile are added in increasing key-tile order,
-                    // starting from the first key tile that this query tile meets
-                    const int need = j - first_key_tile(mk, static_cast<long long>(i) * BQ, 128);
-                    const uint64_t t0 = globaltimer_ns();
-                    while (*sem < need) {
-                        if (*abort || globaltimer_ns() - t0 > lim) {
-                            *abort = 1;
-                            report_error(4);
-                            got = false;
-                            break;
-                        }
-                        __nanosleep(64);
-                    }
-                    __threadfence();
-                }
-                if (got) {
-                    bulk_reduce_add_f32(dst, sStg, STG_BYTES);
+            for (int h = 0; h < 2; ++h, ++half) {
+                float* slot = sStg + (half % STG_SLOTS) * (STG_SLOT / 4);
+                // the reduction issued from this slot STG_SLOTS halves ago has read it
+                if (leader && lane == 0) bulk_wait_read_le2();
+                if (!wg_sync(0)) { run = false; break; }
+#pragma unroll
+                for (int x = 0; x < 32; ++x) slot[x * D + r] = __uint_as_float(u[h * 32 + x]);
+                fence_proxy_async_smem();
+                if (!wg_sync(1)) { run = false; break; }
+                if (leader && lane == 0 && got) {
+                    bulk_reduce_add_f32(dst + h * 32 * D, slot, STG_SLOT);
                     bulk_commit();
-                    if (sem) {
-                        bulk_wait_all();             // the adds are done, not only the reads
-                        __threadfence();
-                        atomicAdd(const_cast<int*>(sem), 1);
-                    }
                 }
+            }
+            if (sem && leader && lane == 0 && got && run) {
+                bulk_wait_all();             // the adds are done, not only the reads
+                __threadfence();
+                atomicAdd(const_cast<int*>(sem), 1);
             }
             if (*abort) break;
         }
