@@ -1,18 +1,23 @@
-"""Ring attention: exact attention over a sequence split into chunks, one chunk per rank
+"""Ring attention: exact attention over a sequence split into chunks held by different ranks
 ("Attention Mechanism: Revolusi Representasi Sequence", §16 "Long Context Training", Ring
 Attention; §6, long-context techniques table).
 
-Rank p holds the queries, keys and values of chunk p (all chunks the same length). In hop r it
-attends its queries to K/V chunk (p - r) mod N, which arrived from rank p - 1, while sending the
-chunk it holds on to rank p + 1; the partial results are folded together with the log-sum-exp
-rule (attn_ring_merge). Under a causal mask a hop is either unmasked (an earlier chunk), causal
-(its own chunk) or skipped (a later chunk). The backward pass walks the same ring with the final
-O and LSE: dQ accumulates locally over the hops, and the dK / dV accumulators travel with their
-chunk and arrive back at its owner after the last hop.
+Layouts. With N ranks the sequence is cut into equal chunks:
+  contiguous  N chunks; rank p holds chunk p.
+  zigzag      2N chunks; rank p holds chunks p and 2N-1-p (its q, k, v are those two chunks one
+              after the other). Under a causal mask every rank then sees the same amount of work
+              (the contiguous layout gives rank N-1 N times the work of rank 0).
+In hop r a rank attends its query chunks to the K/V chunks of rank (p - r) mod N, which arrived
+from rank p - 1, while sending the chunks it holds on to rank p + 1; the partial results of each
+query chunk are folded together with the log-sum-exp rule (attn_ring_merge). Under a causal mask
+a (query chunk, key chunk) pair is unmasked (earlier key chunk), causal (same chunk) or skipped
+(later key chunk). The backward pass walks the same ring with the final O and LSE: dQ accumulates
+locally, and the dK / dV accumulators travel with their chunks and arrive back at their owner
+after the last hop.
 
-Every arithmetic step runs in the library's CUDA kernels (attn_fwd_ex / attn_bwd_ex per hop,
-attn_ring_merge / attn_ring_accumulate between hops); this module only schedules them and moves
-chunks with torch.distributed point-to-point operations (NCCL on GPUs), which run on NCCL's
+Every arithmetic step runs in the library's CUDA kernels (attn_fwd_ex / attn_bwd_ex per chunk
+pair, attn_ring_merge / attn_ring_accumulate between them); this module only schedules them and
+moves chunks with torch.distributed point-to-point operations (NCCL on GPUs), which run on NCCL's
 stream and overlap the current hop's kernels. `ring_forward_emulated` / `ring_backward_emulated`
 run the same schedule for N ranks inside one process (chunks are indexed instead of sent), which
 is how the kernels of the multi-rank path are checked on a single GPU.
@@ -35,13 +40,13 @@ def hop_window(q_chunk: int, kv_chunk: int, causal: bool):
     return None
 
 
-def _last_hop(rank: int, world: int, causal: bool) -> int:
-    # hop r visits chunk (rank - r) mod world; with a causal mask chunks after `rank` are skipped
-    return rank if causal else world - 1
+def rank_chunks(rank: int, world: int, zigzag: bool):
+    """Global indices of the chunks rank `rank` holds, in the order its tensors store them."""
+    return [rank, 2 * world - 1 - rank] if zigzag else [rank]
 
 
 class CudaOps:
-    """The per-hop operations, all in libattn.so."""
+    """The per-chunk-pair operations, all in libattn.so."""
 
     def __init__(self):
         import exact_attention_138_b200 as ea
@@ -65,37 +70,65 @@ def _scale(q, scale):
     return 1.0 / math.sqrt(q.shape[-1]) if scale is None else float(scale)
 
 
+def _split(x, parts):
+    """The chunks of a rank's (B, H, parts·c, d) tensor as contiguous tensors."""
+    if parts == 1:
+        return [x.contiguous()]
+    return [c.contiguous() for c in torch.chunk(x, parts, dim=2)]
+
+
+def _join(chunks):
+    return chunks[0] if len(chunks) == 1 else torch.cat(chunks, dim=2)
+
+
 class _FwdState:
     def __init__(self, q):
         self.o_acc = torch.empty(q.shape, dtype=torch.float32, device=q.device)
         self.lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
-        self.out = torch.empty_like(q)
         self.first = True
 
 
-def _fwd_hop(ops, st, q, k, v, rank, world, r, causal, scale):
-    w = hop_window(rank, (rank - r) % world, causal)
-    if w is None:
-        return
-    o_p, l_p = ops.fwd(q, k, v, scale, w)
-    last = r == _last_hop(rank, world, causal)
-    ops.merge(st.o_acc, st.lse, o_p, l_p, st.first, st.out if last else None)
-    st.first = False
+def _fwd_hop(ops, states, qs, q_ids, kvs, kv_ids, causal, scale):
+    """Fold every visible (query chunk, key chunk) pair of one hop into the running results."""
+    for qi, q in enumerate(qs):
+        for ki, (k, v) in enumerate(kvs):
+            w = hop_window(q_ids[qi], kv_ids[ki], causal)
+            if w is None:
+                continue
+            o_p, l_p = ops.fwd(q, k, v, scale, w)
+            st = states[qi]
+            ops.merge(st.o_acc, st.lse, o_p, l_p, st.first, None)
+            st.first = False
 
 
-class _BwdState:
-    def __init__(self, q):
-        self.dq_acc = torch.zeros(q.shape, dtype=torch.float32, device=q.device)
+def _fwd_outputs(ops, states, qs):
+    outs = []
+    for st, q in zip(states, qs):
+        out = torch.empty_like(q)
+        ops.accumulate(st.o_acc, None, False, out)    # fp32 running output -> q's dtype
+        outs.append(out)
+    return _join(outs), _join([st.lse for st in states])
 
 
-def _bwd_hop(ops, st, q, k, v, o, do, lse, dk_acc, dv_acc, rank, world, r, causal, scale, det):
-    w = hop_window(rank, (rank - r) % world, causal)
-    if w is None:
-        return
-    dq_p, dk_p, dv_p = ops.bwd(q, k, v, o, do, lse, scale, w, det)
-    ops.accumulate(st.dq_acc, dq_p, False, None)
-    ops.accumulate(dk_acc, dk_p, False, None)
-    ops.accumulate(dv_acc, dv_p, False, None)
+def _bwd_hop(ops, dq_acc, qs, q_ids, os_, dos, lses, kvs, kv_ids, dkv_acc, causal, scale, det):
+    for qi, q in enumerate(qs):
+        for ki, (k, v) in enumerate(kvs):
+            w = hop_window(q_ids[qi], kv_ids[ki], causal)
+            if w is None:
+                continue
+            dq_p, dk_p, dv_p = ops.bwd(q, k, v, os_[qi], dos[qi], lses[qi], scale, w, det)
+            ops.accumulate(dq_acc[qi], dq_p, False, None)
+            ops.accumulate(dkv_acc[ki][0], dk_p, False, None)
+            ops.accumulate(dkv_acc[ki][1], dv_p, False, None)
+
+
+def _convert(ops, accs, likes):
+    outs = []
+    for acc, like in zip(accs, likes):
+        out = torch.empty_like(like)
+        ops.accumulate(acc, None, False, out)
+        outs.append(out)
+    return _join(outs)
 
 
 def _peers(group):
@@ -114,92 +147,113 @@ def _exchange(tensors, nxt, prv, group):
     return recv, dist.batch_isend_irecv(ops)
 
 
-def ring_forward(q, k, v, causal=False, scale=None, group=None, ops=None):
-    """O, LSE of attention over the whole sequence for this rank's query chunk. q: (B,H,n,d),
-    k, v: (B,Hkv,n,d) chunks of the same length on every rank (chunk index = rank)."""
+def ring_forward(q, k, v, causal=False, scale=None, group=None, ops=None, zigzag=False):
+    """O, LSE of attention over the whole sequence for this rank's query chunks. q: (B,H,n,d),
+    k, v: (B,Hkv,n,d) holding this rank's chunk(s) of the layout (n = one chunk, or two chunks
+    for zigzag); every rank's chunks have the same length."""
     ops = ops or CudaOps()
     scale = _scale(q, scale)
     rank, world, nxt, prv = _peers(group)
-    st = _FwdState(q)
-    cur = [k.contiguous(), v.contiguous()]
+    parts = 2 if zigzag else 1
+    q_ids = rank_chunks(rank, world, zigzag)
+    qs = _split(q, parts)
+    states = [_FwdState(c) for c in qs]
+    cur = _split(k, parts) + _split(v, parts)          # k chunks, then v chunks
     for r in range(world):
         reqs = None
         if r < world - 1:
             nxt_kv, reqs = _exchange(cur, nxt, prv, group)
-        _fwd_hop(ops, st, q, cur[0], cur[1], rank, world, r, causal, scale)
+        kv_ids = rank_chunks((rank - r) % world, world, zigzag)
+        kvs = list(zip(cur[:parts], cur[parts:]))
+        _fwd_hop(ops, states, qs, q_ids, kvs, kv_ids, causal, scale)
         if reqs is not None:
             for req in reqs:
                 req.wait()
             cur = nxt_kv
-    return st.out, st.lse
+    return _fwd_outputs(ops, states, qs)
 
 
 def ring_backward(q, k, v, o, do, lse, causal=False, scale=None, group=None, ops=None,
-                  deterministic=False):
-    """dQ, dK, dV of ring attention for this rank's chunk, given the final O and LSE of
-    `ring_forward` and dO."""
+                  deterministic=False, zigzag=False):
+    """dQ, dK, dV of ring attention for this rank's chunks, given the final O and LSE of
+    `ring_forward` (same layout) and dO."""
     ops = ops or CudaOps()
     scale = _scale(q, scale)
     rank, world, nxt, prv = _peers(group)
-    st = _BwdState(q)
-    cur = [k.contiguous(), v.contiguous()]
-    acc = [torch.zeros(k.shape, dtype=torch.float32, device=k.device),
-           torch.zeros(v.shape, dtype=torch.float32, device=v.device)]
+    parts = 2 if zigzag else 1
+    q_ids = rank_chunks(rank, world, zigzag)
+    qs, os_, dos = _split(q, parts), _split(o, parts), _split(do, parts)
+    lses = [c.contiguous() for c in torch.chunk(lse, parts, dim=2)]
+    dq_acc = [torch.zeros(c.shape, dtype=torch.float32, device=c.device) for c in qs]
+    ks, vs = _split(k, parts), _split(v, parts)
+    cur = ks + vs
+    acc = [torch.zeros(c.shape, dtype=torch.float32, device=c.device) for c in ks + vs]
     for r in range(world):
         reqs = None
         if r < world - 1:
             nxt_kv, reqs = _exchange(cur, nxt, prv, group)
-        _bwd_hop(ops, st, q, cur[0], cur[1], o, do, lse, acc[0], acc[1], rank, world, r, causal,
-                 scale, deterministic)
-        # the dK / dV accumulators travel on with their chunk; after the last hop each rank holds
-        # its own chunk's
+        kv_ids = rank_chunks((rank - r) % world, world, zigzag)
+        kvs = list(zip(cur[:parts], cur[parts:]))
+        dkv = list(zip(acc[:parts], acc[parts:]))
+        _bwd_hop(ops, dq_acc, qs, q_ids, os_, dos, lses, kvs, kv_ids, dkv, causal, scale,
+                 deterministic)
+        # the dK / dV accumulators travel on with their chunks; after the last hop each rank
+        # holds its own chunks'
         nxt_acc, acc_reqs = _exchange(acc, nxt, prv, group)
         for req in (reqs or []) + acc_reqs:
             req.wait()
         if reqs is not None:
             cur = nxt_kv
         acc = nxt_acc
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ops.accumulate(st.dq_acc, None, False, dq)
-    ops.accumulate(acc[0], None, False, dk)
-    ops.accumulate(acc[1], None, False, dv)
-    return dq, dk, dv
+    return (_convert(ops, dq_acc, qs), _convert(ops, acc[:parts], ks),
+            _convert(ops, acc[parts:], vs))
 
 
-def ring_forward_emulated(qs, ks, vs, causal=False, scale=None, ops=None):
-    """The ring_forward schedule for len(qs) ranks in one process (chunk lists, one per rank)."""
+def ring_forward_emulated(qs, ks, vs, causal=False, scale=None, ops=None, zigzag=False):
+    """The ring_forward schedule for len(qs) ranks in one process: qs[p], ks[p], vs[p] are rank
+    p's tensors in the chosen layout."""
     ops = ops or CudaOps()
     world = len(qs)
     scale = _scale(qs[0], scale)
-    states = [_FwdState(q) for q in qs]
+    parts = 2 if zigzag else 1
+    q_chunks = [_split(q, parts) for q in qs]
+    kv_chunks = [list(zip(_split(k, parts), _split(v, parts))) for k, v in zip(ks, vs)]
+    states = [[_FwdState(c) for c in qc] for qc in q_chunks]
     for r in range(world):
         for p in range(world):
-            s = (p - r) % world      # the chunk rank p holds in hop r
-            _fwd_hop(ops, states[p], qs[p], ks[s], vs[s], p, world, r, causal, scale)
-    return [s.out for s in states], [s.lse for s in states]
+            s = (p - r) % world      # the rank whose chunks rank p holds in hop r
+            _fwd_hop(ops, states[p], q_chunks[p], rank_chunks(p, world, zigzag), kv_chunks[s],
+                     rank_chunks(s, world, zigzag), causal, scale)
+    outs = [_fwd_outputs(ops, states[p], q_chunks[p]) for p in range(world)]
+    return [o for o, _ in outs], [l for _, l in outs]
 
 
 def ring_backward_emulated(qs, ks, vs, os_, dos, lses, causal=False, scale=None, ops=None,
-                           deterministic=False):
+                           deterministic=False, zigzag=False):
     """The ring_backward schedule for len(qs) ranks in one process."""
     ops = ops or CudaOps()
     world = len(qs)
     scale = _scale(qs[0], scale)
-    states = [_BwdState(q) for q in qs]
-    dk_acc = [torch.zeros(k.shape, dtype=torch.float32, device=k.device) for k in ks]
-    dv_acc = [torch.zeros(v.shape, dtype=torch.float32, device=v.device) for v in vs]
+    parts = 2 if zigzag else 1
+    q_chunks = [_split(q, parts) for q in qs]
+    o_chunks = [_split(o, parts) for o in os_]
+    do_chunks = [_split(x, parts) for x in dos]
+    l_chunks = [[c.contiguous() for c in torch.chunk(x, parts, dim=2)] for x in lses]
+    kv_chunks = [list(zip(_split(k, parts), _split(v, parts))) for k, v in zip(ks, vs)]
+    dq_acc = [[torch.zeros(c.shape, dtype=torch.float32, device=c.device) for c in qc]
+              for qc in q_chunks]
+    dkv_acc = [[(torch.zeros(k.shape, dtype=torch.float32, device=k.device),
+                 torch.zeros(v.shape, dtype=torch.float32, device=v.device)) for k, v in kvc]
+               for kvc in kv_chunks]
     for r in range(world):
         for p in range(world):
             s = (p - r) % world
-            _bwd_hop(ops, states[p], qs[p], ks[s], vs[s], os_[p], dos[p], lses[p], dk_acc[s],
-                     dv_acc[s], p, world, r, causal, scale, deterministic)
+            _bwd_hop(ops, dq_acc[p], q_chunks[p], rank_chunks(p, world, zigzag), o_chunks[p],
+                     do_chunks[p], l_chunks[p], kv_chunks[s], rank_chunks(s, world, zigzag),
+                     dkv_acc[s], causal, scale, deterministic)
     dqs, dks, dvs = [], [], []
     for p in range(world):
-        dq, dk, dv = torch.empty_like(qs[p]), torch.empty_like(ks[p]), torch.empty_like(vs[p])
-        ops.accumulate(states[p].dq_acc, None, False, dq)
-        ops.accumulate(dk_acc[p], None, False, dk)
-        ops.accumulate(dv_acc[p], None, False, dv)
-        dqs.append(dq)
-        dks.append(dk)
-        dvs.append(dv)
+        dqs.append(_convert(ops, dq_acc[p], q_chunks[p]))
+        dks.append(_convert(ops, [a for a, _ in dkv_acc[p]], [k for k, _ in kv_chunks[p]]))
+        dvs.append(_convert(ops, [b for _, b in dkv_acc[p]], [v for _, v in kv_chunks[p]]))
     return dqs, dks, dvs

@@ -18,27 +18,43 @@ import exact_attention_138_b200 as ea  # noqa: E402
 from exact_attention_138_b200 import ring  # noqa: E402
 
 
-def _split(x, world):
-    return [c.contiguous() for c in torch.chunk(x, world, dim=2)]
+def _split(x, world, zigzag=False):
+    """Each rank's tensor: chunk p (contiguous) or chunks p and 2N-1-p (zigzag)."""
+    if not zigzag:
+        return [c.contiguous() for c in torch.chunk(x, world, dim=2)]
+    c = torch.chunk(x, 2 * world, dim=2)
+    return [torch.cat([c[p], c[2 * world - 1 - p]], dim=2).contiguous() for p in range(world)]
 
 
-@pytest.mark.parametrize("world,causal,H,Hkv,n_chunk,d", [
-    (2, True, 2, 2, 384, 128), (4, True, 2, 2, 256, 128), (3, False, 2, 2, 300, 64),
-    (4, True, 4, 2, 200, 64), (2, False, 2, 1, 512, 32), (8, True, 1, 1, 128, 128)])
-def test_emulated_ring_equals_full_attention(cuda_device, world, causal, H, Hkv, n_chunk, d):
+def _unsplit(parts, world, zigzag=False):
+    if not zigzag:
+        return torch.cat(parts, 2)
+    halves = [torch.chunk(t, 2, dim=2) for t in parts]
+    return torch.cat([halves[p][0] for p in range(world)] +
+                     [halves[p][1] for p in reversed(range(world))], 2)
+
+
+@pytest.mark.parametrize("world,causal,H,Hkv,n_chunk,d,zigzag", [
+    (2, True, 2, 2, 384, 128, False), (4, True, 2, 2, 256, 128, False),
+    (3, False, 2, 2, 300, 64, False), (4, True, 4, 2, 200, 64, False),
+    (2, False, 2, 1, 512, 32, False), (8, True, 1, 1, 128, 128, False),
+    (2, True, 2, 2, 384, 128, True), (4, True, 4, 2, 256, 64, True),
+    (3, False, 2, 2, 300, 128, True), (8, True, 1, 1, 128, 128, True)])
+def test_emulated_ring_equals_full_attention(cuda_device, world, causal, H, Hkv, n_chunk, d,
+                                             zigzag):
     n = world * n_chunk
     q, do = attn_inputs.random_draws((1, H, n, d), seed=world * 10 + d, count=2)
     k, v = attn_inputs.random_draws((1, Hkv, n, d), seed=world * 10 + d + 1, count=2)
     scale = 1.0 / math.sqrt(d)
     dev = torch.device("cuda:0")
-    qs, ks, vs, dos = (_split(x.to(dev), world) for x in (q, k, v, do))
-    os_, lses = ring.ring_forward_emulated(qs, ks, vs, causal=causal, scale=scale)
+    qs, ks, vs, dos = (_split(x.to(dev), world, zigzag) for x in (q, k, v, do))
+    os_, lses = ring.ring_forward_emulated(qs, ks, vs, causal=causal, scale=scale, zigzag=zigzag)
     dqs, dks, dvs = ring.ring_backward_emulated(qs, ks, vs, os_, dos, lses, causal=causal,
-                                                scale=scale)
+                                                scale=scale, zigzag=zigzag)
     torch.cuda.synchronize()
     assert ea.device_status() == ea.ATTN_OK
-    o, lse = torch.cat(os_, 2), torch.cat(lses, 2)
-    dq, dk, dv = torch.cat(dqs, 2), torch.cat(dks, 2), torch.cat(dvs, 2)
+    o, lse = _unsplit(os_, world, zigzag), _unsplit(lses, world, zigzag)
+    dq, dk, dv = (_unsplit(x, world, zigzag) for x in (dqs, dks, dvs))
     wr = 0 if causal else -1
     ro, rlse = oracle.fwd_ex(q, k, v, scale, -1, wr)
     rq, rk, rv = oracle.bwd_ex(q, k, v, do, scale, -1, wr)

@@ -33,7 +33,18 @@ def _inputs(world, n_chunk, H, Hkv, d):
     return q, k, v, do
 
 
-def _worker(rank, world, port, causal, n_chunk, H, Hkv, d, out):
+def _layout(world, n_chunk, zigzag):
+    """Global row indices of each rank's tensors (contiguous: one chunk; zigzag: chunks p and
+    2N-1-p)."""
+    if not zigzag:
+        return [np.arange(p * n_chunk, (p + 1) * n_chunk) for p in range(world)]
+    c = n_chunk // 2
+    return [np.concatenate([np.arange(p * c, (p + 1) * c),
+                            np.arange((2 * world - 1 - p) * c, (2 * world - p) * c)])
+            for p in range(world)]
+
+
+def _worker(rank, world, port, causal, n_chunk, H, Hkv, d, zigzag, out):
     sys.path.insert(0, ROOT)
     sys.path.insert(0, os.path.join(ROOT, "tests"))
     from exact_attention_138_b200 import ring
@@ -43,32 +54,38 @@ def _worker(rank, world, port, causal, n_chunk, H, Hkv, d, out):
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         q, k, v, do = _inputs(world, n_chunk, H, Hkv, d)
-        sl = slice(rank * n_chunk, (rank + 1) * n_chunk)
-        mine = [x[:, :, sl].contiguous() for x in (q, k, v, do)]
+        rows = torch.from_numpy(_layout(world, n_chunk, zigzag)[rank])
+        mine = [x.index_select(2, rows).contiguous() for x in (q, k, v, do)]
         scale = 1.0 / math.sqrt(d)
         ops = CpuOps()
-        o, lse = ring.ring_forward(mine[0], mine[1], mine[2], causal=causal, scale=scale, ops=ops)
+        o, lse = ring.ring_forward(mine[0], mine[1], mine[2], causal=causal, scale=scale, ops=ops,
+                                   zigzag=zigzag)
         dq, dk, dv = ring.ring_backward(mine[0], mine[1], mine[2], o, mine[3], lse, causal=causal,
-                                        scale=scale, ops=ops)
+                                        scale=scale, ops=ops, zigzag=zigzag)
         out[rank] = tuple(x.numpy() for x in (o, lse, dq, dk, dv))
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,causal,H,Hkv", [(2, True, 2, 2), (2, False, 2, 1), (3, True, 4, 2)])
-def test_ring_schedule_on_cpu_ranks_equals_full_attention(world, causal, H, Hkv):
+@pytest.mark.parametrize("world,causal,H,Hkv,zigzag", [
+    (2, True, 2, 2, False), (2, False, 2, 1, False), (3, True, 4, 2, False),
+    (2, True, 2, 2, True), (3, True, 2, 1, True), (3, False, 2, 2, True)])
+def test_ring_schedule_on_cpu_ranks_equals_full_attention(world, causal, H, Hkv, zigzag):
     import oracle
     n_chunk, d = 24, 8
     mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
-    mp.start_processes(_worker, args=(world, _free_port(), causal, n_chunk, H, Hkv, d, out),
+    mp.start_processes(_worker, args=(world, _free_port(), causal, n_chunk, H, Hkv, d, zigzag,
+                                      out),
                        nprocs=world, join=True, start_method="spawn")
     q, k, v, do = _inputs(world, n_chunk, H, Hkv, d)
     scale = 1.0 / math.sqrt(d)
     qf, kf, vf, dof = (x.float().numpy() for x in (q, k, v, do))
     ro, rlse = oracle.fwd_ex(qf, kf, vf, scale, -1, 0 if causal else -1)
     rq, rk, rv = oracle.bwd_ex(qf, kf, vf, dof, scale, -1, 0 if causal else -1)
-    got = [np.concatenate([out[r][i] for r in range(world)], axis=2) for i in range(5)]
+    order = np.argsort(np.concatenate(_layout(world, n_chunk, zigzag)))
+    got = [np.concatenate([out[r][i] for r in range(world)], axis=2)[:, :, order]
+           for i in range(5)]
     np.testing.assert_allclose(got[0], ro, rtol=0, atol=1e-5)
     np.testing.assert_allclose(got[1], rlse, rtol=0, atol=1e-5)
     for g, want in zip(got[2:], (rq, rk, rv)):
@@ -81,3 +98,20 @@ def test_hop_windows():
     assert ring.hop_window(2, 2, True) == (-1, 0)
     assert ring.hop_window(1, 2, True) is None
     assert all(ring.hop_window(p, s, False) == (-1, -1) for p in range(3) for s in range(3))
+
+
+def test_zigzag_layout_balances_causal_work():
+    from exact_attention_138_b200 import ring
+    world = 4
+    for zigzag, balanced in ((False, False), (True, True)):
+        work = []
+        for p in range(world):
+            mine = ring.rank_chunks(p, world, zigzag)
+            pairs = 0.0
+            for r in range(world):
+                for a in mine:
+                    for b in ring.rank_chunks((p - r) % world, world, zigzag):
+                        w = ring.hop_window(a, b, True)
+                        pairs += 0 if w is None else (0.5 if w == (-1, 0) else 1.0)
+            work.append(pairs)
+        assert (len(set(work)) == 1) == balanced, work
