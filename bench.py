@@ -229,6 +229,82 @@ def run_reference(args, w):
     return 0
 
 
+def visible_pairs(nq, nk, wl, wr):
+    """Number of (query, key) pairs a mask leaves visible (query i aligned with key i + nk - nq;
+    key j visible iff i + off - wl <= j <= i + off + wr, negative = unbounded)."""
+    total, off = 0, nk - nq
+    for i in range(nq):
+        lo = 0 if wl < 0 else max(0, i + off - wl)
+        hi = nk - 1 if wr < 0 else min(nk - 1, i + off + wr)
+        total += max(0, hi - lo + 1)
+    return total
+
+
+def time_variants(args, w, ea, q, k, v, do, ws, stream, causal_flops):
+    """fwd+bwd time of grouped-query, sliding-window and (emulated) ring attention on the bench
+    tensors. TFLOPS count only visible (query, key) pairs: 4·d FLOP per pair forward, 2.5 times
+    that backward."""
+    import torch
+    from exact_attention_138_b200 import ring
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.variant_steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        if ea.device_status() != ea.ATTN_OK:
+            raise SystemExit("device status not OK in the variant timings")
+        return a.elapsed_time(b) / args.variant_steps
+
+    per_pair = 3.5 * 4 * w.d          # forward 4·d FLOP per visible pair, backward 2.5x
+    out = {"steps": args.variant_steps, "flops": "3.5 x 4·d per visible (query, key) pair"}
+    B, H, n = w.B, w.H, w.n
+    # grouped-query: 8 K/V heads (the first 8 of each batch's K and V)
+    kv_heads = 8
+    kg, vg = (t[:, :kv_heads].contiguous() for t in (k, v))
+
+    def gqa():
+        o, lse = ea.forward(q, kg, vg, causal=True, scale=w.scale, stream=stream)
+        ea.backward(q, kg, vg, o, do, lse, causal=True, scale=w.scale, workspace=ws,
+                    stream=stream)
+    ms = timed(gqa)
+    out["gqa_kv8"] = {"ms": ms, "tflops": causal_flops / (ms * 1e-3) / 1e12,
+                      "config": f"H={H}, Hkv={kv_heads}, causal"}
+    # sliding window: causal, 1024 keys to the left
+    win = (1024, 0)
+    pairs = B * H * visible_pairs(n, n, *win)
+
+    def window():
+        o, lse = ea.forward(q, k, v, scale=w.scale, window=win, stream=stream)
+        ea.backward(q, k, v, o, do, lse, scale=w.scale, window=win, workspace=ws, stream=stream)
+    ms = timed(window)
+    out["window_1024"] = {"ms": ms, "tflops": pairs * per_pair / (ms * 1e-3) / 1e12,
+                          "config": "causal window of 1025 keys (left 1024, right 0)"}
+    # ring attention, 4 ranks emulated in one process (zigzag chunks): the whole job's kernels
+    ranks = 4
+    c = torch.chunk
+    chunks = [c(t, 2 * ranks, dim=2) for t in (q, k, v, do)]
+    per_rank = [[torch.cat([x[p], x[2 * ranks - 1 - p]], dim=2).contiguous() for p in range(ranks)]
+                for x in chunks]
+    rq, rk, rv, rdo = per_rank
+    os_, lses = ring.ring_forward_emulated(rq, rk, rv, causal=True, scale=w.scale, zigzag=True)
+
+    def ring_step():
+        o_, l_ = ring.ring_forward_emulated(rq, rk, rv, causal=True, scale=w.scale, zigzag=True)
+        ring.ring_backward_emulated(rq, rk, rv, o_, rdo, l_, causal=True, scale=w.scale,
+                                    zigzag=True)
+    ms = timed(ring_step)
+    out["ring_zigzag_4"] = {"ms": ms, "tflops": causal_flops / (ms * 1e-3) / 1e12,
+                            "config": "4 ranks emulated on one GPU (all ranks' hops in turn), "
+                                      "zigzag chunks of 1024 rows; same FLOPs as the bench step"}
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -241,6 +317,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp8", action="store_true",
                     help="skip the extra timing of the FP8 (E4M3) forward pass")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the extra timings of grouped-query, sliding-window and ring "
+                         "attention on the bench inputs")
+    ap.add_argument("--variant-steps", type=int, default=20)
     ap.add_argument("--workload", default=WORKLOAD,
                     help="named workload of attn_inputs.WORKLOADS (profiling runs use a smaller "
                          "one; the headline is the default)")
@@ -374,6 +454,11 @@ def main():
                "steps": args.steps}
         del q8, k8, v8
 
+    # --- extra: the next rows on the same inputs (fwd + bwd per step, short runs)
+    variants = None
+    if not args.no_variants and world == 1:
+        variants = time_variants(args, w, ea, q, k, v, do, ws, stream, fwd_flops + bwd_flops)
+
     # --- end to end through the public API with host buffers (pinned), copies inside the timing.
     # Three streams run as a pipeline: while step k computes, step k+1's inputs travel host ->
     # device and step k-1's results device -> host (two device buffer sets; every step copies
@@ -468,6 +553,8 @@ def main():
     }
     if fp8 is not None:
         line["fp8_fwd"] = fp8
+    if variants is not None:
+        line["variants"] = variants
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, dt, rows_n, threads = oracle_sample(args.cpu_seconds, q_h, k_h, v_h, do_h, w)
         line["cpu_baseline"] = {
