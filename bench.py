@@ -275,6 +275,13 @@ def time_variants(args, w, ea, q, k, v, do, ws, stream, causal_flops):
     ms = timed(gqa)
     out["gqa_kv8"] = {"ms": ms, "tflops": causal_flops / (ms * 1e-3) / 1e12,
                       "config": f"H={H}, Hkv={kv_heads}, causal"}
+    # no mask: every (query, key) pair (twice the causal FLOPs)
+    def full():
+        o, lse = ea.forward(q, k, v, causal=False, scale=w.scale, stream=stream)
+        ea.backward(q, k, v, o, do, lse, causal=False, scale=w.scale, workspace=ws, stream=stream)
+    ms = timed(full)
+    out["no_mask"] = {"ms": ms, "tflops": B * H * n * n * per_pair / (ms * 1e-3) / 1e12,
+                      "config": "unmasked (cross-attention shape with n_q = n_k)"}
     # sliding window: causal, 1024 keys to the left
     win = (1024, 0)
     pairs = B * H * visible_pairs(n, n, *win)
