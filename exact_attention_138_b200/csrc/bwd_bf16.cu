@@ -290,7 +290,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
     } else if (warp == 9) {
         // ---------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        // The whole warp runs this loop (warp-uniform state); one elected lane issues.
+        {
+            auto vss = [](uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+                if (elect_one()) mma_ss(d, a, b, id, acc);
+            };
+            auto vts = [](uint32_t d, uint32_t a, uint64_t b, uint32_t id, uint32_t acc) {
+                if (elect_one()) mma_ts(d, a, b, id, acc);
+            };
+            auto vcommit = [](uint64_t* bar) {
+                if (elect_one()) mma_commit(bar);
+            };
             constexpr uint32_t idSS = idesc_bf16_f32(128, 128, 0, 0);    // K-major x K-major
             constexpr uint32_t idKN = idesc_bf16_f32(128, D, 0, 1);      // A K-major, B MN-major
             constexpr uint32_t idDQ = C::DQT ? idesc_bf16_f32(128, 128, 1, 1)   // dQ^T
@@ -319,59 +329,59 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 const SDesc bq = stage(Q_k, it & 1);
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks)
-                    mma_ss(tmem + COL_S, sdesc_at(K_k, koff(ks)), sdesc_at(bq, koff(ks)), idSS,
+                    vss(tmem + COL_S, sdesc_at(K_k, koff(ks)), sdesc_at(bq, koff(ks)), idSS,
                            ks > 0 ? 1u : 0u);
             };
             auto issue_dp = [&](int it) {               // dP^T = V_j · dO_i^T
                 const SDesc bo = stage(dO_k, it & 1);
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks)
-                    mma_ss(tmem + COL_DP, sdesc_at(V_k, koff(ks)), sdesc_at(bo, koff(ks)), idSS,
+                    vss(tmem + COL_DP, sdesc_at(V_k, koff(ks)), sdesc_at(bo, koff(ks)), idSS,
                            ks > 0 ? 1u : 0u);
             };
-            bool ok = NTT > 0 && bounded_wait(&bars->kv_full, 0, abort, lim);
-            if (ok) ok = bounded_wait(&bars->q_full[0], 0, abort, lim);
+            bool ok = NTT > 0 && bounded_wait_warp(&bars->kv_full, 0, abort, lim);
+            if (ok) ok = bounded_wait_warp(&bars->q_full[0], 0, abort, lim);
             tc_fence_after();
             if (ok) {
                 issue_s(0);
-                mma_commit(&bars->s_full);
+                vcommit(&bars->s_full);
                 issue_dp(0);
-                mma_commit(&bars->dp_full);
+                vcommit(&bars->dp_full);
             }
             for (int it = 0; ok && it < NTT; ++it) {
                 const int st = it & 1;
                 if (it > 0) {
-                    if (!(ok = bounded_wait(&bars->dq_drained, (it - 1) & 1, abort, lim))) break;
+                    if (!(ok = bounded_wait_warp(&bars->dq_drained, (it - 1) & 1, abort, lim))) break;
                     tc_fence_after();
                     issue_dp(it);
-                    mma_commit(&bars->dp_full);
+                    vcommit(&bars->dp_full);
                 }
-                if (!(ok = bounded_wait(&bars->p_full, it & 1, abort, lim))) break;
+                if (!(ok = bounded_wait_warp(&bars->p_full, it & 1, abort, lim))) break;
                 tc_fence_after();
                 {   // dV_j += P^T · dO_i   (P^T in TMEM: queries 0-63 at S+0.., 64-127 at S+64..)
                     const SDesc bo = stage(dO_mn, st);
-                    mma_ts(tmem + COL_DV, tmem + COL_S, sdesc_at(bo, 0), idKN, it > 0 ? 1u : 0u);
+                    vts(tmem + COL_DV, tmem + COL_S, sdesc_at(bo, 0), idKN, it > 0 ? 1u : 0u);
 #pragma unroll
                     for (int ks = 1; ks < 8; ++ks)
-                        mma_ts(tmem + COL_DV, tmem + COL_S + (ks >> 2) * 64 + (ks & 3) * 8,
+                        vts(tmem + COL_DV, tmem + COL_S + (ks >> 2) * 64 + (ks & 3) * 8,
                                sdesc_at(bo, roff(ks)), idKN, 1u);
                 }
                 if (it + 1 < NTT) {
-                    if (!(ok = bounded_wait(&bars->q_full[(it + 1) & 1], ((it + 1) >> 1) & 1,
+                    if (!(ok = bounded_wait_warp(&bars->q_full[(it + 1) & 1], ((it + 1) >> 1) & 1,
                                             abort, lim)))
                         break;
                     tc_fence_after();
                     issue_s(it + 1);
-                    mma_commit(&bars->s_full);
+                    vcommit(&bars->s_full);
                 }
-                if (!(ok = bounded_wait(&bars->ds_full, it & 1, abort, lim))) break;
+                if (!(ok = bounded_wait_warp(&bars->ds_full, it & 1, abort, lim))) break;
                 tc_fence_after();
                 {   // dK_j += dS^T · Q_i   (A = dS^T K-major, B = Q_i MN-major)
                     const SDesc bq = stage(Q_mn, st);
-                    mma_ss(tmem + COL_DK, sdesc_at(dS_k, 0), sdesc_at(bq, 0), idKN, it > 0 ? 1u : 0u);
+                    vss(tmem + COL_DK, sdesc_at(dS_k, 0), sdesc_at(bq, 0), idKN, it > 0 ? 1u : 0u);
 #pragma unroll
                     for (int ks = 1; ks < 8; ++ks)
-                        mma_ss(tmem + COL_DK,
+                        vss(tmem + COL_DK,
                                sdesc_at(dS_k, static_cast<uint32_t>(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4)),
                                sdesc_at(bq, roff(ks)), idKN, 1u);
                 }
@@ -381,16 +391,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     const uint64_t kd = sdesc_at(K_mn, roff(ks));
                     const uint64_t sd = sdesc_at(dS_mn, static_cast<uint32_t>((ks * 2048) >> 4));
                     if (C::DQT)
-                        mma_ss(tmem + COL_DP, kd, sd, idDQ, ks > 0 ? 1u : 0u);
+                        vss(tmem + COL_DP, kd, sd, idDQ, ks > 0 ? 1u : 0u);
                     else
-                        mma_ss(tmem + COL_DP, sd, kd, idDQ, ks > 0 ? 1u : 0u);
+                        vss(tmem + COL_DP, sd, kd, idDQ, ks > 0 ? 1u : 0u);
                 }
-                mma_commit(&bars->dq_full);
-                mma_commit(&bars->ds_free);
-                mma_commit(&bars->q_empty[st]);
+                vcommit(&bars->dq_full);
+                vcommit(&bars->ds_free);
+                vcommit(&bars->q_empty[st]);
             }
-            if (ok) mma_commit(&bars->dkv_done);
-            mma_commit(&bars->teardown);
+            if (ok) vcommit(&bars->dkv_done);
+            vcommit(&bars->teardown);
             drain_wait_bwd(&bars->teardown, 0, 100000000ull);
         }
         __syncwarp();
