@@ -72,8 +72,12 @@ WsLayout ws_layout(int B, int H, int n, int d, int deterministic) {
     return w;
 }
 
+// Longest sequence accepted: tile and row arithmetic runs in 32-bit integers up to the length
+// rounded up to a multiple of 128 (plus one tile).
+constexpr int kMaxSeq = 0x7fffffff - 256;
+
 int validate_common(int B, int H, int n, int d, float scale, int dtype) {
-    if (B < 1 || H < 1 || n < 1) return ATTN_ERR_INVALID;
+    if (B < 1 || H < 1 || n < 1 || n > kMaxSeq) return ATTN_ERR_INVALID;
     if (!(scale > 0.f) || !isfinite(scale)) return ATTN_ERR_INVALID;
     if (static_cast<long long>(B) * H > 0x7fffffffLL) return ATTN_ERR_INVALID;
     if (dtype != ATTN_BF16 && dtype != ATTN_FP32) return ATTN_ERR_UNSUPPORTED;
@@ -142,7 +146,7 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
     if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID;
     int rc = validate_common(B, H, nq, d, scale, dtype);
     if (rc) return rc;
-    if (nk < 1) return ATTN_ERR_INVALID;
+    if (nk < 1 || nk > kMaxSeq) return ATTN_ERR_INVALID;
     if (Hkv < 1 || H % Hkv != 0) return ATTN_ERR_INVALID;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
         return ATTN_ERR_INVALID;
@@ -184,7 +188,7 @@ int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* ls
     int rc = validate_common(B, H, nq, d, scale, ATTN_BF16);
     if (rc) return rc;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-    if (nk < 1 || Hkv < 1 || H % Hkv != 0) return ATTN_ERR_INVALID;
+    if (nk < 1 || nk > kMaxSeq || Hkv < 1 || H % Hkv != 0) return ATTN_ERR_INVALID;
     const float ds[3] = {q_descale, k_descale, v_descale};
     for (float x : ds)
         if (!(x > 0.f) || !isfinite(x)) return ATTN_ERR_INVALID;
@@ -215,7 +219,7 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
     if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return ATTN_ERR_INVALID;
     int rc = validate_common(B, H, nq, d, scale, dtype);
     if (rc) return rc;
-    if (nk < 1) return ATTN_ERR_INVALID;
+    if (nk < 1 || nk > kMaxSeq) return ATTN_ERR_INVALID;
     if (Hkv < 1 || H % Hkv != 0) return ATTN_ERR_INVALID;
     if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
     const void* ptrs[] = {q, k, v, o, dO, lse, dq, dk, dv};

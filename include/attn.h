@@ -21,15 +21,17 @@
  *     element (b, h, i, c) at offset ((b*H + h)*n + i)*d + c. bf16 (ATTN_BF16) or fp32
  *     (ATTN_FP32) elements. Base addresses must be 16-byte aligned (TMA requirement).
  *   - lse: caller-owned DEVICE memory, fp32, (B, H, n), 16-byte aligned.
- *   - Self-attention only: the query and key lengths are both n; d is the head dimension of Q, K
- *     and V alike.
+ *   - attn_fwd / attn_bwd: query and key lengths are both n; d is the head dimension of Q, K
+ *     and V alike. Other lengths, masks and K/V head counts: the *_gqa and *_ex entry points.
  *   - scale: the factor applied to Q·K^T (normally 1/sqrt(d)); any finite positive value.
  *   - stream: a cudaStream_t (NULL = the legacy default stream). Every call is asynchronous on
- *     that stream; the library keeps no allocation between calls except cached tensor-map
- *     encoder entry points.
+ *     that stream and allocates nothing; the library's only device memory is the fixed scratch
+ *     array of attn_bwd_noalloc (see there). Calls are capturable into CUDA graphs (make one
+ *     call outside capture first, so that one-time driver lookups happen there).
  *
  * Errors: each call validates its arguments before launching anything and returns ATTN_OK or
- *   ATTN_ERR_INVALID   null pointer, B, H or n < 1, misaligned pointer, non-finite or <= 0 scale,
+ *   ATTN_ERR_INVALID   null pointer, B, H or n < 1, n > 2^31 - 257, misaligned pointer,
+ *                      non-finite or <= 0 scale,
  *                      workspace pointer null while ws_bytes > 0;
  *   ATTN_ERR_UNSUPPORTED  d not in {32, 64, 128}; fp32 backward; an unknown dtype;
  *   ATTN_ERR_WORKSPACE    ws_bytes smaller than attn_bwd_workspace_bytes();

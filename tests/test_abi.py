@@ -50,6 +50,7 @@ def _fwd(**kw):
     (dict(q=0), ea.ATTN_ERR_INVALID),
     (dict(lse=0), ea.ATTN_ERR_INVALID),
     (dict(n=0), ea.ATTN_ERR_INVALID),
+    (dict(n=2**31 - 200), ea.ATTN_ERR_INVALID),     # tile arithmetic would overflow
     (dict(B=0), ea.ATTN_ERR_INVALID),
     (dict(H=-1), ea.ATTN_ERR_INVALID),
     (dict(scale=0.0), ea.ATTN_ERR_INVALID),
@@ -116,6 +117,7 @@ def test_ex_rejects_bad_lengths_and_heads():
     f = lambda B, H, Hkv, nq, nk, d=64: ea.attn_fwd_ex(*a, B, H, Hkv, nq, nk, d, 0.125, 4, 4,
                                                        ea.ATTN_BF16, None)
     assert f(1, 2, 2, 128, 0) == ea.ATTN_ERR_INVALID
+    assert f(1, 2, 2, 128, 2**31 - 1) == ea.ATTN_ERR_INVALID
     assert f(1, 2, 2, 0, 128) == ea.ATTN_ERR_INVALID
     assert f(1, 6, 4, 128, 128) == ea.ATTN_ERR_INVALID
     assert f(1, 2, 2, 128, 64, d=80) == ea.ATTN_ERR_UNSUPPORTED
