@@ -13,12 +13,13 @@
 // Kernels:
 //   bwd_preprocess  D = rowsum(dO∘O) per query row; zeroes the fp32 dQ accumulator (and the
 //                   ordering semaphores of the deterministic mode).           HBM-bound
-//   bwd_main        one CTA per (key tile j, head): K_j and V_j stay in shared memory, Q_i and
-//                   dO_i stream through a 2-deep TMA ring. One thread issues the five tcgen05
-//                   MMAs per query tile; 4 compute warps (one thread per key row = TMEM lane) form
-//                   P^T and dS^T and add the dQ partial tile into the accumulator.
-//                   TMEM (512 columns): dV | dK | S^T (P^T as bf16) | dP^T, and the dQ tile reuses
-//                   the dP^T columns once dS^T is formed.
+//   bwd_main        (d = 32, 64) one CTA per (key tile j, K/V head): K_j and V_j stay in shared
+//                   memory, Q_i and dO_i stream through a 2-deep TMA ring. One warp issues the five
+//                   tcgen05 MMAs per query tile; 8 compute warps (one thread per key row = TMEM
+//                   lane, half the query columns each) form P^T and dS^T and add the dQ partial
+//                   tile into the accumulator. TMEM (512 columns): dV | dK | dQ x2 | S^T (P^T as
+//                   bf16) | dP^T, dQ double-buffered so the next tile's MMAs never wait for it.
+//   bwd_main_q64    (d = 128) see below.
 //   bwd_dq_convert  dQ = scale·acc -> bf16.                                    HBM-bound
 // Masks (causal, sliding window, query/key lengths that differ; see MaskSpec): key tile j only
 // meets the query tiles that hold a query which sees one of its keys; a key tile that no query
@@ -43,14 +44,14 @@ struct BwdCfg {
     static constexpr int TILE = NCH * CHUNK;              // 128 x D bf16
     static constexpr int DS_BYTES = 128 * 128 * 2;         // dS^T tile, 2 x [128 x 64] SW128
     static constexpr int STAT_BYTES = 2 * 2 * 128 * 4;     // [warpgroup][buffer][LSE2 | D] x 64
-    static constexpr bool DQT = (D == 128);                // dQ computed transposed (see kernel)
     static constexpr int SMEM = 6 * TILE + DS_BYTES + STAT_BYTES + 256;
 };
 
 struct BwdBars {
     uint64_t kv_full;
     uint64_t q_full[2], q_empty[2];
-    uint64_t s_full, dp_full, p_full, ds_full, dq_full, dq_drained, ds_free, dkv_done, teardown;
+    uint64_t s_full, dp_full, p_full, ds_full, ds_free, dkv_done, teardown;
+    uint64_t dq_full[2], dq_drained[2];   // dQ double-buffered in its own TMEM columns
     uint32_t tmem_base;
     int abort;
 };
@@ -180,15 +181,13 @@ __global__ void __launch_bounds__(256) bwd_dq_convert_kernel(const float* __rest
 // Roles (320 threads): warps 0-3 = compute warpgroup 0 (query columns 0-63 of each tile),
 // warps 4-7 = compute warpgroup 1 (query columns 64-127), warp 8 = TMA producer, warp 9 = MMA
 // issuer. Every compute thread owns one key row (= TMEM lane) and half of the tile's columns.
-// Per query tile i the MMA thread issues, in this order,
-//     dP^T(i) [after dQ(i-1) has been drained out of the dP columns],
+// Per query tile i the MMA warp issues, in this order,
 //     dV += P^T(i)·dO(i) [after P^T(i) is in TMEM],   S^T(i+1) = K·Q(i+1)^T,
-//     dK += dS^T(i)·Q(i) and dQ(i) [after dS^T(i) is in shared memory],
+//     dK += dS^T(i)·Q(i), dQ(i) = dS·K into buffer i mod 2 [after dS^T(i) is in shared memory
+//     and dQ(i-2) has been drained], then dP^T(i+1) = V·dO(i+1)^T,
 // while the compute warps run P(i) -> drain dQ(i-1) -> dS(i): the dQ drain of one tile and the
-// softmax of the next overlap the dK/dQ MMAs.
-// dQ: for d = 128 the MMA computes dQ^T = K^T·dS^T (TMEM lane = head-dim index, column = query),
-// so one warp-wide reduction covers 32 consecutive floats (128 B) of one dQ row; for d < 128 it
-// computes dQ = dS·K (lane = query) and each thread reduces 16-byte pieces of its row.
+// softmax of the next overlap the dK/dQ MMAs. dQ has TMEM lane = query, and each thread adds
+// 16-byte pieces of its row to the fp32 accumulator with red.global.
 // ------------------------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
@@ -205,7 +204,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     float* sStat = reinterpret_cast<float*>(sdS + C::DS_BYTES);   // [wg][buf][LSE2 64 | D 64]
     BwdBars* bars = reinterpret_cast<BwdBars*>(sdS + C::DS_BYTES + C::STAT_BYTES);
 
-    constexpr uint32_t COL_DV = 0, COL_DK = 128, COL_S = 256, COL_DP = 384;
+    // TMEM: dV [0,64) | dK [64,128) | dQ x2 [128,192),[192,256) | S^T [256,384) | dP^T [384,512)
+    static_assert(D <= 64, "d = 128 runs bwd_main_q64_kernel");
+    constexpr uint32_t COL_DV = 0, COL_DK = 64, COL_DQ = 128, COL_S = 256, COL_DP = 384;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -235,8 +236,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_init(&bars->dp_full, 1);
         mbar_init(&bars->p_full, 256);
         mbar_init(&bars->ds_full, 256);
-        mbar_init(&bars->dq_full, 1);
-        mbar_init(&bars->dq_drained, 256);
+        for (int b2 = 0; b2 < 2; ++b2) {
+            mbar_init(&bars->dq_full[b2], 1);
+            mbar_init(&bars->dq_drained[b2], 256);
+        }
         mbar_init(&bars->ds_free, 1);
         mbar_init(&bars->dkv_done, 1);
         mbar_init(&bars->teardown, 1);
@@ -303,8 +306,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             };
             constexpr uint32_t idSS = idesc_bf16_f32(128, 128, 0, 0);    // K-major x K-major
             constexpr uint32_t idKN = idesc_bf16_f32(128, D, 0, 1);      // A K-major, B MN-major
-            constexpr uint32_t idDQ = C::DQT ? idesc_bf16_f32(128, 128, 1, 1)   // dQ^T
-                                             : idesc_bf16_f32(128, D, 1, 1);    // dQ
+            constexpr uint32_t idDQ = idesc_bf16_f32(128, D, 1, 1);      // dQ = dS · K    // dQ
             const uint32_t aK = smem_addr(sK), aV = smem_addr(sV), aQ = smem_addr(sQ),
                            adO = smem_addr(sdO), adS = smem_addr(sdS);
             // Descriptor words of every operand view, built once (the issuing lane shares its SM
@@ -350,12 +352,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             for (int it = 0; ok && it < NTT; ++it) {
                 const int st = it & 1;
-                if (it > 0) {
-                    if (!(ok = bounded_wait_warp(&bars->dq_drained, (it - 1) & 1, abort, lim))) break;
-                    tc_fence_after();
-                    issue_dp(it);
-                    vcommit(&bars->dp_full);
-                }
                 if (!(ok = bounded_wait_warp(&bars->p_full, it & 1, abort, lim))) break;
                 tc_fence_after();
                 {   // dV_j += P^T · dO_i   (P^T in TMEM: queries 0-63 at S+0.., 64-127 at S+64..)
@@ -385,19 +381,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                sdesc_at(dS_k, static_cast<uint32_t>(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4)),
                                sdesc_at(bq, roff(ks)), idKN, 1u);
                 }
-                // dQ^T_i = K_j^T · dS^T  (d = 128)   or   dQ_i = dS · K_j   (d < 128)
+                // dQ_i = dS · K_j into buffer it mod 2, once the partial of tile it-2 is drained
+                const int b2 = it & 1;
+                if (it >= 2) {
+                    if (!(ok = bounded_wait_warp(&bars->dq_drained[b2], ((it - 2) >> 1) & 1, abort, lim))) break;
+                    tc_fence_after();
+                }
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint64_t kd = sdesc_at(K_mn, roff(ks));
                     const uint64_t sd = sdesc_at(dS_mn, static_cast<uint32_t>((ks * 2048) >> 4));
-                    if (C::DQT)
-                        vss(tmem + COL_DP, kd, sd, idDQ, ks > 0 ? 1u : 0u);
-                    else
-                        vss(tmem + COL_DP, sd, kd, idDQ, ks > 0 ? 1u : 0u);
+                    vss(tmem + COL_DQ + b2 * 64, sd, kd, idDQ, ks > 0 ? 1u : 0u);
                 }
-                vcommit(&bars->dq_full);
+                vcommit(&bars->dq_full[b2]);
                 vcommit(&bars->ds_free);
                 vcommit(&bars->q_empty[st]);
+                // dP^T(i+1): its columns were last read for dS^T(i) (ds_full(i)), and dO(i+1)
+                // arrived before S^T(i+1)
+                if (it + 1 < NTT) {
+                    issue_dp(it + 1);
+                    vcommit(&bars->dp_full);
+                }
             }
             if (ok) vcommit(&bars->dkv_done);
             vcommit(&bars->teardown);
@@ -437,7 +441,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         auto drain = [&](int it) -> bool {
             const int i = i_begin + it % NT;
             const int qbh = kvbh * p.kv_group + it / NT;
-            if (!wait_all(&bars->dq_full, it & 1)) return false;
+            const int b2 = it & 1;
+            if (!wait_all(&bars->dq_full[b2], (it >> 1) & 1)) return false;
             tc_fence_after();
             if (p.deterministic) {
                 // add this tile's partial only after every lower key tile has added its own
@@ -462,28 +467,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 if (*abort) got = false;
                 if (!__all_sync(0xffffffffu, got)) {
                     tc_fence_before();
-                    mbar_arrive(&bars->dq_drained);
+                    mbar_arrive(&bars->dq_drained[b2]);
                     return false;
                 }
             }
             float* acc_tile = p.dq_acc + (static_cast<size_t>(qbh) * p.n_pad + i * 128) * D;
-            if constexpr (C::DQT) {
-                // lane r = head-dim index; columns = queries cb .. cb+63
-#pragma unroll 1
-                for (int c = 0; c < 2; ++c) {
-                    uint32_t u[32];
-                    tmem_ld32(tDP + cb + c * 32, u);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int x = 0; x < 32; ++x)
-                        red_add_f32(acc_tile + (cb + c * 32 + x) * D + r, __uint_as_float(u[x]));
-                }
-            } else {
+            {
                 // lane r = query row; columns = head-dim g*D/2 .. (g+1)*D/2-1
+                const uint32_t tDQ = tmem + lane_base + COL_DQ + b2 * 64 + g * (D / 2);
                 float* row = acc_tile + r * D + g * (D / 2);
                 if constexpr (D / 2 == 32) {
                     uint32_t u[32];
-                    tmem_ld32(tDP + g * 32, u);
+                    tmem_ld32(tDQ, u);
                     tmem_ld_wait();
 #pragma unroll
                     for (int x = 0; x < 8; ++x)
@@ -491,7 +486,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                        __uint_as_float(u[4 * x + 2]), __uint_as_float(u[4 * x + 3]));
                 } else {
                     uint32_t u[16];
-                    tmem_ld16(tDP + g * 16, u);
+                    tmem_ld16(tDQ, u);
                     tmem_ld_wait();
 #pragma unroll
                     for (int x = 0; x < 4; ++x)
@@ -500,7 +495,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 }
             }
             tc_fence_before();
-            mbar_arrive(&bars->dq_drained);
+            mbar_arrive(&bars->dq_drained[b2]);
             if (p.deterministic) {
                 __threadfence();
                 wg_bar();
