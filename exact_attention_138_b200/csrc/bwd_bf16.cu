@@ -216,7 +216,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int gbase = (L / (p.group * p.nkt)) * p.group;
     const int gsize = min(p.group, p.BH - gbase);
     const int r_in = L - gbase * p.nkt;
-    const int j = r_in / gsize;
+    // deterministic mode adds dQ partials in decreasing key-tile order, so CTAs of high key tiles
+    // are launched first (a CTA only ever waits for CTAs launched before it)
+    const int j = p.deterministic ? p.nkt - 1 - r_in / gsize : r_in / gsize;
     const int kvbh = gbase + r_in % gsize;        // K/V head of this CTA
     const MaskSpec& mk = p.mask;
     const int nk = mk.nk;
@@ -445,10 +447,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!wait_all(&bars->dq_full[b2], (it >> 1) & 1)) return false;
             tc_fence_after();
             if (p.deterministic) {
-                // add this tile's partial only after every lower key tile has added its own
-                // (each CTA contributes two halves, one per warpgroup)
+                // add this tile's partial only after every higher key tile that meets the query
+                // tile has added its own (each CTA contributes two halves, one per warpgroup)
                 volatile int* sem = p.sems + static_cast<size_t>(qbh) * qt128 + i;
-                const int need = 2 * (j - first_key_tile(mk, i * 128LL, 128));
+                const int need = 2 * (last_key_tile(mk, i * 128LL, 128, 128) - j);
                 bool got = true;
                 if (t == 0) {
                     const uint64_t t0 = globaltimer_ns();
@@ -713,7 +715,8 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
     const int gbase = (L / (p.group * p.nkt)) * p.group;
     const int gsize = min(p.group, p.BH - gbase);
     const int r_in = L - gbase * p.nkt;
-    const int j = r_in / gsize;
+    // deterministic mode: high key tiles first (see bwd_main_kernel)
+    const int j = p.deterministic ? p.nkt - 1 - r_in / gsize : r_in / gsize;
     const int kvbh = gbase + r_in % gsize;         // K/V head of this CTA
     const MaskSpec& mk = p.mask;
     const int nk = mk.nk;
@@ -895,6 +898,7 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
         };
         int half = 0;                                      // half tiles staged so far
         bool run = true;
+        volatile int* pending = nullptr;                   // semaphore still to be released
         for (int it = 0; run && it < NTT; ++it) {
             const int b2 = it & 1;
             if (!bounded_wait_warp(&bars->dq_full[b2], (it >> 1) & 1, abort, lim)) break;
@@ -911,22 +915,6 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
             float* dst = p.dq_acc + (static_cast<size_t>(qbh) * p.n_pad + i * BQ) * D;
             volatile int* sem = p.deterministic ? p.sems + static_cast<size_t>(qbh) * qt64 + i : nullptr;
             bool got = true;
-            if (sem && leader && lane == 0) {
-                // contributions to one query tile are added in increasing key-tile order,
-                // starting from the first key tile that this query tile meets
-                const int need = j - first_key_tile(mk, static_cast<long long>(i) * BQ, 128);
-                const uint64_t t0 = globaltimer_ns();
-                while (*sem < need) {
-                    if (*abort || globaltimer_ns() - t0 > lim) {
-                        *abort = 1;
-                        report_error(4);
-                        got = false;
-                        break;
-                    }
-                    __nanosleep(64);
-                }
-                __threadfence();
-            }
 #pragma unroll
             for (int h = 0; h < 2; ++h, ++half) {
                 float* slot = sStg + (half % STG_SLOTS) * (STG_SLOT / 4);
@@ -937,19 +925,46 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
                 for (int x = 0; x < 32; ++x) slot[x * D + r] = __uint_as_float(u[h * 32 + x]);
                 fence_proxy_async_smem();
                 if (!wg_sync(1)) { run = false; break; }
+                if (h == 0 && sem && leader && lane == 0) {
+                    // Contributions to one query tile are added in decreasing key-tile order,
+                    // starting from the last key tile that this query tile meets: those CTAs
+                    // began at higher query tiles and reached this one earlier, so in the steady
+                    // state nobody waits. The check sits after staging the first half, so that
+                    // staging overlaps the load.
+                    const int need = last_key_tile(mk, static_cast<long long>(i) * BQ, BQ, 128) - j;
+                    const uint64_t t0 = globaltimer_ns();
+                    while (ld_acquire_gpu(sem) < need) {   // the acquire orders the adds below
+                        if (*abort || globaltimer_ns() - t0 > lim) {
+                            *abort = 1;
+                            report_error(4);
+                            got = false;
+                            break;
+                        }
+                        __nanosleep(64);
+                    }
+                }
                 if (leader && lane == 0 && got) {
                     bulk_reduce_add_f32(dst + h * 32 * D, slot, STG_SLOT);
                     bulk_commit();
                 }
             }
             if (sem && leader && lane == 0 && got && run) {
-                bulk_wait_all();             // the adds are done, not only the reads
-                __threadfence();
-                atomicAdd(const_cast<int*>(sem), 1);
+                // Release the previous tile's semaphore one tile late, once its adds (not only
+                // their reads) are complete, i.e. at most this tile's two groups are pending:
+                // the drain keeps reductions in flight, and the CTAs of lower key tiles that wait
+                // on it reach that query tile two tiles after this one did.
+                if (pending) {
+                    bulk_wait_le2_complete();
+                    red_release_gpu_add(pending, 1);
+                }
+                pending = sem;
             }
             if (*abort) break;
         }
-        if (leader && lane == 0) bulk_wait_all();
+        if (leader && lane == 0) {
+            bulk_wait_all();
+            if (pending && !*abort) red_release_gpu_add(pending, 1);
+        }
         __syncwarp();
     } else if (warp < 8) {
         // ---------------------------------------------------------------- compute warpgroups

@@ -60,6 +60,15 @@ __host__ __device__ inline int first_key_tile(const MaskSpec& m, long long a, in
     return lo <= 0 ? 0 : static_cast<int>(lo / bk);
 }
 
+// Last key tile of `bk` keys met by the query tile of rows [a, a + bq) (clipped to nq); only
+// meaningful when the tile meets some key.
+__host__ __device__ inline int last_key_tile(const MaskSpec& m, long long a, int bq, int bk) {
+    long long lo, hi;
+    const long long b = a + bq - 1 < m.nq - 1 ? a + bq - 1 : m.nq - 1;
+    visible_keys(m, a, b, lo, hi);
+    return hi < 0 ? 0 : static_cast<int>(hi / bk);
+}
+
 __host__ __device__ inline int clamp_int(long long x) {
     return x < -0x7fffffffLL ? -0x7fffffff : (x > 0x7fffffffLL ? 0x7fffffff : static_cast<int>(x));
 }

@@ -150,6 +150,19 @@ __device__ __forceinline__ void bulk_wait_read_le1() {
 __device__ __forceinline__ void bulk_wait_read_le2() {
     asm volatile("cp.async.bulk.wait_group.read 2;" ::: "memory");
 }
+// Acquire load / release add at GPU scope on a global int (ordering across CTAs without a full
+// fence).
+__device__ __forceinline__ int ld_acquire_gpu(const volatile int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void red_release_gpu_add(volatile int* p, int v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_le2_complete() {
+    asm volatile("cp.async.bulk.wait_group 2;" ::: "memory");
+}
 __device__ __forceinline__ void bulk_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }

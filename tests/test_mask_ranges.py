@@ -31,6 +31,9 @@ extern "C" void qtiles(int nq, int nk, int wl, int wr, long long c, long long e,
 extern "C" int first_ktile(int nq, int nk, int wl, int wr, long long a, int bk) {
     return first_key_tile(spec(nq, nk, wl, wr), a, bk);
 }
+extern "C" int last_ktile(int nq, int nk, int wl, int wr, long long a, int bq, int bk) {
+    return last_key_tile(spec(nq, nk, wl, wr), a, bq, bk);
+}
 """
 
 
@@ -52,6 +55,8 @@ def lib(tmp_path_factory):
     L.qtiles.argtypes = [ctypes.c_int] * 4 + [LL, LL, ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
     L.first_ktile.argtypes = [ctypes.c_int] * 4 + [LL, ctypes.c_int]
     L.first_ktile.restype = ctypes.c_int
+    L.last_ktile.argtypes = [ctypes.c_int] * 4 + [LL, ctypes.c_int, ctypes.c_int]
+    L.last_ktile.restype = ctypes.c_int
     return L
 
 
@@ -118,10 +123,11 @@ def test_both_passes_agree_on_tile_pairs(lib, nq, nk, wl, wr, bq):
         if o2[0] <= o2[1]:
             fwd[t, o2[0] // 128:o2[1] // 128 + 1] = True
     assert np.array_equal(fwd, exact)
-    # deterministic ordering: the first key tile met by each query tile
+    # deterministic ordering: the first and last key tiles met by each query tile
     for t in range(nqt):
         if exact[t].any():
             assert lib.first_ktile(nq, nk, wl, wr, t * bq, 128) == np.nonzero(exact[t])[0][0]
+            assert lib.last_ktile(nq, nk, wl, wr, t * bq, bq, 128) == np.nonzero(exact[t])[0][-1]
 
 
 def test_full_visibility_test_matches_brute_force(lib):
