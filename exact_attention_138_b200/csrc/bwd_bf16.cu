@@ -638,20 +638,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // Same per-tile mathematics as bwd_main_kernel, arranged so that the dQ partial never blocks the
 // other MMAs: with 64 query rows per tile, TMEM holds
 //     dV [0,128) | dK [128,256) | S^T [256,320) | dP^T [320,384) | dQ^T x2 [384,448),[448,512)
-// so dQ^T is double-buffered in its own columns. Roles (352 threads):
+// so dQ^T is double-buffered in its own columns. Roles (512 threads; warps 10-11 idle):
 //   warps 0-3, 4-7  compute warpgroups, query columns 0-31 and 32-63 of each tile; one thread per
 //                   key row (TMEM lane).
 //   warp 8          TMA producer: K_j, V_j once; Q_i, dO_i (64 rows) and the matching 64 values of
 //                   LSE·log2e and D through a 3-deep ring.
-//   warp 9          MMA issuer, per tile:  dP^T(i) -> [P^T(i)] dV += P^T dO -> S^T(i+1) ->
-//                   [dS^T(i)] dK += dS^T Q -> dQ^T(i) = K^T dS^T (into buffer i mod 2).
+//   warp 9          MMA issuer (whole warp in the loop, one elected lane issues), per tile:
+//                   dP^T(i) -> [P^T(i)] dV += P^T dO -> S^T(i+1) -> [dS^T(i)] dK += dS^T Q ->
+//                   dQ^T(i) = K^T dS^T (into buffer i mod 2).
 //   warps 12-15     dQ drain warpgroup: copies dQ^T(i) out of TMEM (one head-dim row per thread)
 //                   into shared-memory staging laid out like the accumulator rows, one half tile
 //                   (32 queries x 128 fp32, 16 KB contiguous in global memory) per slot of a
 //                   3-slot ring, and one elected lane adds each half with a bulk reduction. The
 //                   reductions are limited by L2's read-modify-write rate, so two of them stay in
 //                   flight while the next half is staged. This work never sits on the compute
-//                   warps' path.
+//                   warps' path. Deterministic mode: a query tile's partials are added in
+//                   decreasing key-tile order, gated by one semaphore per query tile (acquire
+//                   load before the first half's reduction, release add one tile later, once the
+//                   tile's reductions are complete).
 // ------------------------------------------------------------------------------------------
 // Single-lane issue helpers for a converged warp (see elect_one).
 #define MMA_SS(...) do { if (elect_one()) mma_ss(__VA_ARGS__); } while (0)
