@@ -328,6 +328,8 @@ def main():
                     help="skip the extra timings of grouped-query, sliding-window and ring "
                          "attention on the bench inputs")
     ap.add_argument("--variant-steps", type=int, default=20)
+    ap.add_argument("--deterministic", action="store_true",
+                    help="time the backward with deterministic (ordered) dQ accumulation")
     ap.add_argument("--workload", default=WORKLOAD,
                     help="named workload of attn_inputs.WORKLOADS (profiling runs use a smaller "
                          "one; the headline is the default)")
@@ -365,14 +367,15 @@ def main():
     o = torch.empty_like(q)
     lse = torch.empty((w.B, w.H, w.n), dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws = torch.empty(ea.attn_bwd_workspace_bytes(w.B, w.H, w.n, w.d, 0), dtype=torch.uint8,
+    det = bool(args.deterministic)
+    ws = torch.empty(ea.attn_bwd_workspace_bytes(w.B, w.H, w.n, w.d, int(det)), dtype=torch.uint8,
                      device=dev)
     stream = torch.cuda.current_stream()
 
     def step():
         ea.forward(q, k, v, causal=True, scale=w.scale, out=o, lse=lse, stream=stream)
         ea.backward(q, k, v, o, do, lse, causal=True, scale=w.scale, dq=dq, dk=dk, dv=dv,
-                    workspace=ws, stream=stream)
+                    workspace=ws, stream=stream, deterministic=det)
 
     def barrier():
         if dist is not None:
@@ -402,7 +405,7 @@ def main():
             ea.forward(q, k, v, causal=True, scale=w.scale, out=o, lse=lse, stream=stream)
             ea.attn_set_bwd_phase_events(e[1:5])
             ea.backward(q, k, v, o, do, lse, causal=True, scale=w.scale, dq=dq, dk=dk, dv=dv,
-                        workspace=ws, stream=stream)
+                        workspace=ws, stream=stream, deterministic=det)
             ea.attn_set_bwd_phase_events(None)
             e[5].record(stream)
         t_end.record(stream)
@@ -500,7 +503,7 @@ def main():
             stream.wait_event(ev_out[b])             # step st-2's results have left outs[b]
             ea.forward(qb, kb, vb, causal=True, scale=w.scale, out=ob, lse=lseb, stream=stream)
             ea.backward(qb, kb, vb, ob, dob, lseb, causal=True, scale=w.scale, dq=dqb, dk=dkb,
-                        dv=dvb, workspace=ws, stream=stream)
+                        dv=dvb, workspace=ws, stream=stream, deterministic=det)
             ev_comp[b].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_comp[b])
@@ -536,6 +539,7 @@ def main():
         "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "n": w.n, "d": w.d, "causal": True,
                    "input_factor": w.factor, "global_batch": w.B * world,
+                   "dq_accumulation": "deterministic" if det else "atomic",
                    "parallelism": f"dp{world}" if world > 1 else "single",
                    "l2": f"inputs larger than L2 (q,k,v,dO {w.B*w.H*w.n*w.d*2/2**20:.0f} MiB "
                          f"each); no flush"},
