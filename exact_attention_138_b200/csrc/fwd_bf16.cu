@@ -38,11 +38,6 @@ namespace {
 constexpr int kFwdThreads = 384;   // 3 warpgroups
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
-#ifndef ATTN_FWD_EXP_FMA_PER8
-#define ATTN_FWD_EXP_FMA_PER8 0
-#endif
-constexpr int kExpFmaPer8 = ATTN_FWD_EXP_FMA_PER8;   // column pairs (of every 8) whose exp2 runs
-                                                     // on the FMA pipe
 
 template <int D, bool F8>
 struct FwdCfg {
@@ -441,35 +436,17 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap* tmQ_, const CUtensor
             const uint64_t sl2x2 = f2_pack(sl2, sl2);
             const uint64_t nm2 = f2_pack(-m_use, -m_use);
             uint64_t rsa = f2_pack(0.f, 0.f), rsb = f2_pack(0.f, 0.f);
-            if (edge) {
-                // tiles with masked (-inf) scores: every exponential on the MUFU, exact zeros
+            // P = exp2(s·c - m) on the MUFU (masked -inf scores give exact zeros), two row-sum
+            // accumulators to shorten the add chain
 #pragma unroll
-                for (int c = 0; c < 128; c += 2) {
-                    float x0, x1;
-                    f2_unpack(f2_fma(f2_pack(__uint_as_float(u[c]), __uint_as_float(u[c + 1])),
-                                     sl2x2, nm2), x0, x1);
-                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-                    if (c & 2) rsb = f2_add(rsb, f2_pack(p0, p1));
-                    else rsa = f2_add(rsa, f2_pack(p0, p1));
-                    store_p<F8>(u, c, p0, p1);
-                }
-            } else {
-                // kExpFmaPer8 of every 8 column pairs use the FMA-pipe exp2, the rest the MUFU
-#pragma unroll
-                for (int c = 0; c < 128; c += 2) {
-                    float x0, x1, p0, p1;
-                    f2_unpack(f2_fma(f2_pack(__uint_as_float(u[c]), __uint_as_float(u[c + 1])),
-                                     sl2x2, nm2), x0, x1);
-                    if (((c / 2) & 7) >= 8 - kExpFmaPer8) {
-                        exp2_fma_x2(x0, x1, p0, p1);
-                    } else {
-                        p0 = ex2_approx(x0);
-                        p1 = ex2_approx(x1);
-                    }
-                    if (c & 2) rsb = f2_add(rsb, f2_pack(p0, p1));
-                    else rsa = f2_add(rsa, f2_pack(p0, p1));
-                    store_p<F8>(u, c, p0, p1);
-                }
+            for (int c = 0; c < 128; c += 2) {
+                float x0, x1;
+                f2_unpack(f2_fma(f2_pack(__uint_as_float(u[c]), __uint_as_float(u[c + 1])),
+                                 sl2x2, nm2), x0, x1);
+                const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                if (c & 2) rsb = f2_add(rsb, f2_pack(p0, p1));
+                else rsa = f2_add(rsa, f2_pack(p0, p1));
+                store_p<F8>(u, c, p0, p1);
             }
             float ra0, ra1, rb0, rb1;
             f2_unpack(rsa, ra0, ra1);

@@ -420,33 +420,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return d;
 }
 
-// 2^x for two values on the FMA pipe (no MUFU). Reduction x = n + f with n = round(x) obtained
-// by adding 1.5·2^23 (the integer lands in the low mantissa bits), f in [-1/2, 1/2]; 2^f from a
-// degree-3 polynomial fitted by the Remez exchange algorithm for minimax relative error
-// (coefficients derived in exp2_poly_fit.py; max relative error 7.5e-5 in fp32), and 2^n applied
-// by adding n to the exponent field with one integer multiply-add on the bit patterns.
-// Inputs are clamped to >= -125 so that the result stays a normal number; the true value there
-// is below 2.4e-38. Used only where no element is masked to -inf.
-__device__ __forceinline__ void exp2_fma_x2(float x0, float x1, float& y0, float& y1) {
-    constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
-    x0 = fmaxf(x0, -125.f);
-    x1 = fmaxf(x1, -125.f);
-    const uint64_t x = f2_pack(x0, x1);
-    const uint64_t j = f2_add(x, f2_pack(kMagic, kMagic));
-    const uint64_t nround = f2_add(j, f2_pack(-kMagic, -kMagic));
-    const uint64_t f = f2_fma(nround, f2_pack(-1.f, -1.f), x);
-    uint64_t p = f2_fma(f2_pack(0.0551716685295105f, 0.0551716685295105f), f,
-                        f2_pack(0.2426111251115799f, 0.2426111251115799f));
-    p = f2_fma(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
-    p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
-    float p0, p1, j0, j1;
-    f2_unpack(p, p0, p1);
-    f2_unpack(j, j0, j1);
-    // bits(j) = 0x4B400000 + n, so bits(j) * 2^23 == n << 23 (mod 2^32)
-    y0 = __uint_as_float(__float_as_uint(j0) * 8388608u + __float_as_uint(p0));
-    y1 = __uint_as_float(__float_as_uint(j1) * 8388608u + __float_as_uint(p1));
-}
-
 // Two floats -> packed bf16x2 (round to nearest even); `lo` goes to the low 16 bits.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
