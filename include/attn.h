@@ -127,7 +127,7 @@ int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse
  * memory of at least attn_bwd_workspace_bytes() bytes, 256-byte aligned) is overwritten.
  *   deterministic == 0: dQ partial tiles are added to the fp32 accumulator with atomic adds, so
  *                       the rounding order (and the last bits of dq) can vary between runs.
- *   deterministic != 0: each query tile's partials are added in increasing key-tile order, so
+ *   deterministic != 0: each query tile's partials are added in decreasing key-tile order, so
  *                       repeated runs give identical bits. */
 int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
              const float* lse, void* dq, void* dk, void* dv,
@@ -146,8 +146,8 @@ int attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, con
 /* Backward pass of attn_fwd_ex (bf16 only): dq (B, H, nq, d); dk, dv (B, Hkv, nk, d), summed over
  * the query heads of each K/V head. Keys that no query sees get dk = dv = 0. The workspace is
  * attn_bwd_workspace_bytes(B, H, nq, d, deterministic) (query rows). Everything else as attn_bwd;
- * the deterministic mode adds the dQ partials of a query tile in increasing key-tile order,
- * starting from the first key tile that the tile meets. */
+ * the deterministic mode adds the dQ partials of a query tile in decreasing key-tile order,
+ * starting from the last key tile that the tile meets. */
 int attn_bwd_ex(const void* q, const void* k, const void* v, const void* o, const void* dO,
                 const float* lse, void* dq, void* dk, void* dv,
                 int B, int H, int Hkv, int nq, int nk, int d, float scale,
