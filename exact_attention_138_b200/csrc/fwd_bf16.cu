@@ -11,8 +11,9 @@
 //
 // B200 mapping (one CTA per pair of 128-row query tiles of one (b,h)):
 //   warp 8      TMA producer: Q tiles once, then K_j / V_j tiles through a STAGES-deep ring.
-//   warp 9      one thread issues every tcgen05.mma:  S_g = Q_g·K_j^T (SMEM x SMEM -> TMEM) and
-//               O_g += P_g·V_j (P from TMEM, V from SMEM), and signals through tcgen05.commit.
+//   warp 9      issues every tcgen05.mma (the whole warp runs the loop, one lane chosen by
+//               elect.sync issues): S_g = Q_g·K_j^T (SMEM x SMEM -> TMEM) and O_g += P_g·V_j
+//               (P from TMEM, V from SMEM), and signals through tcgen05.commit.
 //   warps 0-3   softmax of query tile 0, warps 4-7 softmax of query tile 1: one thread per row
 //               (= one TMEM lane). They read S from TMEM, apply the mask on tiles that straddle
 //               its boundary, update m/l, rescale O in TMEM when m grows, and write P (bf16)
