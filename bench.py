@@ -229,6 +229,110 @@ def run_reference(args, w):
     return 0
 
 
+# The pages' small forward-only cases: short n (2x3x128x32 fp32) and small d (1x1x4096x64 fp32
+# and bf16). They fill a small fraction of the GPU, so they are timed per launch with L2 flushed
+# in between and reported as achieved HBM bandwidth beside the FLOP rate.
+SMALL_CASES = ("p1_fp32_2x3x128x32", "rowtile_fp32_4096x64", "rowtile_bf16_4096x64")
+L2_FLUSH_BYTES = 256 << 20          # written between timed launches (L2 is 126 MB)
+SM_COUNT = 148
+
+
+def fwd_case_bytes(w):
+    """Algorithmic HBM bytes of one forward launch: q, k, v read once, O written, fp32 LSE
+    written."""
+    e = 4 if w.dtype == "fp32" else 2
+    return 4 * w.B * w.H * w.n * w.d * e + 4 * w.B * w.H * w.n
+
+
+def fwd_case_ctas(w):
+    """CTAs of one forward launch: 64-row query tiles in fp32, pairs of 128-row tiles in bf16."""
+    rows = 64 if w.dtype == "fp32" else 256
+    return w.B * w.H * ((w.n + rows - 1) // rows)
+
+
+def time_forward_case(ea, w, dev, stream, iters, warmup, hbm_peak, fma_peak):
+    """Median device time of one forward launch of workload `w` over `iters` launches, each
+    preceded by a write of a buffer larger than L2 so that q, k, v come from HBM."""
+    import torch
+    import attn_inputs
+    q, k, v, _ = attn_inputs.workload_inputs(w)
+    q, k, v = (t.to(dev) for t in (q, k, v))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.n), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def fwd():
+        ea.forward(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse, stream=stream)
+
+    for _ in range(warmup):
+        fwd()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(iters)]
+    with torch.cuda.stream(stream):
+        for a, b in ev:
+            flush.zero_()
+            a.record(stream)
+            fwd()
+            b.record(stream)
+    torch.cuda.synchronize()
+    if ea.device_status() != ea.ATTN_OK:
+        raise SystemExit(f"device status not OK in the {w.name} forward timings")
+    us = statistics.median(a.elapsed_time(b) * 1e3 for a, b in ev)
+    nbytes = fwd_case_bytes(w)
+    flops = 4.0 * w.B * w.H * w.n * w.n * w.d * (0.5 if w.causal else 1.0)
+    gbs = nbytes / (us * 1e-6) / 1e9
+    tflops = flops / (us * 1e-6) / 1e12
+    out = {"us": us, "launches": iters, "bytes": nbytes, "hbm_gbs": gbs,
+           "hbm_frac": gbs / hbm_peak, "tflops": tflops, "ctas": fwd_case_ctas(w),
+           "sms": SM_COUNT, "dtype": w.dtype,
+           "l2": f"{L2_FLUSH_BYTES >> 20} MiB written before every launch"}
+    if w.dtype == "fp32":
+        out["fma_frac"] = tflops / fma_peak
+    return out
+
+
+def fma_peak_tflops(sm_max_mhz):
+    """fp32 FFMA peak: SMs x 128 lanes x 2 FLOP x the maximum SM clock."""
+    return SM_COUNT * 128 * 2 * sm_max_mhz * 1e6 / 1e12
+
+
+def run_forward_case(args, w):
+    """One forward-only workload (the pages' small cases): one JSON line with its per-launch time,
+    achieved HBM bandwidth and FLOP rate. A profiling and reporting mode; the headline run carries
+    the same numbers under `small_cases`."""
+    import torch
+    if int(os.environ.get("WORLD_SIZE", "1")) != 1:
+        raise SystemExit("forward-only workloads run on one GPU")
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    import exact_attention_138_b200 as ea
+    peaks, peak_src = load_peaks()
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    stream = torch.cuda.current_stream()
+    with ClockSampler(0) as clocks:
+        r = time_forward_case(ea, w, dev, stream, args.steps, args.warmup, hbm,
+                              fma_peak_tflops(1965.0))
+    clk = clocks.summary()
+    fma = fma_peak_tflops(clk["sm_max_mhz"] or 1965.0)
+    if "fma_frac" in r:
+        r["fma_frac"] = r["tflops"] / fma
+    line = {
+        "metric": "attention forward latency and achieved HBM bandwidth (small case)",
+        "value": r["us"], "unit": "us", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "higher_is_better": False, "dtype": w.dtype,
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "n": w.n, "d": w.d,
+                   "causal": w.causal, "l2": r["l2"]},
+        "roofline": {"bound": "hbm", "achieved": r["hbm_gbs"], "peak": hbm, "unit": "GB/s",
+                     "frac": r["hbm_frac"], "peak_kind": f"hbm_gbs ({peak_src})",
+                     "traffic": None},
+        "case": r, "gpu_launches": args.steps, "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def visible_pairs(nq, nk, wl, wr):
     """Number of (query, key) pairs a mask leaves visible (query i aligned with key i + nk - nq;
     key j visible iff i + off - wl <= j <= i + off + wr, negative = unbounded)."""
@@ -328,6 +432,9 @@ def main():
                     help="skip the extra timings of grouped-query, sliding-window and ring "
                          "attention on the bench inputs")
     ap.add_argument("--variant-steps", type=int, default=20)
+    ap.add_argument("--no-small-cases", action="store_true",
+                    help="skip the per-launch timings of the small forward-only cases")
+    ap.add_argument("--small-case-launches", type=int, default=50)
     ap.add_argument("--deterministic", action="store_true",
                     help="time the backward with deterministic (ordered) dQ accumulation")
     ap.add_argument("--workload", default=WORKLOAD,
@@ -339,7 +446,11 @@ def main():
 
     import attn_inputs
     w = attn_inputs.WORKLOADS[args.workload]
-    if not (w.causal and w.dtype == "bf16" and w.backward):
+    if not w.backward:
+        if args.impl == "reference":
+            ap.error("the reference arm times the forward+backward workloads")
+        return run_forward_case(args, w)
+    if not (w.causal and w.dtype == "bf16"):
         ap.error("the bench workload must be a causal bf16 forward+backward workload")
     if args.impl == "reference":
         return run_reference(args, w)
@@ -469,6 +580,17 @@ def main():
     if not args.no_variants and world == 1:
         variants = time_variants(args, w, ea, q, k, v, do, ws, stream, fwd_flops + bwd_flops)
 
+    # --- extra: the pages' small forward-only cases, per launch with L2 flushed in between
+    small = None
+    if not args.no_small_cases and world == 1:
+        hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        fma = fma_peak_tflops(1965.0)
+        small = {name: time_forward_case(ea, attn_inputs.WORKLOADS[name], dev, stream,
+                                         args.small_case_launches, args.warmup, hbm, fma)
+                 for name in SMALL_CASES}
+        small["peaks"] = {"hbm_gbs": hbm, "fp32_fma_tflops": fma,
+                          "fp32_fma_kind": "148 SMs x 128 lanes x 2 FLOP x 1965 MHz"}
+
     # --- end to end through the public API with host buffers (pinned), copies inside the timing.
     # Three streams run as a pipeline: while step k computes, step k+1's inputs travel host ->
     # device and step k-1's results device -> host (two device buffer sets; every step copies
@@ -566,6 +688,8 @@ def main():
         line["fp8_fwd"] = fp8
     if variants is not None:
         line["variants"] = variants
+    if small is not None:
+        line["small_cases"] = small
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, dt, rows_n, threads = oracle_sample(args.cpu_seconds, q_h, k_h, v_h, do_h, w)
         line["cpu_baseline"] = {

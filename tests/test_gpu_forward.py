@@ -103,3 +103,20 @@ def test_gqa_forward_fp32(cuda_device, Hkv):
     ro, rlse = oracle.fwd_gqa(q, k, v, 0.125, True)
     assert np.abs(to_np(o) - ro).max() <= TOL_O["fp32"]
     assert np.abs(to_np(lse) - rlse).max() <= TOL_LSE["fp32"]
+
+
+# fp32 grids on both sides of the key split. A query tile is 64 rows; when the tiles alone leave
+# the GPU under-filled the kernel splits each tile's key range over a cluster of 2-8 CTAs and
+# merges their (m, l, O) on chip. (2,8,1000,64) and (1,12,1000,128) give 256 and 192 tiles (no
+# split, many key tiles per CTA); (1,1,1000,128) 16 tiles (8 shares, some empty under the causal
+# mask); (2,3,700,32) 66 tiles (4 uneven shares of 11 key tiles).
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", [(2, 8, 1000, 64), (1, 12, 1000, 128), (1, 1, 1000, 128),
+                                   (2, 3, 700, 32)], ids=lambda s: "x".join(map(str, s)))
+def test_forward_fp32_split_and_unsplit_grids(cuda_device, shape, causal):
+    q, k, v = attn_inputs.random_draws(shape, dtype="fp32", seed=sum(shape), count=3)
+    scale = 1.0 / math.sqrt(shape[-1])
+    o, lse, _ = cuda_forward(q, k, v, causal, scale)
+    ro, rlse = oracle.fwd(q, k, v, scale, causal)
+    assert np.abs(to_np(o) - ro).max() <= TOL_O["fp32"]
+    assert np.abs(to_np(lse) - rlse).max() <= TOL_LSE["fp32"]
