@@ -244,9 +244,10 @@ def fwd_case_bytes(w):
     return 4 * w.B * w.H * w.n * w.d * e + 4 * w.B * w.H * w.n
 
 
-def fwd_case_ctas(w):
-    """CTAs of one forward launch: 64-row query tiles in fp32, pairs of 128-row tiles in bf16."""
-    rows = 64 if w.dtype == "fp32" else 256
+def fwd_case_query_tiles(w):
+    """Query tiles of one forward launch: 64 rows in fp32, 128 rows in bf16 (the fp32 kernel may
+    split each tile's keys over a cluster of CTAs; the bf16 kernel runs tiles in pairs)."""
+    rows = 64 if w.dtype == "fp32" else 128
     return w.B * w.H * ((w.n + rows - 1) // rows)
 
 
@@ -284,7 +285,7 @@ def time_forward_case(ea, w, dev, stream, iters, warmup, hbm_peak, fma_peak):
     gbs = nbytes / (us * 1e-6) / 1e9
     tflops = flops / (us * 1e-6) / 1e12
     out = {"us": us, "launches": iters, "bytes": nbytes, "hbm_gbs": gbs,
-           "hbm_frac": gbs / hbm_peak, "tflops": tflops, "ctas": fwd_case_ctas(w),
+           "hbm_frac": gbs / hbm_peak, "tflops": tflops, "query_tiles": fwd_case_query_tiles(w),
            "sms": SM_COUNT, "dtype": w.dtype,
            "l2": f"{L2_FLUSH_BYTES >> 20} MiB written before every launch"}
     if w.dtype == "fp32":
