@@ -66,6 +66,9 @@ int attn_version(void);
  *   dtype ATTN_BF16: tcgen05 tensor-core kernel, fp32 accumulation, P rounded to bf16 before P·V,
  *                    O rounded to bf16 (round-to-nearest-even).
  *   dtype ATTN_FP32: exact fp32 kernel on the FMA pipes (no TF32), for the pages' float32 cases.
+ *                    When B*H*ceil(n/64) query tiles would leave the SMs under-filled, each tile's
+ *                    keys are split over a thread-block cluster of up to 8 CTAs whose partial
+ *                    (max, sum, O) are merged on chip; still one launch and no library memory.
  * causal != 0 applies the mask M of §4.4 (query i sees keys 0..i). */
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              int B, int H, int n, int d, float scale, int causal, int dtype, void* stream);
