@@ -29,6 +29,8 @@
 //   Masks (causal, sliding window, query/key lengths that differ; see MaskSpec): each query tile
 //   visits only the key tiles that hold a key it can see; the two tiles of a pair stream the
 //   union of their ranges once. A row that sees no key gets O = 0 and LSE = -inf.
+#include <cooperative_groups.h>
+
 #include "kernels.h"
 #include "sm100_ptx.cuh"
 
@@ -54,6 +56,9 @@ struct FwdCfg {
     static constexpr int TILE = NCH * CHUNK;             // bytes of one 128 x D tile
     static constexpr int STAGES = TILE >= 32768 ? 2 : 3;
     static constexpr int SMEM = (2 + 2 * STAGES) * TILE + 512;
+    // the split kernel's partials (bf16 only: 2 x 128 rows x (D + 4) fp32, then 256 x (m, l)) fit in the
+    // Q/K/V staging memory they overwrite
+    static_assert(F8 || (2 * BM * (D + 4) + 2 * 2 * BM) * 4 <= (2 + 2 * STAGES) * TILE, "partials");
     static_assert(SWB == 128 || SWB == 64, "tile rows of 64 or 128 bytes");
 };
 
@@ -75,7 +80,15 @@ struct FwdKParams {
     float scale_log2;
     float o_scale;    // output multiplier (v_descale for E4M3 inputs, 1 for bf16)
     uint64_t timeout_ns;
+    int split;        // key shares per tile pair (cluster size of the split kernel; else 1)
 };
+
+// Every thread of every CTA of the cluster arrives, then waits (release / acquire ordering of
+// shared-memory writes across the cluster). Threads of a warp may arrive at different times.
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release;\n" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire;\n" ::: "memory");
+}
 
 // Bounded wait that ignores the abort flag: used while draining in-flight copies/MMAs on the
 // way out, so that nothing is left writing into shared memory or TMEM after the CTA exits.
@@ -106,7 +119,10 @@ __device__ __forceinline__ void store_p(uint32_t* u, int c, float p0, float p1) 
     }
 }
 
-template <int D, bool F8>
+// SPLIT: the CTAs of a cluster share the key tiles of one tile pair (small grids); each keeps its
+// unnormalised O and (m, l) for its share, and the cluster merges them through distributed
+// shared memory with the rule that joins two softmax blocks (weights 2^(m_s - M)).
+template <int D, bool F8, bool SPLIT>
 __device__ __forceinline__ void fwd_body(const CUtensorMap* tmQ_, const CUtensorMap* tmK_,
                                          const CUtensorMap* tmV_, const FwdKParams& p) {
     using C = FwdCfg<D, F8>;
@@ -124,7 +140,7 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap* tmQ_, const CUtensor
     // Heads are processed in groups of p.group (sized so that a group's K and V stay in L2);
     // within a group, tile pairs go from the last to the first (longest first under a causal
     // mask) across the group's heads.
-    const int L = blockIdx.x;
+    const int L = SPLIT ? static_cast<int>(blockIdx.x) / p.split : static_cast<int>(blockIdx.x);
     const int gbase = (L / (p.group * p.n_pairs)) * p.group;
     const int gsize = min(p.group, p.BH - gbase);
     const int r_in = L - gbase * p.n_pairs;
@@ -147,6 +163,16 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap* tmQ_, const CUtensor
                 J0[g] = static_cast<int>(lo / C::BN);
                 T[g] = static_cast<int>(hi / C::BN) + 1 - J0[g];
             }
+        }
+    }
+    if constexpr (SPLIT) {
+        // this CTA's share (its rank in the cluster) of each tile's key tiles
+        const int rank = static_cast<int>(blockIdx.x) % p.split;
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+            const int a0 = T[g] * rank / p.split, a1 = T[g] * (rank + 1) / p.split;
+            J0[g] += a0;
+            T[g] = a1 - a0;
         }
     }
     const int Jmin = T[0] > 0 ? (T[1] > 0 ? min(J0[0], J0[1]) : J0[0]) : J0[1];
@@ -352,6 +378,10 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap* tmQ_, const CUtensor
         }
         __syncwarp();
     }
+    if constexpr (SPLIT) {   // the producer warpgroup takes part in the two cluster barriers
+        cluster_sync_all();
+        cluster_sync_all();
+    }
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 208;");
         // ---------------------------------------------------------------- softmax warpgroups
@@ -462,7 +492,78 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap* tmQ_, const CUtensor
             tc_fence_before();
             mbar_arrive(&bars->p_full[g]);
         }
-        if (ok && T[g] > 0) {
+        if constexpr (SPLIT) {
+            // Partial of this share: unnormalised O (fp32, rows padded to D + 4 floats) and
+            // (m, l) per row, written over the Q/K/V staging memory once both tiles' MMAs are
+            // complete; a row with no key in this share has m = -inf, l = 0.
+            bool have = ok && T[g] > 0;
+            if (have) {
+                have = bounded_wait(&bars->o_done[g], 0, abort, lim);
+                have = __all_sync(0xffffffffu, have);
+            }
+            asm volatile("bar.sync 1, 256;" ::: "memory");   // both softmax warpgroups
+            tc_fence_after();
+            constexpr int OP = D + 4;
+            float* Ob = reinterpret_cast<float*>(smem);
+            float* ML = Ob + 2 * C::BM * OP;
+            const int row = g * C::BM + r;
+            if (have) {
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t u[32];
+                    tmem_ld32(tO + c * 32, u);
+                    tmem_ld_wait();
+                    float4* dst = reinterpret_cast<float4*>(Ob + row * OP + c * 32);
+#pragma unroll
+                    for (int x = 0; x < 8; ++x)
+                        dst[x] = make_float4(__uint_as_float(u[4 * x]), __uint_as_float(u[4 * x + 1]),
+                                             __uint_as_float(u[4 * x + 2]),
+                                             __uint_as_float(u[4 * x + 3]));
+                }
+            }
+            ML[2 * row] = have ? m : -INFINITY;
+            ML[2 * row + 1] = have ? l : 0.f;
+            cluster_sync_all();
+            // Merge: this CTA finishes rows [rank*R, rank*R + R) of the pair's 256 rows.
+            namespace cg = cooperative_groups;
+            cg::cluster_group cluster = cg::this_cluster();
+            const int split = p.split;
+            const int rank = static_cast<int>(blockIdx.x) % split;
+            const int R = 2 * C::BM / split;
+            constexpr int C4 = D / 4;
+            for (int idx = static_cast<int>(threadIdx.x); idx < R * C4; idx += 256) {
+                const int rw = rank * R + idx / C4, c4 = idx % C4;
+                const int qi = (2 * pair + rw / C::BM) * C::BM + rw % C::BM;
+                if (qi >= nq) continue;
+                float M = -INFINITY;
+                for (int s2 = 0; s2 < split; ++s2)
+                    M = fmaxf(M, cluster.map_shared_rank(ML, s2)[2 * rw]);
+                float Lsum = 0.f;
+                float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int s2 = 0; s2 < split; ++s2) {
+                    const float* mls = cluster.map_shared_rank(ML, s2);
+                    const float ms = mls[2 * rw];
+                    if (ms == -INFINITY) continue;
+                    const float w = ex2_approx(ms - M);
+                    Lsum = fmaf(w, mls[2 * rw + 1], Lsum);
+                    const float4 t = *reinterpret_cast<const float4*>(
+                        cluster.map_shared_rank(Ob, s2) + rw * OP + c4 * 4);
+                    o.x = fmaf(w, t.x, o.x);
+                    o.y = fmaf(w, t.y, o.y);
+                    o.z = fmaf(w, t.z, o.z);
+                    o.w = fmaf(w, t.w, o.w);
+                }
+                const float inv = Lsum > 0.f ? p.o_scale / Lsum : 0.f;
+                __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) +
+                                      (static_cast<size_t>(bh) * nq + qi) * D;
+                *reinterpret_cast<uint2*>(orow + c4 * 4) =
+                    make_uint2(pack_bf16x2(o.x * inv, o.y * inv), pack_bf16x2(o.z * inv, o.w * inv));
+                if (c4 == 0)
+                    p.lse[static_cast<size_t>(bh) * nq + qi] =
+                        Lsum > 0.f ? (M + __log2f(Lsum)) * kLn2 : -INFINITY;
+            }
+            cluster_sync_all();   // peers may still be reading this CTA's shared memory
+        } else if (ok && T[g] > 0) {
             ok = bounded_wait(&bars->o_done[g], 0, abort, lim);
             ok = __all_sync(0xffffffffu, ok);
             if (ok) {
@@ -515,7 +616,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdKParams p) {
-    fwd_body<D, false>(&tmQ, &tmK, &tmV, p);
+    fwd_body<D, false, false>(&tmQ, &tmK, &tmV, p);
+}
+
+// Small grids: launched in clusters of p.split CTAs that share each tile pair's key tiles.
+template <int D>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    fwd_bf16_split_kernel(const __grid_constant__ CUtensorMap tmQ,
+                          const __grid_constant__ CUtensorMap tmK,
+                          const __grid_constant__ CUtensorMap tmV, const FwdKParams p) {
+    fwd_body<D, false, true>(&tmQ, &tmK, &tmV, p);
 }
 
 template <int D>
@@ -523,7 +633,31 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ,
                    const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const FwdKParams p) {
-    fwd_body<D, true>(&tmQ, &tmK, &tmV, p);
+    fwd_body<D, true, false>(&tmQ, &tmK, &tmV, p);
+}
+
+// Key shares per tile pair for the bf16 forward: 1 when the pairs alone fill half the SMs, else the
+// smallest power of two (at most 8, at most the largest number of key tiles a query tile sees)
+// that brings the grid close to one CTA per SM.
+int choose_fwd_split(const MaskSpec& mk, int qtiles, long long pairs_total) {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+        sms = 148;
+    if (pairs_total * 2 > sms) return 1;
+    int max_tiles = 0;
+    for (int t = 0; t < qtiles; ++t) {
+        long long lo, hi;
+        const long long a = static_cast<long long>(t) * 128;
+        visible_keys(mk, a, a + 127 < mk.nq - 1 ? a + 127 : mk.nq - 1, lo, hi);
+        if (lo <= hi) {
+            const int c = static_cast<int>(hi / 128 - lo / 128 + 1);
+            if (c > max_tiles) max_tiles = c;
+        }
+    }
+    int s = 1;
+    while (s < 8 && pairs_total * s * 2 <= sms && s * 2 <= max_tiles) s *= 2;
+    return s;
 }
 
 template <int D, bool F8>
@@ -559,10 +693,30 @@ cudaError_t launch_fwd_d(const FwdArgs& a, cudaStream_t stream) {
     kp.scale_log2 = a.scale * kLog2e * (F8 ? a.q_descale * a.k_descale : 1.f);
     kp.o_scale = F8 ? a.v_descale : 1.f;
     kp.timeout_ns = a.timeout_ns;
-    const long long grid = static_cast<long long>(kp.n_pairs) * BH;
+    const long long pairs_total = static_cast<long long>(kp.n_pairs) * BH;
+    kp.split = F8 ? 1 : choose_fwd_split(kp.mask, qtiles, pairs_total);
+    const long long grid = pairs_total * kp.split;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    kern<<<static_cast<unsigned>(grid), kFwdThreads, C::SMEM, stream>>>(mq, mk, mv, kp);
-    return cudaGetLastError();
+    if (kp.split == 1) {
+        kern<<<static_cast<unsigned>(grid), kFwdThreads, C::SMEM, stream>>>(mq, mk, mv, kp);
+        return cudaGetLastError();
+    }
+    e = cudaFuncSetAttribute(fwd_bf16_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kFwdThreads);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(kp.split);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, fwd_bf16_split_kernel<D>, mq, mk, mv, kp);
 }
 
 }  // namespace
