@@ -636,10 +636,46 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     fwd_body<D, true, false>(&tmQ, &tmK, &tmV, p);
 }
 
+// Clusters of `split` CTAs of the split kernel that the GPU holds at once (each CTA takes a whole
+// SM, and a cluster must fit in one GPC); queried once per (d, split). While `stream` is being
+// captured into a graph the query is not made and half of SMs / split is assumed.
+template <int D>
+int max_active_clusters(int split, int sms, cudaStream_t stream) {
+    static int cache[4] = {0, 0, 0, 0};
+    const int slot = split == 2 ? 0 : split == 4 ? 1 : split == 8 ? 2 : 3;
+    if (cache[slot] > 0) return cache[slot];
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone)
+        return sms / (2 * split);
+    using C = FwdCfg<D, false>;
+    if (cudaFuncSetAttribute(fwd_bf16_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM) != cudaSuccess)
+        return 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(split * 256));
+    cfg.blockDim = dim3(kFwdThreads);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(split);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, fwd_bf16_split_kernel<D>, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return 0;
+    }
+    cache[slot] = n;
+    return n;
+}
+
 // Key shares per tile pair for the bf16 forward: 1 when the pairs alone fill half the SMs, else the
-// smallest power of two (at most 8, at most the largest number of key tiles a query tile sees)
-// that brings the grid close to one CTA per SM.
-int choose_fwd_split(const MaskSpec& mk, int qtiles, long long pairs_total) {
+// largest power of two (at most 8, at most the largest number of key tiles a query tile sees)
+// that keeps the grid within one CTA per SM and every cluster resident at once.
+template <int D>
+int choose_fwd_split(const MaskSpec& mk, int qtiles, long long pairs_total, cudaStream_t stream) {
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
@@ -656,7 +692,9 @@ int choose_fwd_split(const MaskSpec& mk, int qtiles, long long pairs_total) {
         }
     }
     int s = 1;
-    while (s < 8 && pairs_total * s * 2 <= sms && s * 2 <= max_tiles) s *= 2;
+    while (s < 8 && pairs_total * s * 2 <= sms && s * 2 <= max_tiles &&
+           pairs_total <= max_active_clusters<D>(s * 2, sms, stream))
+        s *= 2;
     return s;
 }
 
@@ -694,7 +732,7 @@ cudaError_t launch_fwd_d(const FwdArgs& a, cudaStream_t stream) {
     kp.o_scale = F8 ? a.v_descale : 1.f;
     kp.timeout_ns = a.timeout_ns;
     const long long pairs_total = static_cast<long long>(kp.n_pairs) * BH;
-    kp.split = F8 ? 1 : choose_fwd_split(kp.mask, qtiles, pairs_total);
+    kp.split = F8 ? 1 : choose_fwd_split<D>(kp.mask, qtiles, pairs_total, stream);
     const long long grid = pairs_total * kp.split;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     if (kp.split == 1) {
