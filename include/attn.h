@@ -64,7 +64,9 @@ int attn_version(void);
 
 /* Forward pass. Writes o (same dtype as q) and lse (fp32).
  *   dtype ATTN_BF16: tcgen05 tensor-core kernel, fp32 accumulation, P rounded to bf16 before P·V,
- *                    O rounded to bf16 (round-to-nearest-even).
+ *                    O rounded to bf16 (round-to-nearest-even). Small grids (fewer pairs of
+ *                    128-row query tiles than half the SMs) split each pair's keys over a cluster
+ *                    of 2-8 CTAs merged on chip; one launch, no library memory.
  *   dtype ATTN_FP32: exact fp32 kernel on the FMA pipes (no TF32), for the pages' float32 cases.
  *                    When B*H*ceil(n/64) query tiles would leave the SMs under-filled, each tile's
  *                    keys are split over a thread-block cluster of up to 8 CTAs whose partial
