@@ -5,7 +5,9 @@ import this package. It shares no code with the CUDA library (``exact_attention_
 neither imports the other.
 
 The arithmetic lives in ``attn_oracle.c`` (plain loops, fp64, OpenMP over independent rows);
-this module builds it with gcc when needed and marshals numpy arrays through ctypes. Inputs are
+this module builds it with gcc when needed and marshals numpy arrays through ctypes. One
+function, ``bwd_key_rows_batched``, is numpy instead: the same derivative with fp64 matrix
+products over batches of query rows, for sequences where the C loops would take days. Inputs are
 passed as float32 arrays: fp32 inputs and bf16-rounded inputs are both represented exactly in
 float32 and are widened to float64 inside the C code.
 
@@ -200,6 +202,63 @@ def bwd_key_rows(q, k, v, do, scale, causal, bh, keys):
     dv = np.empty((len(keys), d), np.float64)
     _check(_load().oracle_bwd_key_rows(q, k, v, do, B, H, n, d, float(scale), int(bool(causal)),
                                        int(bh), keys, len(keys), dk, dv), "oracle_bwd_key_rows")
+    return dk, dv
+
+
+def bwd_key_rows_batched(q, k, v, do, scale, causal, bh, keys, block_rows=256):
+    """dK and dV for key rows `keys` of head bh, for sequences too long for ``bwd_key_rows``.
+
+    Same derivative as ``bwd_key_rows`` (the exact gradient of "Attention Mechanism ...", §3
+    Steps 1-4 with the causal mask of §4.4; the pages only say that the backward pass recomputes
+    the softmax: "Apa itu FlashAttention", "Cara kerja teknik Tiling dan Recomputation", item 2),
+    but every query row's score row, softmax and dP row come from an fp64 matrix product
+    (numpy matmul, a library primitive) over a batch of `block_rows` query rows at a time — the
+    row batching of "Efficient Attention" (efficient_attention.py, part 3), which changes no
+    row's arithmetic. The C loops of ``bwd_key_rows`` stream all of K for every query row, which
+    at n = 131072 is petabytes of memory traffic; this form does the same steps in minutes.
+
+    Per batch of query rows i in [r0, r1), in fp64:
+      1. S = scale · Q_rows · K^T over keys j < r1 under the causal mask (keys j >= r1 are masked
+         for every row of the batch: their P entries are exactly 0 and drop out of every sum);
+         over all keys otherwise; then S_ij = -inf for j > i when causal.
+      2. m_i = max_j S_ij, P_ij = exp(S_ij - m_i) / sum_j exp(S_ij - m_i)   (full rows).
+      3. dP = dO_rows · V^T;  D_i = sum_j P_ij dP_ij;  dS = P ∘ (dP - D).
+      4. for each sampled key t: dK_t += scale · sum_i dS_it q_i,  dV_t += sum_i P_it dO_i.
+    Returns (dK rows, dV rows), each (len(keys), d) fp64.
+    """
+    q, k, v, do = _f32(q), _f32(k), _f32(v), _f32(do)
+    B, H, n, d = _shape4(q)
+    bh = int(bh)
+    if not (0 <= bh < B * H):
+        raise ValueError("head index out of range")
+    keys = np.asarray(keys, dtype=np.int64)
+    if keys.size < 1 or keys.min() < 0 or keys.max() >= n:
+        raise ValueError("key index out of range")
+    Q = q.reshape(B * H, n, d)[bh].astype(np.float64)
+    K = k.reshape(B * H, n, d)[bh].astype(np.float64)
+    V = v.reshape(B * H, n, d)[bh].astype(np.float64)
+    dO = do.reshape(B * H, n, d)[bh].astype(np.float64)
+    dk = np.zeros((keys.size, d), np.float64)
+    dv = np.zeros((keys.size, d), np.float64)
+    r_start = int(keys.min()) if causal else 0      # rows i < min key see none of the keys
+    for r0 in range(r_start, n, block_rows):
+        r1 = min(n, r0 + block_rows)
+        kend = r1 if causal else n
+        S = (Q[r0:r1] @ K[:kend].T) * scale                              # step 1
+        if causal:
+            rows = np.arange(r0, r1)[:, None]
+            S[np.arange(kend)[None, :] > rows] = -np.inf
+        m = S.max(axis=1, keepdims=True)                                 # step 2
+        P = np.exp(S - m)
+        P /= P.sum(axis=1, keepdims=True)
+        dP = dO[r0:r1] @ V[:kend].T                                      # step 3
+        D = (P * dP).sum(axis=1, keepdims=True)
+        dS = P * (dP - D)
+        sel = keys < kend                                                # step 4
+        if sel.any():
+            cols = keys[sel]
+            dk[sel] += scale * (dS[:, cols].T @ Q[r0:r1])
+            dv[sel] += P[:, cols].T @ dO[r0:r1]
     return dk, dv
 
 

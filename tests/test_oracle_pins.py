@@ -253,6 +253,33 @@ def test_sampled_rows_equal_full(causal):
         np.testing.assert_allclose(vv, dv.reshape(4, 150, 32)[bh][keys], rtol=0, atol=1e-13)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_batched_key_rows_equal_full(causal):
+    # The batched form (matrix products over 64-row batches, a ragged last batch of 44 rows)
+    # reproduces the loop oracle's full backward at keys on both sides of batch edges.
+    q, k, v, do = (_rand((2, 2, 300, 32), s) for s in (60, 61, 62, 63))
+    dq, dk, dv, _ = oracle.bwd(q, k, v, do, 0.18, causal)
+    keys = [0, 1, 63, 64, 150, 256, 299]
+    for bh in (0, 3):
+        kk, vv = oracle.bwd_key_rows_batched(q, k, v, do, 0.18, causal, bh, keys, block_rows=64)
+        np.testing.assert_allclose(kk, dk.reshape(4, 300, 32)[bh][keys], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(vv, dv.reshape(4, 300, 32)[bh][keys], rtol=0, atol=1e-12)
+
+
+def test_batched_key_rows_match_autograd_fp64():
+    # Independent of the loop oracle: torch fp64 autograd of the causal definition.
+    q, k, v, do = (_rand((1, 2, 70, 8), s) for s in (64, 65, 66, 67))
+    scale = 0.4
+    Q, K, V = (torch.from_numpy(x.astype(np.float64)).requires_grad_() for x in (q, k, v))
+    S = (Q @ K.transpose(-1, -2) * scale).masked_fill(
+        torch.ones(70, 70, dtype=torch.bool).triu(1), float("-inf"))
+    (torch.softmax(S, -1) @ V).backward(torch.from_numpy(do.astype(np.float64)))
+    keys = [0, 15, 16, 40, 69]
+    kk, vv = oracle.bwd_key_rows_batched(q, k, v, do, scale, True, 1, keys, block_rows=16)
+    np.testing.assert_allclose(kk, K.grad.numpy()[0, 1][keys], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(vv, V.grad.numpy()[0, 1][keys], rtol=0, atol=1e-12)
+
+
 # --------------------------------------------------------------------------------------------
 # Backward: autograd fp64, finite differences, invariants
 # --------------------------------------------------------------------------------------------
