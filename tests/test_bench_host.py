@@ -35,3 +35,23 @@ def test_small_case_bytes_and_tiles():
 def test_fma_peak():
     # 148 SMs x 128 fp32 lanes x 2 FLOP per FFMA at 1965 MHz
     assert abs(bench.fma_peak_tflops(1965.0) - 74.44992) < 1e-9
+
+
+def test_roofline_peak_choice():
+    # burst unless the timed region is over a second AND the power cap was seen
+    burst, sust = 1655.5, 1405.2
+    p, why = bench.roofline_peak(burst, sust, 80.0, {"reasons": ["sw_power_cap"]}, "measured")
+    assert p == burst and "burst" in why
+    p, why = bench.roofline_peak(burst, sust, 5000.0, {"reasons": []}, "measured")
+    assert p == burst
+    p, why = bench.roofline_peak(burst, sust, 5000.0, {"reasons": ["sw_power_cap"]}, "measured")
+    assert p == sust and "sustained" in why
+
+
+def test_backward_main_algorithmic_bytes():
+    # 2x32x8192x128: Q, K, V, dO in and dK, dV out (bf16), LSE·log2e and D (fp32), fp32 dQ
+    # accumulator read and written once
+    w = attn_inputs.WORKLOADS["causal_bf16_2x32x8192x128"]
+    rows = 2 * 32 * 8192
+    assert bench.bwd_main_bytes(w) == rows * 128 * 2 * 6 + rows * 8 + rows * 128 * 8
+    assert abs(bench.bwd_main_bytes(w) / 1e9 - 1.3465) < 1e-3
