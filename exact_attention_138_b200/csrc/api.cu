@@ -110,6 +110,23 @@ cudaError_t make_tmap(CUtensorMap* map, const void* base, int esize, int BH, int
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// Argument checks of the backward entry points, everything but the workspace: null and
+// misaligned pointers, sizes, scale, head counts and dtype.
+int validate_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                 const float* lse, const void* dq, const void* dk, const void* dv, int B, int H,
+                 int Hkv, int nq, int nk, int d, float scale, int dtype) {
+    if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return ATTN_ERR_INVALID;
+    int rc = validate_common(B, H, nq, d, scale, dtype);
+    if (rc) return rc;
+    if (nk < 1 || nk > kMaxSeq) return ATTN_ERR_INVALID;
+    if (Hkv < 1 || H % Hkv != 0) return ATTN_ERR_INVALID;
+    if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+    const void* ptrs[] = {q, k, v, o, dO, lse, dq, dk, dv};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return ATTN_ERR_INVALID;
+    return ATTN_OK;
+}
+
 cudaError_t launch_wait_selftest(uint64_t timeout_ns, cudaStream_t stream) {
     wait_selftest_kernel<<<1, 32, 0, stream>>>(timeout_ns);
     return cudaGetLastError();
@@ -216,15 +233,8 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
                     const float* lse, void* dq, void* dk, void* dv, int B, int H, int Hkv, int nq,
                     int nk, int d, float scale, int wl, int wr, int dtype, int deterministic,
                     void* workspace, size_t ws_bytes, void* stream) {
-    if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return ATTN_ERR_INVALID;
-    int rc = validate_common(B, H, nq, d, scale, dtype);
+    int rc = validate_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, H, Hkv, nq, nk, d, scale, dtype);
     if (rc) return rc;
-    if (nk < 1 || nk > kMaxSeq) return ATTN_ERR_INVALID;
-    if (Hkv < 1 || H % Hkv != 0) return ATTN_ERR_INVALID;
-    if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
-    const void* ptrs[] = {q, k, v, o, dO, lse, dq, dk, dv};
-    for (const void* p : ptrs)
-        if (!aligned16(p)) return ATTN_ERR_INVALID;
     WsLayout w = ws_layout(B, H, nq, d, deterministic);
     if (!workspace) return ATTN_ERR_INVALID;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_INVALID;

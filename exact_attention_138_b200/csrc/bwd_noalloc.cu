@@ -18,8 +18,12 @@
 //     accumulator and the semaphores are produced by its first kernel), so no clearing is needed
 //     between calls; but two calls whose kernels overlap on the GPU (different streams without an
 //     ordering between them, or several host threads) race on the array and give wrong results.
-//   - The device address of the array is looked up with cudaGetSymbolAddress by the first call
-//     on each device (with that device current); make that first call before any stream capture.
+//   - Outside stream capture every call looks up the array's device address on the current
+//     device (cudaGetSymbolAddress, cheap), so a context that was reset and re-created is seen
+//     at once. While the stream is being captured into a graph no runtime lookup is made: the
+//     address that the latest uncaptured call on that device found is used, so make one call on
+//     each device (outside capture) before capturing; a captured call without one fails with
+//     ATTN_ERR_CUDA.
 #include <mutex>
 
 #include "../../include/attn.h"
@@ -38,20 +42,32 @@ constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
 void* g_noalloc_ptr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device, looked up once per device.
-cudaError_t scratch_for_current_device(void** out) {
+// Device address of the scratch array on the current device: looked up afresh outside capture,
+// taken from the last lookup on this device while `stream` is capturing.
+cudaError_t scratch_for_current_device(cudaStream_t stream, void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_ptr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        g_noalloc_ptr[dev] = p;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    bool capturing = false;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) {
+        (void)cudaGetLastError();   // e.g. the legacy stream while another stream captures
+        capturing = true;
+    } else {
+        capturing = cap != cudaStreamCaptureStatusNone;
     }
-    *out = g_noalloc_ptr[dev];
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (capturing) {
+        if (!g_noalloc_ptr[dev]) return cudaErrorStreamCaptureUnsupported;
+        *out = g_noalloc_ptr[dev];
+        return cudaSuccess;
+    }
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[dev] = p;
+    *out = p;
     return cudaSuccess;
 }
 
@@ -62,8 +78,16 @@ extern "C" int attn_bwd_noalloc(const void* q, const void* k, const void* v, con
                                 const void* dO, const float* lse, void* dq, void* dk, void* dv,
                                 int B, int H, int n, int d, float scale, int causal, int dtype,
                                 int deterministic, void* stream) {
+    // The arguments and the size limit are checked before the device is touched, so an invalid
+    // call returns its own error even where no device is usable.
+    int rc = attn::validate_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, H, H, n, n, d, scale, dtype);
+    if (rc != ATTN_OK) return rc;
+    if (attn_bwd_workspace_bytes(B, H, n, d, deterministic) > attn::kNoAllocScratchBytes)
+        return ATTN_ERR_WORKSPACE;
     void* scratch = nullptr;
-    if (attn::scratch_for_current_device(&scratch) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (attn::scratch_for_current_device(static_cast<cudaStream_t>(stream), &scratch) !=
+        cudaSuccess)
+        return ATTN_ERR_CUDA;
     // Same validation, kernels and error codes as attn_bwd; the workspace is the fixed array.
     return attn_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, H, n, d, scale, causal, dtype,
                     deterministic, scratch, attn::kNoAllocScratchBytes, stream);

@@ -31,6 +31,8 @@
 //   union of their ranges once. A row that sees no key gets O = 0 and LSE = -inf.
 #include <cooperative_groups.h>
 
+#include <atomic>
+
 #include "kernels.h"
 #include "sm100_ptx.cuh"
 
@@ -637,16 +639,33 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 }
 
 // Clusters of `split` CTAs of the split kernel that the GPU holds at once (each CTA takes a whole
-// SM, and a cluster must fit in one GPC); queried once per (d, split). While `stream` is being
-// captured into a graph the query is not made and half of SMs / split is assumed.
+// SM, and a cluster must fit in one GPC); queried once per (device, d, split) and kept in a
+// per-device table of atomics, so concurrent host threads and GPUs of different layouts each see
+// their own device's answer. While `stream` is being captured into a graph the query is not made
+// and half of SMs / split is assumed.
+constexpr int kClusterCacheDevices = 64;
+
 template <int D>
 int max_active_clusters(int split, int sms, cudaStream_t stream) {
-    static int cache[4] = {0, 0, 0, 0};
+    static std::atomic<int> cache[kClusterCacheDevices][4];
     const int slot = split == 2 ? 0 : split == 4 ? 1 : split == 8 ? 2 : 3;
-    if (cache[slot] > 0) return cache[slot];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return 0;
+    }
+    std::atomic<int>* entry =
+        (dev >= 0 && dev < kClusterCacheDevices) ? &cache[dev][slot] : nullptr;
+    if (entry) {
+        const int known = entry->load(std::memory_order_relaxed);
+        if (known > 0) return known;
+    }
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone)
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) {
+        (void)cudaGetLastError();
         return sms / (2 * split);
+    }
+    if (cap != cudaStreamCaptureStatusNone) return sms / (2 * split);
     using C = FwdCfg<D, false>;
     if (cudaFuncSetAttribute(fwd_bf16_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM) != cudaSuccess)
@@ -667,7 +686,7 @@ int max_active_clusters(int split, int sms, cudaStream_t stream) {
         (void)cudaGetLastError();
         return 0;
     }
-    cache[slot] = n;
+    if (entry) entry->store(n, std::memory_order_relaxed);
     return n;
 }
 

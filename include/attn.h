@@ -32,7 +32,7 @@
  * Errors: each call validates its arguments before launching anything and returns ATTN_OK or
  *   ATTN_ERR_INVALID   null pointer, B, H or n < 1, n > 2^31 - 257, misaligned pointer,
  *                      non-finite or <= 0 scale,
- *                      workspace pointer null while ws_bytes > 0;
+ *                      workspace pointer null or not 256-byte aligned;
  *   ATTN_ERR_UNSUPPORTED  d not in {32, 64, 128}; fp32 backward; an unknown dtype;
  *   ATTN_ERR_WORKSPACE    ws_bytes smaller than attn_bwd_workspace_bytes();
  *   ATTN_ERR_CUDA      a launch or encode error reported by the CUDA runtime / driver;
@@ -169,8 +169,10 @@ int attn_bwd_ex(const void* q, const void* k, const void* v, const void* o, cons
  * deterministic) exceeds 32 MiB (33,554,432 bytes). All calls on a device share the array and
  * leave their contents in it; each call rewrites or zeroes what it reads, but calls whose kernels
  * overlap on the GPU (unordered streams, concurrent host threads) race and give wrong results.
- * The first call on each device looks up the array's device address (cudaGetSymbolAddress, with
- * that device current): make that first call before any stream capture. */
+ * Arguments and the size limit are checked before any CUDA call. Outside stream capture each call
+ * looks up the array's device address on the current device (cudaGetSymbolAddress); while the
+ * stream is being captured the address found by the latest uncaptured call on that device is
+ * used, so make one call on each device before capturing (otherwise ATTN_ERR_CUDA). */
 int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO,
                      const float* lse, void* dq, void* dk, void* dv,
                      int B, int H, int n, int d, float scale, int causal, int dtype,

@@ -146,3 +146,24 @@ def test_fp8_and_ring_entry_points_validate_before_launch():
     assert ea.attn_ring_accumulate(f, f, 12, ea.ATTN_BF16, 0, None, 0, None) == ea.ATTN_ERR_INVALID
     assert ea.attn_ring_accumulate(ctypes.c_void_p(FAKE + 4), None, 16, 0, 0, None, 0, None) == \
         ea.ATTN_ERR_INVALID
+
+
+def test_noalloc_validates_before_touching_the_device():
+    # Argument errors and the 32 MiB scratch limit are reported before any CUDA call, so these
+    # return their own codes on a host without a GPU.
+    fn = ea.library().attn_bwd_noalloc
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.c_void_p] * 9 + [ctypes.c_int] * 4 + [ctypes.c_float] + \
+        [ctypes.c_int] * 3 + [ctypes.c_void_p]
+
+    def call(ptrs, B=1, H=2, n=300, d=128, scale=0.1, dtype=ea.ATTN_BF16, det=0):
+        return fn(*[ctypes.c_void_p(p) for p in ptrs], B, H, n, d, scale, 1, dtype, det, None)
+
+    ok = [FAKE] * 9
+    assert call([0] + ok[1:]) == ea.ATTN_ERR_INVALID
+    assert call(ok[:6] + [FAKE + 4] + ok[7:]) == ea.ATTN_ERR_INVALID
+    assert call(ok, d=48) == ea.ATTN_ERR_UNSUPPORTED
+    assert call(ok, dtype=ea.ATTN_FP32) == ea.ATTN_ERR_UNSUPPORTED
+    assert call(ok, scale=0.0) == ea.ATTN_ERR_INVALID
+    assert ea.attn_bwd_workspace_bytes(1, 64, 8192, 128, 0) > (32 << 20)
+    assert call(ok, B=1, H=64, n=8192) == ea.ATTN_ERR_WORKSPACE

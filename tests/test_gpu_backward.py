@@ -56,7 +56,7 @@ def full_run(request, cuda_device):
 
 def test_backward_full_size_sampled_query_rows(full_run):
     w, (q, k, v, do), (dq, _, _) = full_run
-    rows = attn_inputs.sampled_rows(w, count=128)
+    rows = attn_inputs.sampled_rows(w, count=256)
     rq, _ = oracle.bwd_query_rows(q, k, v, do, w.scale, True, rows)
     idx = torch.tensor(rows, device=dq.device)
     got = to_np(dq.reshape(-1, w.d).index_select(0, idx))

@@ -1,7 +1,11 @@
 """GPU test of attn_bwd_noalloc, the backward entry point that needs no caller workspace (for
-callers that cannot allocate device memory where they run the backward pass). It must give the
-same gradients as attn_bwd, call after call, since its fixed scratch array keeps the previous
-call's contents. This file is collected last on purpose."""
+callers that cannot allocate device memory where they run the backward pass, such as a plug-in
+whose host framework owns every allocation). Its scratch is one fixed array that keeps the
+previous call's contents, so the test checks call after call: against the fp64 oracle, against
+attn_bwd with a workspace (bit for bit in the deterministic mode, which fixes the order of every
+addition), and across calls of different sizes and modes whose leftovers (semaphores, padded D /
+LSE rows, accumulator rows) sit where the next call's data goes. Outputs are NaN-filled before
+each call, so a row the call fails to write shows up. This file is collected last on purpose."""
 import ctypes
 import math
 
@@ -11,7 +15,8 @@ import torch
 
 import attn_inputs
 import exact_attention_138_b200 as ea
-from parity_util import TOL_GRAD_REL, rel_fro
+import oracle
+from parity_util import TOL_GRAD_REL, grad_close, rel_fro, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -25,27 +30,68 @@ def _noalloc():
     return fn
 
 
-@pytest.mark.parametrize("shape,causal,det", [((1, 2, 300, 128), True, 0), ((2, 1, 200, 64), False, 1)])
-def test_noalloc_matches_workspace_entry_point(cuda_device, shape, causal, det):
-    q, k, v, do = (t.to(cuda_device) for t in attn_inputs.random_draws(shape, seed=21, count=4))
-    B, H, n, d = shape
-    scale = 1.0 / math.sqrt(d)
-    o, lse = ea.forward(q, k, v, causal=causal, scale=scale)
-    ref = ea.backward(q, k, v, o, do, lse, causal=causal, scale=scale, deterministic=bool(det))
-    fn = _noalloc()
-    stream = _vp(torch.cuda.current_stream().cuda_stream)
-    P = lambda t: _vp(t.data_ptr())
-    for _ in range(2):        # two calls in a row: the shared array holds the previous call's data
-        dq, dk, dv = (torch.full_like(q, float("nan")) for _ in range(3))
-        rc = fn(P(q), P(k), P(v), P(o), P(do), P(lse), P(dq), P(dk), P(dv), B, H, n, d, scale,
-                int(causal), ea.ATTN_BF16, det, stream)
+class Case:
+    """Inputs on the GPU, the forward outputs, the oracle's gradients and attn_bwd's."""
+
+    def __init__(self, device, shape, causal, det, seed):
+        host = attn_inputs.random_draws(shape, seed=seed, count=4)
+        self.shape, self.causal, self.det = shape, causal, det
+        self.scale = 1.0 / math.sqrt(shape[-1])
+        self.q, self.k, self.v, self.do = (t.to(device) for t in host)
+        self.o, self.lse = ea.forward(self.q, self.k, self.v, causal=causal, scale=self.scale)
+        self.want = oracle.bwd(*host, self.scale, causal)[:3]
+        self.ws_result = [t.clone() for t in ea.backward(
+            self.q, self.k, self.v, self.o, self.do, self.lse, causal=causal, scale=self.scale,
+            deterministic=bool(det))]
+        torch.cuda.synchronize()
+        assert ea.device_status() == ea.ATTN_OK
+
+    def run_noalloc(self):
+        B, H, n, d = self.shape
+        grads = [torch.full_like(self.q, float("nan")) for _ in range(3)]
+        P = lambda t: _vp(t.data_ptr())   # noqa: E731
+        rc = _noalloc()(P(self.q), P(self.k), P(self.v), P(self.o), P(self.do), P(self.lse),
+                        *(P(g) for g in grads), B, H, n, d, self.scale, int(self.causal),
+                        ea.ATTN_BF16, self.det, _vp(torch.cuda.current_stream().cuda_stream))
         assert rc == ea.ATTN_OK
         assert ea.device_status() == ea.ATTN_OK
-        for got, want in zip((dq, dk, dv), ref):
-            g = got.float().cpu().numpy().astype(np.float64)
-            w = want.float().cpu().numpy().astype(np.float64)
+        return grads
+
+    def check(self, grads):
+        for got, want, ref in zip(grads, self.want, self.ws_result):
+            g = to_np(got)
             assert np.isfinite(g).all()
-            assert rel_fro(g, w) <= TOL_GRAD_REL
+            assert grad_close(g, want)                      # the oracle
+            if self.det:
+                assert torch.equal(got, ref)                # same order of additions
+            else:
+                assert rel_fro(g, to_np(ref)) <= TOL_GRAD_REL
+
+
+@pytest.mark.parametrize("shape,causal,det", [((1, 2, 300, 128), True, 0),
+                                              ((2, 1, 200, 64), False, 1)])
+def test_noalloc_matches_oracle_and_workspace_entry_point(cuda_device, shape, causal, det):
+    case = Case(cuda_device, shape, causal, det, seed=21)
+    for _ in range(2):        # two calls in a row: the shared array holds the previous call's data
+        case.check(case.run_noalloc())
+
+
+def test_noalloc_leftovers_of_other_sizes_do_not_leak(cuda_device):
+    # A larger deterministic call fills semaphores, padded rows and accumulator rows far past
+    # where the smaller calls that follow put theirs; the smaller ones change the layout (heads,
+    # lengths, d, mask, dQ mode), and the first call is repeated at the end.
+    big = Case(cuda_device, (1, 4, 2048, 128), True, 1, seed=22)
+    small_atomic = Case(cuda_device, (2, 1, 300, 64), False, 0, seed=23)
+    mid_det = Case(cuda_device, (1, 3, 1000, 128), True, 1, seed=24)
+    assert ea.attn_bwd_workspace_bytes(1, 4, 2048, 128, 1) <= (32 << 20)
+    first = big.run_noalloc()
+    big.check(first)
+    for case in (small_atomic, mid_det, small_atomic):
+        case.check(case.run_noalloc())
+    again = big.run_noalloc()
+    big.check(again)
+    for a, b in zip(first, again):
+        assert torch.equal(a, b)
 
 
 def test_noalloc_rejects_sizes_beyond_its_array(cuda_device):
