@@ -58,7 +58,7 @@ struct WsLayout {
     size_t d_off, l2_off, acc_off, sem_off, total;
 };
 
-// D (fp32) | LSE·log2e (fp32) | dQ accumulator (fp32, d per row) | semaphores (one per 64 rows),
+// D (fp32) | LSE·log2e (fp32) | dQ accumulator (fp32, d per row) | semaphores (four per 64 rows),
 // every per-row array padded per head to a multiple of 128 rows.
 WsLayout ws_layout(int B, int H, int n, int d, int deterministic) {
     const size_t BH = static_cast<size_t>(B) * H;
@@ -68,7 +68,7 @@ WsLayout ws_layout(int B, int H, int n, int d, int deterministic) {
     w.l2_off = round_up(BH * n_pad * sizeof(float));
     w.acc_off = w.l2_off + round_up(BH * n_pad * sizeof(float));
     w.sem_off = w.acc_off + round_up(BH * n_pad * d * sizeof(float));
-    w.total = w.sem_off + (deterministic ? round_up(BH * (n_pad / 64) * sizeof(int)) : 0);
+    w.total = w.sem_off + (deterministic ? round_up(BH * (n_pad / 64) * 4 * sizeof(int)) : 0);
     return w;
 }
 
@@ -125,6 +125,20 @@ int validate_bwd(const void* q, const void* k, const void* v, const void* o, con
     for (const void* p : ptrs)
         if (!aligned16(p)) return ATTN_ERR_INVALID;
     return ATTN_OK;
+}
+
+cudaError_t make_tmap_acc(CUtensorMap* map, float* base, long long rows, int d) {
+    auto fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    if (rows < 1 || rows > 0x7fffffffLL) return cudaErrorInvalidValue;   // 32-bit box coordinates
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * sizeof(float)};
+    cuuint32_t box[2] = {32u, 32u};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 cudaError_t launch_wait_selftest(uint64_t timeout_ns, cudaStream_t stream) {

@@ -633,60 +633,72 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 }
 
 // ------------------------------------------------------------------------------------------
-// Main backward kernel for d = 128 with 64-row query tiles.
+// Main backward kernel for d = 128: 64-row query tiles, two of them in flight.
 //
-// Same per-tile mathematics as bwd_main_kernel, arranged so that the dQ partial never blocks the
-// other MMAs: with 64 query rows per tile, TMEM holds
-//     dV [0,128) | dK [128,256) | S^T [256,320) | dP^T [320,384) | dQ^T x2 [384,448),[448,512)
-// so dQ^T is double-buffered in its own columns. Roles (512 threads; warps 10-11 idle):
-//   warps 0-3, 4-7  compute warpgroups, query columns 0-31 and 32-63 of each tile; one thread per
-//                   key row (TMEM lane).
+// A CTA owns one 128-key tile j (K_j and V_j stay in shared memory, dK and dV accumulate in
+// TMEM) and walks the 64-row query tiles that meet it. Per query tile i the work is a chain whose
+// links alternate between the tensor cores and the SIMT warps:
+//     S^T = K·Q^T -> P^T = exp2(S^T·c - LSE·log2e) -> dV += P^T·dO
+//     dP^T = V·dO^T -> dS^T = P^T∘(dP^T - D) -> dK += dS^T·Q,  dQ^T = K^T·dS^T -> drain
+// With one tile in flight the tensor cores idle whenever the warps form P^T or dS^T. Here two
+// compute warpgroups each take every other query tile, so while one works on tile i the tensor
+// cores run the products of its neighbour. TMEM (512 columns):
+//     dV [0,128) | dK [128,256) | S^T, then P^T, of even tiles [256,320), of odd tiles
+//     [320,384) | dP^T, then dQ^T, of even tiles [384,448), of odd tiles [448,512)
+// dQ^T(i) is written over dP^T(i) once dS^T(i) has been formed from it; tile i+2 reuses both
+// column ranges, its dP^T after the drain has read dQ^T(i) out.
+// Roles (512 threads; warp 11 idle):
+//   warps 0-3, 4-7  compute warpgroups 0 and 1: even and odd query tiles, all 64 query columns;
+//                   one thread per key row (TMEM lane).
 //   warp 8          TMA producer: K_j, V_j once; Q_i, dO_i (64 rows) and the matching 64 values of
 //                   LSE·log2e and D through a 3-deep ring.
-//   warp 9          MMA issuer (whole warp in the loop, one elected lane issues), per tile:
-//                   dP^T(i) -> [P^T(i)] dV += P^T dO -> S^T(i+1) -> [dS^T(i)] dK += dS^T Q ->
-//                   dQ^T(i) = K^T dS^T (into buffer i mod 2).
-//   warps 12-15     dQ drain warpgroup: copies dQ^T(i) out of TMEM (one head-dim row per thread)
-//                   into shared-memory staging laid out like the accumulator rows, one half tile
-//                   (32 queries x 128 fp32, 16 KB contiguous in global memory) per slot of a
-//                   3-slot ring, and one elected lane adds each half with a bulk reduction. The
-//                   reductions are limited by L2's read-modify-write rate, so two of them stay in
-//                   flight while the next half is staged. This work never sits on the compute
-//                   warps' path. Deterministic mode: a query tile's partials are added in
-//                   decreasing key-tile order, gated by one semaphore per query tile (acquire
-//                   load before the first half's reduction, release add one tile later, once the
-//                   tile's reductions are complete).
+//   warps 9, 10     MMA issuers (one elected lane issues each batch of MMAs with its commits;
+//                   a tcgen05.mma costs its issuing warp tens of cycles, so two warps on two SM
+//                   sub-partitions feed the tensor pipe):
+//                   warp 9:  S^T, dP^T of tile i [dQ^T(i-2) read out, Q/dO(i) loaded];
+//                   warp 10: dV(i) [P^T(i) ready], then dK(i), dQ^T(i) [dS^T(i) ready].
+//                   The commits of warp 10 cover warp 9's products of the same tile: P^T(i)
+//                   and dS^T(i) exist only once S^T(i) and dP^T(i) are complete.
+//   warps 12-15     dQ drain, each warp on its own: 32 head-dim columns of dQ(i) out of TMEM
+//                   (one column per lane), staged per half tile as a [32 queries][32 columns]
+//                   fp32 box and added to the fp32 accumulator by a TMA tensor reduction. The
+//                   deterministic mode orders the additions to each (query tile, column block)
+//                   by key tile, from the last key tile that meets the query tile down, with one
+//                   semaphore per query tile and drain warp (acquire load before the first
+//                   box, release add one tile later, once the tile's reductions are complete).
 // ------------------------------------------------------------------------------------------
-// Single-lane issue helpers for a converged warp (see elect_one).
-#define MMA_SS(...) do { if (elect_one()) mma_ss(__VA_ARGS__); } while (0)
-#define MMA_TS(...) do { if (elect_one()) mma_ts(__VA_ARGS__); } while (0)
-#define MMA_COMMIT(bar) do { if (elect_one()) mma_commit(bar); } while (0)
-
 namespace q64 {
-constexpr int kThreads = 512;              // warps 10-11 idle: the drain warpgroup must start at
-                                           // warp 12 to cover TMEM lane quarters 0-3
+constexpr int kThreads = 512;              // warp 11 idle: the drain warps must be warps
+                                           // 12-15 to cover TMEM lane quarters 0-3
 constexpr int BQ = 64;                     // query rows per tile
 constexpr int KTILE = 128 * 128 * 2;       // K_j or V_j: 2 chunks [128 rows][64 d], SW128
 constexpr int QTILE = 64 * 128 * 2;        // Q_i or dO_i: 2 chunks [64 rows][64 d]
 constexpr int QCHUNK = 64 * 128;           // bytes of one [64 rows][64 d] chunk
-constexpr int STAGES = 3;
+constexpr int STAGES = 3;                  // two tiles in flight plus one loading
 constexpr int DS_BYTES = 128 * 64 * 2;     // dS^T [128 keys][64 queries], one SW128 chunk
-constexpr int STG_SLOT = 32 * 128 * 4;     // dQ staging slot: [32 queries][128 d] fp32
-constexpr int STG_SLOTS = 3;
-constexpr int STG_BYTES = STG_SLOTS * STG_SLOT;
+constexpr int BOX = 32 * 32 * 4;           // drain box: [32 queries][32 columns] fp32
+constexpr int BOXES = 2;                   // boxes per drain warp (one reduction may be reading)
+constexpr int STG_BYTES = 4 * BOXES * BOX;
 constexpr int OFF_K = 0, OFF_V = KTILE, OFF_Q = 2 * KTILE, OFF_DO = OFF_Q + STAGES * QTILE;
-constexpr int OFF_DS = OFF_DO + STAGES * QTILE, OFF_STG = OFF_DS + DS_BYTES;
+constexpr int OFF_DS = OFF_DO + STAGES * QTILE;            // two buffers, by tile parity
+constexpr int OFF_STG = OFF_DS + 2 * DS_BYTES;
 constexpr int OFF_L2 = OFF_STG + STG_BYTES, OFF_DV = OFF_L2 + STAGES * 256;
 constexpr int OFF_BARS = OFF_DV + STAGES * 256;
 constexpr int SMEM = OFF_BARS + 256;
 static_assert(SMEM <= 232448, "dynamic shared memory per block");
+static_assert(OFF_DS % 1024 == 0 && OFF_STG % 128 == 0, "operand and box alignment");
+// registers: launched at 128 per thread; the producer/MMA warpgroup gives up 64, the drain
+// warpgroup 32, and the compute warpgroups take 48 each: 128·64 + 128·96 + 256·176 <= 512·128
+constexpr int kRegsIdle = 64, kRegsDrain = 96, kRegsCompute = 176;
+static_assert(128 * kRegsIdle + 128 * kRegsDrain + 256 * kRegsCompute <= kThreads * 128,
+              "register split");
 
 struct Bars {
     uint64_t kv_full;
     uint64_t q_full[STAGES], q_empty[STAGES];
-    uint64_t s_full, dp_full, p_full, ds_full, ds_free, dkv_done, teardown;
-    uint64_t dq_full[2], dq_drained[2];
-    uint64_t drain_sync[2];
+    // per tile parity (even / odd query tiles)
+    uint64_t s_full[2], dp_full[2], p_full[2], ds_full[2], ds_free[2], dq_full[2], dq_drained[2];
+    uint64_t dkv_done, teardown;
     uint32_t tmem_base;
     int abort;
 };
@@ -696,7 +708,7 @@ static_assert(sizeof(Bars) <= 256, "barrier block");
 __global__ void __launch_bounds__(q64::kThreads, 1)
     bwd_main_q64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                        const BwdKParams p) {
+                        const __grid_constant__ CUtensorMap tmAcc, const BwdKParams p) {
     using namespace q64;
     constexpr int D = 128;
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -710,7 +722,8 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
     float* sDv = reinterpret_cast<float*>(smem + OFF_DV);     // [STAGES][64]
     Bars* bars = reinterpret_cast<Bars*>(smem + OFF_BARS);
 
-    constexpr uint32_t COL_DV = 0, COL_DK = 128, COL_S = 256, COL_DP = 320, COL_DQ = 384;
+    // S^T/P^T and dP^T/dQ^T columns of a tile: base + 64 * (tile parity)
+    constexpr uint32_t COL_DV = 0, COL_DK = 128, COL_S = 256, COL_DP = 384;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -724,7 +737,7 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
     const int kvbh = gbase + r_in % gsize;         // K/V head of this CTA
     const MaskSpec& mk = p.mask;
     const int nk = mk.nk;
-    const int qt64 = p.n_pad / BQ;                 // semaphore stride per query head
+    const int qt64 = p.n_pad / BQ;                 // 64-row query tiles per query head
     int i_begin, i_end;                            // 64-row query tiles that meet this key tile
     visible_query_tiles(mk, j * 128LL, min(j * 128LL + 127, nk - 1LL), BQ, i_begin, i_end);
     const int NT = i_end - i_begin;                // query tiles per query head
@@ -736,19 +749,17 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
             mbar_init(&bars->q_full[s], 1);
             mbar_init(&bars->q_empty[s], 1);
         }
-        mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->dp_full, 1);
-        mbar_init(&bars->p_full, 256);
-        mbar_init(&bars->ds_full, 256);
-        mbar_init(&bars->ds_free, 1);
-        mbar_init(&bars->dkv_done, 1);
-        mbar_init(&bars->teardown, 1);
-        for (int b2 = 0; b2 < 2; ++b2) {
-            mbar_init(&bars->dq_full[b2], 1);
-            mbar_init(&bars->dq_drained[b2], 128);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&bars->s_full[x], 1);
+            mbar_init(&bars->dp_full[x], 1);
+            mbar_init(&bars->p_full[x], 128);
+            mbar_init(&bars->ds_full[x], 128);
+            mbar_init(&bars->ds_free[x], 1);
+            mbar_init(&bars->dq_full[x], 1);
+            mbar_init(&bars->dq_drained[x], 128);
         }
-        mbar_init(&bars->drain_sync[0], 128);
-        mbar_init(&bars->drain_sync[1], 128);
+        mbar_init(&bars->dkv_done, 1);
+        mbar_init(&bars->teardown, 2);                 // one commit per MMA issuer
         bars->abort = ((smem_addr(smem) & 1023u) != 0) ? 1 : 0;
         if (bars->abort) report_error(3);
         fence_barrier_init();
@@ -760,6 +771,7 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
         tma_prefetch_desc(&tmdO);
+        tma_prefetch_desc(&tmAcc);
     }
     tc_fence_before();
     __syncthreads();
@@ -768,6 +780,8 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
     volatile int* abort = &bars->abort;
     const uint64_t lim = p.timeout_ns;
 
+    if (warp >= 8 && warp < 12) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsIdle));
     if (warp == 8) {
         // ---------------------------------------------------------------- TMA producer
         if (lane == 0 && !*abort && NTT > 0) {
@@ -800,182 +814,184 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
                     drain_wait_bwd(&bars->q_full[it % STAGES], (it / STAGES) & 1, 100000000ull);
             }
         }
-    } else if (warp == 9) {
-        // ---------------------------------------------------------------- MMA issuer
-        // The whole warp runs this loop (warp-uniform state); one elected lane issues.
-        {
-            constexpr uint32_t idS = idesc_bf16_f32(128, 64, 0, 0);      // S^T, dP^T
-            constexpr uint32_t idKV = idesc_bf16_f32(128, 128, 0, 1);    // dV, dK
-            constexpr uint32_t idQ = idesc_bf16_f32(128, 64, 1, 1);      // dQ^T
-            const uint32_t aK = smem_addr(sK), aV = smem_addr(sV), aQ = smem_addr(sQ),
-                           adO = smem_addr(sdO), adS = smem_addr(sdS);
-            const SDesc K_k = sdesc(aK, 16, 1024, 2u), V_k = sdesc(aV, 16, 1024, 2u);
-            const SDesc K_mn = sdesc(aK, 16384, 1024, 2u);
-            const SDesc dS_k = sdesc(adS, 16, 1024, 2u), dS_mn = sdesc(adS, 16384, 1024, 2u);
-            const SDesc Q_k = sdesc(aQ, 16, 1024, 2u), Q_mn = sdesc(aQ, QCHUNK, 1024, 2u);
-            const SDesc dO_k = sdesc(adO, 16, 1024, 2u), dO_mn = sdesc(adO, QCHUNK, 1024, 2u);
-            auto stage = [](SDesc d, int st) { return SDesc{d.lo + st * (QTILE >> 4), d.hi}; };
-            // k-step offsets over d: operand with 128 rows (16 KB chunks) / 64 rows (8 KB chunks)
-            auto k128 = [](int ks) -> uint32_t { return static_cast<uint32_t>(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4); };
-            auto k64 = [](int ks) -> uint32_t { return static_cast<uint32_t>(((ks >> 2) * QCHUNK + (ks & 3) * 32) >> 4); };
-            auto issue_s = [&](int it) {
-                const SDesc bq = stage(Q_k, it % STAGES);
+    } else if (warp == 9 || warp == 10) {
+        // ---------------------------------------------------------------- MMA issuers
+        // The whole warp waits; one elected lane issues a batch of MMAs and its commits.
+        constexpr uint32_t idS = idesc_bf16_f32(128, 64, 0, 0);      // S^T, dP^T
+        constexpr uint32_t idKV = idesc_bf16_f32(128, 128, 0, 1);    // dV, dK
+        constexpr uint32_t idQ = idesc_bf16_f32(128, 64, 1, 1);      // dQ^T
+        const uint32_t aK = smem_addr(sK), aV = smem_addr(sV), aQ = smem_addr(sQ),
+                       adO = smem_addr(sdO), adS = smem_addr(sdS);
+        const SDesc K_k = sdesc(aK, 16, 1024, 2u), V_k = sdesc(aV, 16, 1024, 2u);
+        const SDesc K_mn = sdesc(aK, 16384, 1024, 2u);
+        const SDesc dS_k = sdesc(adS, 16, 1024, 2u), dS_mn = sdesc(adS, 16384, 1024, 2u);
+        const SDesc Q_k = sdesc(aQ, 16, 1024, 2u), Q_mn = sdesc(aQ, QCHUNK, 1024, 2u);
+        const SDesc dO_k = sdesc(adO, 16, 1024, 2u), dO_mn = sdesc(adO, QCHUNK, 1024, 2u);
+        auto shift = [](SDesc d, int bytes) { return SDesc{d.lo + static_cast<uint32_t>(bytes >> 4), d.hi}; };
+        // k-step offsets over d: operand with 128 rows (16 KB chunks) / 64 rows (8 KB chunks)
+        auto k128 = [](int ks) -> uint32_t { return static_cast<uint32_t>(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4); };
+        auto k64 = [](int ks) -> uint32_t { return static_cast<uint32_t>(((ks >> 2) * QCHUNK + (ks & 3) * 32) >> 4); };
+        // S^T(it) and dP^T(it) into the columns of the tile's parity
+        auto issue_sdp = [&](int it) {
+            const uint32_t x = static_cast<uint32_t>(it & 1);
+            const int st = it % STAGES;
+            const SDesc bq = shift(Q_k, st * QTILE), bo = shift(dO_k, st * QTILE);
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    MMA_SS(tmem + COL_S, sdesc_at(K_k, k128(ks)), sdesc_at(bq, k64(ks)), idS, ks > 0 ? 1u : 0u);
-            };
-            auto issue_dp = [&](int it) {
-                const SDesc bo = stage(dO_k, it % STAGES);
+            for (int ks = 0; ks < 8; ++ks)
+                mma_ss(tmem + COL_S + 64 * x, sdesc_at(K_k, k128(ks)), sdesc_at(bq, k64(ks)), idS,
+                       ks > 0 ? 1u : 0u);
+            mma_commit(&bars->s_full[x]);
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    MMA_SS(tmem + COL_DP, sdesc_at(V_k, k128(ks)), sdesc_at(bo, k64(ks)), idS, ks > 0 ? 1u : 0u);
-            };
-            bool ok = NTT > 0 && bounded_wait_warp(&bars->kv_full, 0, abort, lim);
-            if (ok) ok = bounded_wait_warp(&bars->q_full[0], 0, abort, lim);
-            tc_fence_after();
-            if (ok) {
-                issue_s(0);
-                MMA_COMMIT(&bars->s_full);
-            }
-            for (int it = 0; ok && it < NTT; ++it) {
-                const int st = it % STAGES;
-                // dP^T(i): its columns were last read for dS^T(i-1), which ds_full(i-1) covered
-                issue_dp(it);
-                MMA_COMMIT(&bars->dp_full);
-                if (!(ok = bounded_wait_warp(&bars->p_full, it & 1, abort, lim))) break;
-                tc_fence_after();
-                {   // dV += P^T · dO  (P^T: queries 0-31 at S+0.., 32-63 at S+32..)
-                    const SDesc bo = stage(dO_mn, st);
-                    MMA_TS(tmem + COL_DV, tmem + COL_S, sdesc_at(bo, 0), idKV, it > 0 ? 1u : 0u);
-#pragma unroll
-                    for (int ks = 1; ks < 4; ++ks)
-                        MMA_TS(tmem + COL_DV, tmem + COL_S + (ks >> 1) * 32 + (ks & 1) * 8,
-                               sdesc_at(bo, static_cast<uint32_t>((ks * 2048) >> 4)), idKV, 1u);
-                }
-                if (it + 1 < NTT) {
-                    const int st1 = (it + 1) % STAGES;
-                    if (!(ok = bounded_wait_warp(&bars->q_full[st1], ((it + 1) / STAGES) & 1, abort, lim))) break;
-                    tc_fence_after();
-                    issue_s(it + 1);
-                    MMA_COMMIT(&bars->s_full);
-                }
-                if (!(ok = bounded_wait_warp(&bars->ds_full, it & 1, abort, lim))) break;
-                tc_fence_after();
-                {   // dK += dS^T · Q
-                    const SDesc bq = stage(Q_mn, st);
-                    MMA_SS(tmem + COL_DK, sdesc_at(dS_k, 0), sdesc_at(bq, 0), idKV, it > 0 ? 1u : 0u);
-#pragma unroll
-                    for (int ks = 1; ks < 4; ++ks)
-                        MMA_SS(tmem + COL_DK, sdesc_at(dS_k, static_cast<uint32_t>((ks * 32) >> 4)),
-                               sdesc_at(bq, static_cast<uint32_t>((ks * 2048) >> 4)), idKV, 1u);
-                }
-                const int b2 = it & 1;
-                if (it >= 2) {
-                    if (!(ok = bounded_wait_warp(&bars->dq_drained[b2], ((it - 2) >> 1) & 1, abort, lim))) break;
-                    tc_fence_after();
-                }
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)      // dQ^T = K^T · dS^T  (M = d, N = 64 queries)
-                    MMA_SS(tmem + COL_DQ + b2 * 64, sdesc_at(K_mn, static_cast<uint32_t>((ks * 2048) >> 4)),
-                           sdesc_at(dS_mn, static_cast<uint32_t>((ks * 2048) >> 4)), idQ, ks > 0 ? 1u : 0u);
-                MMA_COMMIT(&bars->dq_full[b2]);
-                MMA_COMMIT(&bars->ds_free);
-                MMA_COMMIT(&bars->q_empty[st]);
-            }
-            if (ok) MMA_COMMIT(&bars->dkv_done);
-            MMA_COMMIT(&bars->teardown);
-            drain_wait_bwd(&bars->teardown, 0, 100000000ull);
-        }
-        __syncwarp();
-    } else if (warp >= 12) {
-        // ---------------------------------------------------------------- dQ drain warpgroup
-        const int r = (warp & 3) * 32 + lane;              // head-dim row = TMEM lane
-        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const bool leader = (warp == 12);
-        uint32_t sync_phase[2] = {0, 0};
-        // Warpgroup barrier on an mbarrier with a bounded wait (no thread can hang on it).
-        auto wg_sync = [&](int s) -> bool {
-            mbar_arrive(&bars->drain_sync[s]);
-            const bool okw = bounded_wait_warp(&bars->drain_sync[s], sync_phase[s], abort, lim);
-            sync_phase[s] ^= 1;
-            return okw;
+            for (int ks = 0; ks < 8; ++ks)
+                mma_ss(tmem + COL_DP + 64 * x, sdesc_at(V_k, k128(ks)), sdesc_at(bo, k64(ks)), idS,
+                       ks > 0 ? 1u : 0u);
+            mma_commit(&bars->dp_full[x]);
         };
-        int half = 0;                                      // half tiles staged so far
+        // dV += P^T(it) · dO(it): P^T of query q at column q/2 of the tile's S^T range
+        auto issue_dv = [&](int it) {
+            const uint32_t x = static_cast<uint32_t>(it & 1);
+            const SDesc bo = shift(dO_mn, (it % STAGES) * QTILE);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_ts(tmem + COL_DV, tmem + COL_S + 64 * x + ks * 8,
+                       sdesc_at(bo, static_cast<uint32_t>((ks * 2048) >> 4)), idKV,
+                       (it > 0 || ks > 0) ? 1u : 0u);
+        };
+        // dK += dS^T(it) · Q(it); dQ^T(it) = K^T · dS^T(it) over dP^T(it)
+        auto issue_dkdq = [&](int it) {
+            const int x = it & 1, st = it % STAGES;
+            const SDesc bq = shift(Q_mn, st * QTILE);
+            const SDesc a_ds = shift(dS_k, x * DS_BYTES), b_ds = shift(dS_mn, x * DS_BYTES);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_ss(tmem + COL_DK, sdesc_at(a_ds, static_cast<uint32_t>((ks * 32) >> 4)),
+                       sdesc_at(bq, static_cast<uint32_t>((ks * 2048) >> 4)), idKV,
+                       (it > 0 || ks > 0) ? 1u : 0u);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_ss(tmem + COL_DP + 64 * x, sdesc_at(K_mn, static_cast<uint32_t>((ks * 2048) >> 4)),
+                       sdesc_at(b_ds, static_cast<uint32_t>((ks * 2048) >> 4)), idQ, ks > 0 ? 1u : 0u);
+            mma_commit(&bars->dq_full[x]);
+            mma_commit(&bars->ds_free[x]);
+            mma_commit(&bars->q_empty[st]);
+        };
+        bool ok = NTT > 0;
+        if (warp == 9) {
+            // S^T(i), dP^T(i): tile i takes the columns of tile i-2, free once the drain has read
+            // dQ^T(i-2) (which also means dV(i-2), dK(i-2) and dQ^T(i-2) are complete)
+            if (ok) ok = bounded_wait_warp(&bars->kv_full, 0, abort, lim);
+            for (int it = 0; ok && it < NTT; ++it) {
+                const int x = it & 1;
+                if (it >= 2 && !(ok = bounded_wait_warp(&bars->dq_drained[x], ((it >> 1) - 1) & 1, abort, lim)))
+                    break;
+                if (!(ok = bounded_wait_warp(&bars->q_full[it % STAGES], (it / STAGES) & 1, abort, lim)))
+                    break;
+                tc_fence_after();
+                if (elect_one()) issue_sdp(it);
+                __syncwarp();
+            }
+        } else {
+            for (int it = 0; ok && it < NTT; ++it) {
+                const int x = it & 1;
+                const uint32_t ph = static_cast<uint32_t>((it >> 1) & 1);   // tile it's phase
+                if (!(ok = bounded_wait_warp(&bars->p_full[x], ph, abort, lim))) break;
+                tc_fence_after();
+                if (elect_one()) issue_dv(it);
+                __syncwarp();
+                if (!(ok = bounded_wait_warp(&bars->ds_full[x], ph, abort, lim))) break;
+                tc_fence_after();
+                if (elect_one()) issue_dkdq(it);
+                __syncwarp();
+            }
+            if (ok && elect_one()) mma_commit(&bars->dkv_done);
+            __syncwarp();
+        }
+        if (elect_one()) mma_commit(&bars->teardown);
+        __syncwarp();
+        drain_wait_bwd(&bars->teardown, 0, 100000000ull);
+    }
+    } else if (warp >= 12) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsDrain));
+        // ---------------------------------------------------------------- dQ drain warps
+        const int w = warp & 3;                            // head-dim columns 32w .. 32w+31
+        const uint32_t lane_base = static_cast<uint32_t>(w * 32) << 16;
+        float* boxes = sStg + w * (BOXES * BOX / 4);
+        int nbox = 0;                                      // boxes this warp has issued
         bool run = true;
         volatile int* pending = nullptr;                   // semaphore still to be released
         for (int it = 0; run && it < NTT; ++it) {
-            const int b2 = it & 1;
-            if (!bounded_wait_warp(&bars->dq_full[b2], (it >> 1) & 1, abort, lim)) break;
+            const int x = it & 1;
+            if (!bounded_wait_warp(&bars->dq_full[x], (it >> 1) & 1, abort, lim)) break;
             tc_fence_after();
-            uint32_t u[64];
-            tmem_ld32(tmem + lane_base + COL_DQ + b2 * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
-            tmem_ld32(tmem + lane_base + COL_DQ + b2 * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+            uint32_t u[64];                                // lane = column 32w + lane, 64 queries
+            tmem_ld32(tmem + lane_base + COL_DP + 64 * x, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+            tmem_ld32(tmem + lane_base + COL_DP + 64 * x + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
             tmem_ld_wait();
             reg_fence<64>(u);
             tc_fence_before();
-            mbar_arrive(&bars->dq_drained[b2]);
+            mbar_arrive(&bars->dq_drained[x]);
             const int i = i_begin + it % NT;
             const int qbh = kvbh * p.kv_group + it / NT;
-            float* dst = p.dq_acc + (static_cast<size_t>(qbh) * p.n_pad + i * BQ) * D;
-            volatile int* sem = p.deterministic ? p.sems + static_cast<size_t>(qbh) * qt64 + i : nullptr;
-            bool got = true;
+            const int row0 = qbh * p.n_pad + i * BQ;       // accumulator row of the tile's query 0
+            volatile int* sem = p.deterministic
+                                    ? p.sems + (static_cast<size_t>(qbh) * qt64 + i) * 4 + w
+                                    : nullptr;
 #pragma unroll
-            for (int h = 0; h < 2; ++h, ++half) {
-                float* slot = sStg + (half % STG_SLOTS) * (STG_SLOT / 4);
-                // the reduction issued from this slot STG_SLOTS halves ago has read it
-                if (leader && lane == 0) bulk_wait_read_le2();
-                if (!wg_sync(0)) { run = false; break; }
+            for (int h = 0; h < 2; ++h, ++nbox) {
+                float* box = boxes + (nbox % BOXES) * (BOX / 4);
+                // the reduction issued from this box BOXES boxes ago has finished reading it
+                if (lane == 0) bulk_wait_read_le1();
+                __syncwarp();
 #pragma unroll
-                for (int x = 0; x < 32; ++x) slot[x * D + r] = __uint_as_float(u[h * 32 + x]);
+                for (int q = 0; q < 32; ++q) box[q * 32 + lane] = __uint_as_float(u[h * 32 + q]);
                 fence_proxy_async_smem();
-                if (!wg_sync(1)) { run = false; break; }
-                if (h == 0 && sem && leader && lane == 0) {
-                    // Contributions to one query tile are added in decreasing key-tile order,
-                    // starting from the last key tile that this query tile meets: those CTAs
-                    // began at higher query tiles and reached this one earlier, so in the steady
-                    // state nobody waits. The check sits after staging the first half, so that
-                    // staging overlaps the load.
-                    const int need = last_key_tile(mk, static_cast<long long>(i) * BQ, BQ, 128) - j;
-                    const uint64_t t0 = globaltimer_ns();
-                    while (ld_acquire_gpu(sem) < need) {   // the acquire orders the adds below
-                        if (*abort || globaltimer_ns() - t0 > lim) {
-                            *abort = 1;
-                            report_error(4);
-                            got = false;
-                            break;
+                __syncwarp();
+                if (lane == 0) {
+                    bool got = true;
+                    if (h == 0 && sem) {
+                        // the key tiles above this one that meet query tile i add first
+                        const int need = last_key_tile(mk, static_cast<long long>(i) * BQ, BQ, 128) - j;
+                        const uint64_t t0 = globaltimer_ns();
+                        while (ld_acquire_gpu(sem) < need) {   // the acquire orders the adds below
+                            if (*abort || globaltimer_ns() - t0 > lim) {
+                                *abort = 1;
+                                report_error(4);
+                                got = false;
+                                break;
+                            }
+                            __nanosleep(64);
                         }
-                        __nanosleep(64);
+                    }
+                    if (got && !*abort) {
+                        tma_reduce_add_2d(&tmAcc, box, 32 * w, row0 + 32 * h);
+                        bulk_commit();
                     }
                 }
-                if (leader && lane == 0 && got) {
-                    bulk_reduce_add_f32(dst + h * 32 * D, slot, STG_SLOT);
-                    bulk_commit();
-                }
+                __syncwarp();
+                if (*abort) { run = false; break; }
             }
-            if (sem && leader && lane == 0 && got && run) {
-                // Release the previous tile's semaphore one tile late, once its adds (not only
-                // their reads) are complete, i.e. at most this tile's two groups are pending:
-                // the drain keeps reductions in flight, and the CTAs of lower key tiles that wait
-                // on it reach that query tile two tiles after this one did.
+            if (sem && lane == 0 && run) {
+                // release the previous tile's semaphore one tile late, once its reductions (not
+                // only their reads) are complete: at most this tile's two groups are pending
                 if (pending) {
                     bulk_wait_le2_complete();
                     red_release_gpu_add(pending, 1);
                 }
                 pending = sem;
             }
-            if (*abort) break;
+            __syncwarp();
         }
-        if (leader && lane == 0) {
+        if (lane == 0) {
             bulk_wait_all();
             if (pending && !*abort) red_release_gpu_add(pending, 1);
         }
         __syncwarp();
-    } else if (warp < 8) {
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsCompute));
         // ---------------------------------------------------------------- compute warpgroups
-        const int g = warp >> 2;                           // query columns 32g .. 32g+31
+        const int x = warp >> 2;                           // query tiles of parity x
         const int r = (warp & 3) * 32 + lane;              // key row = TMEM lane
         const int kidx = j * 128 + r;
-        const int cb = g * 32;
         // queries that see key kidx: [qmin, qmax] (empty for a key past the end)
         int qmin = 1, qmax = 0;
         if (kidx < nk) {
@@ -983,93 +999,101 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
             qmax = mk.wl < 0 ? 0x7fffffff : clamp_int(kidx - mk.off + mk.wl);
         }
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + lane_base + COL_S + 64 * x;
+        const uint32_t tDP = tmem + lane_base + COL_DP + 64 * x;
+        uint8_t* ds_row = sdS + x * DS_BYTES + r * 128;
         const float sl2 = p.scale_log2;
         auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
             return __all_sync(0xffffffffu, bounded_wait(bar, par, abort, lim));
         };
-        float pr[32];
+        float pr[64];
         bool ok = true;
 
-        for (int it = 0; it < NTT; ++it) {
+        for (int it = x; it < NTT; it += 2) {
             const int i = i_begin + it % NT;
             const int st = it % STAGES;
-            const float* L2 = sL2 + st * 64 + cb;
-            const float* Dv = sDv + st * 64 + cb;
+            const uint32_t ph = static_cast<uint32_t>((it >> 1) & 1);
+            const float* L2 = sL2 + st * 64;
+            const float* Dv = sDv + st * 64;
             // ---- P^T = exp2(S^T·scale·log2e - LSE·log2e), masked; bf16 into TMEM over S^T
-            if (!(ok = wait_all(&bars->s_full, it & 1))) break;
+            if (!(ok = wait_all(&bars->s_full[x], ph))) break;
             tc_fence_after();
-            {
+            bool edge;
+            {   // every key of the tile visible to every query of the tile: no mask needed
+                long long flo, fhi;
+                visible_keys(mk, static_cast<long long>(i) * BQ + BQ - 1,
+                             static_cast<long long>(i) * BQ, flo, fhi);
+                edge = !(flo <= j * 128LL && j * 128LL + 127 <= fhi);
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
                 uint32_t u[32];
-                tmem_ld32(tmem + lane_base + COL_S + cb, u);
+                tmem_ld32(tS + 32 * h, u);
                 tmem_ld_wait();
                 reg_fence<32>(u);
-                bool edge;
-                {   // every key of the tile visible to every query of the tile: no mask needed
-                    long long flo, fhi;
-                    visible_keys(mk, static_cast<long long>(i) * BQ + BQ - 1,
-                                 static_cast<long long>(i) * BQ, flo, fhi);
-                    edge = !(flo <= j * 128LL && j * 128LL + 127 <= fhi);
-                }
 #pragma unroll
-                for (int x = 0; x < 32; x += 4) {
-                    const float4 l4 = *reinterpret_cast<const float4*>(L2 + x);
-                    pr[x] = ex2_approx(fmaf(__uint_as_float(u[x]), sl2, -l4.x));
-                    pr[x + 1] = ex2_approx(fmaf(__uint_as_float(u[x + 1]), sl2, -l4.y));
-                    pr[x + 2] = ex2_approx(fmaf(__uint_as_float(u[x + 2]), sl2, -l4.z));
-                    pr[x + 3] = ex2_approx(fmaf(__uint_as_float(u[x + 3]), sl2, -l4.w));
+                for (int c = 0; c < 32; c += 4) {
+                    const float4 l4 = *reinterpret_cast<const float4*>(L2 + 32 * h + c);
+                    pr[32 * h + c] = ex2_approx(fmaf(__uint_as_float(u[c]), sl2, -l4.x));
+                    pr[32 * h + c + 1] = ex2_approx(fmaf(__uint_as_float(u[c + 1]), sl2, -l4.y));
+                    pr[32 * h + c + 2] = ex2_approx(fmaf(__uint_as_float(u[c + 2]), sl2, -l4.z));
+                    pr[32 * h + c + 3] = ex2_approx(fmaf(__uint_as_float(u[c + 3]), sl2, -l4.w));
                 }
-                if (edge) {
-                    const int q0 = i * BQ + cb;
+            }
+            if (edge) {
+                const int q0 = i * BQ;
 #pragma unroll
-                    for (int x = 0; x < 32; ++x)
-                        if (q0 + x < qmin || q0 + x > qmax) pr[x] = 0.f;
-                }
-                uint32_t w[16];
+                for (int c = 0; c < 64; ++c)
+                    if (q0 + c < qmin || q0 + c > qmax) pr[c] = 0.f;
+            }
+            {
+                uint32_t w[32];
 #pragma unroll
-                for (int x = 0; x < 16; ++x) w[x] = pack_bf16x2(pr[2 * x], pr[2 * x + 1]);
-                tmem_st16(tmem + lane_base + COL_S + cb, w);
+                for (int c = 0; c < 32; ++c) w[c] = pack_bf16x2(pr[2 * c], pr[2 * c + 1]);
+                tmem_st32(tS, w);                          // query q at column q/2
                 tmem_st_wait();
             }
             tc_fence_before();
-            mbar_arrive(&bars->p_full);
+            mbar_arrive(&bars->p_full[x]);
             // ---- dS^T = P^T ∘ (dP^T - D) -> bf16 into shared memory (row r, swizzled)
-            if (!(ok = wait_all(&bars->dp_full, it & 1))) break;
-            if (it > 0 && !(ok = wait_all(&bars->ds_free, (it - 1) & 1))) break;
+            if (!(ok = wait_all(&bars->dp_full[x], ph))) break;
+            if (it >= 2 && !(ok = wait_all(&bars->ds_free[x], ph ^ 1u))) break;
             tc_fence_after();
-            {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
                 uint32_t u[32];
-                tmem_ld32(tmem + lane_base + COL_DP + cb, u);
+                tmem_ld32(tDP + 32 * h, u);
                 tmem_ld_wait();
                 reg_fence<32>(u);
                 uint32_t w[16];
 #pragma unroll
-                for (int x = 0; x < 16; x += 2) {
-                    const float4 d4 = *reinterpret_cast<const float4*>(Dv + 2 * x);
-                    w[x] = pack_bf16x2(pr[2 * x] * (__uint_as_float(u[2 * x]) - d4.x),
-                                       pr[2 * x + 1] * (__uint_as_float(u[2 * x + 1]) - d4.y));
-                    w[x + 1] = pack_bf16x2(pr[2 * x + 2] * (__uint_as_float(u[2 * x + 2]) - d4.z),
-                                           pr[2 * x + 3] * (__uint_as_float(u[2 * x + 3]) - d4.w));
+                for (int c = 0; c < 16; c += 2) {
+                    const float4 d4 = *reinterpret_cast<const float4*>(Dv + 32 * h + 2 * c);
+                    w[c] = pack_bf16x2(pr[32 * h + 2 * c] * (__uint_as_float(u[2 * c]) - d4.x),
+                                       pr[32 * h + 2 * c + 1] * (__uint_as_float(u[2 * c + 1]) - d4.y));
+                    w[c + 1] = pack_bf16x2(pr[32 * h + 2 * c + 2] * (__uint_as_float(u[2 * c + 2]) - d4.z),
+                                           pr[32 * h + 2 * c + 3] * (__uint_as_float(u[2 * c + 3]) - d4.w));
                 }
-                uint8_t* ds_row = sdS + r * 128;
 #pragma unroll
                 for (int t = 0; t < 4; ++t) {
-                    const int unit = g * 4 + t;
+                    const int unit = 4 * h + t;                // queries 8·unit .. 8·unit+7
                     *reinterpret_cast<uint4*>(ds_row + ((unit ^ (r & 7)) << 4)) =
                         make_uint4(w[4 * t], w[4 * t + 1], w[4 * t + 2], w[4 * t + 3]);
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(&bars->ds_full);
+            mbar_arrive(&bars->ds_full[x]);
         }
+        // ---- epilogue: warpgroup x writes head-dim columns 64x .. 64x+63 of dV and dK
         if (ok && NTT == 0) {
             // no query sees these keys: dK = dV = 0
             if (kidx < nk) {
-                const size_t orow = (static_cast<size_t>(kvbh) * nk + kidx) * D + g * 64;
+                const size_t orow = (static_cast<size_t>(kvbh) * nk + kidx) * D + x * 64;
 #pragma unroll
-                for (int x = 0; x < 8; ++x) {
-                    reinterpret_cast<uint4*>(p.dk + orow)[x] = make_uint4(0u, 0u, 0u, 0u);
-                    reinterpret_cast<uint4*>(p.dv + orow)[x] = make_uint4(0u, 0u, 0u, 0u);
+                for (int c = 0; c < 8; ++c) {
+                    reinterpret_cast<uint4*>(p.dk + orow)[c] = make_uint4(0u, 0u, 0u, 0u);
+                    reinterpret_cast<uint4*>(p.dv + orow)[c] = make_uint4(0u, 0u, 0u, 0u);
                 }
             }
             ok = false;
@@ -1077,10 +1101,10 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
         if (ok) ok = wait_all(&bars->dkv_done, 0);
         if (ok) {
             tc_fence_after();
-            const size_t orow = (static_cast<size_t>(kvbh) * nk + kidx) * D + g * 64;
+            const size_t orow = (static_cast<size_t>(kvbh) * nk + kidx) * D + x * 64;
 #pragma unroll 1
             for (int which = 0; which < 2; ++which) {
-                const uint32_t tacc = tmem + lane_base + (which == 0 ? COL_DV : COL_DK) + g * 64;
+                const uint32_t tacc = tmem + lane_base + (which == 0 ? COL_DV : COL_DK) + x * 64;
                 const float mul = which == 0 ? 1.f : p.scale;
                 __nv_bfloat16* dst = (which == 0 ? p.dv : p.dk) + orow;
 #pragma unroll 1
@@ -1091,14 +1115,14 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
                     reg_fence<32>(u);
                     uint32_t w[16];
 #pragma unroll
-                    for (int x = 0; x < 16; ++x)
-                        w[x] = pack_bf16x2(__uint_as_float(u[2 * x]) * mul,
-                                           __uint_as_float(u[2 * x + 1]) * mul);
+                    for (int c = 0; c < 16; ++c)
+                        w[c] = pack_bf16x2(__uint_as_float(u[2 * c]) * mul,
+                                           __uint_as_float(u[2 * c + 1]) * mul);
                     if (kidx < nk) {
                         uint4* o = reinterpret_cast<uint4*>(dst + cc);
 #pragma unroll
-                        for (int x = 0; x < 4; ++x)
-                            o[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
+                        for (int c = 0; c < 4; ++c)
+                            o[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
                     }
                 }
             }
@@ -1140,7 +1164,7 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
         const int rpw = 32 / (D / 8);
         long long blocks = (rows + (8 * rpw) - 1) / (8 * rpw);
         if (blocks > 148 * 16) blocks = 148 * 16;
-        const int n_sems = a.deterministic ? BH * (n_pad / 64) : 0;
+        const int n_sems = a.deterministic ? BH * (n_pad / 64) * 4 : 0;
         bwd_preprocess_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
             static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dO), a.lse,
             a.L2vec, a.Dvec, a.dq_acc, a.deterministic ? a.sems : nullptr, a.nq, n_pad, rows,
@@ -1175,12 +1199,15 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
     if ((e = make_tmap_bf16(&mv, a.v, BHkv, a.nk, D)) != cudaSuccess) return e;
     if ((e = make_tmap_bf16(&mdo, a.dO, BH, a.nq, D, qbox)) != cudaSuccess) return e;
     if constexpr (D == 128) {
+        CUtensorMap macc;   // the fp32 dQ accumulator as (B·H·n_pad) rows x 128 columns
+        if ((e = make_tmap_acc(&macc, a.dq_acc, static_cast<long long>(BH) * n_pad, D)) != cudaSuccess)
+            return e;
         e = cudaFuncSetAttribute(bwd_main_q64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  q64::SMEM);
         if (e != cudaSuccess) return e;
         if (ev && ev[1] && (e = cudaEventRecord(ev[1], stream)) != cudaSuccess) return e;
         bwd_main_q64_kernel<<<static_cast<unsigned>(grid), q64::kThreads, q64::SMEM, stream>>>(
-            mq, mk, mv, mdo, kp);
+            mq, mk, mv, mdo, macc, kp);
     } else {
         e = cudaFuncSetAttribute(bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  C::SMEM);

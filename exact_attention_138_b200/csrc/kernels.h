@@ -107,7 +107,7 @@ struct BwdArgs {
     float* L2vec;     // workspace: B*H*n_pad, LSE_i·log2(e) (+inf on padding rows and on rows
                       // that see no key)
     float* dq_acc;    // workspace: B*H*n_pad*d
-    int* sems;        // workspace: B*H*(n_pad/64), deterministic mode only
+    int* sems;        // workspace: B*H*(n_pad/64)*4, deterministic mode only
     uint64_t timeout_ns;
     const cudaEvent_t* phase_events;   // 4 events or nullptr (measurement hook)
 };
@@ -121,6 +121,10 @@ inline cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int BH, in
                                   int box_rows = 128) {
     return make_tmap(map, base, 2, BH, n, d, box_rows);
 }
+
+// Encodes a 2-D tensor map over the fp32 dQ accumulator: `rows` rows of `d` fp32 values, box of
+// 32 rows x 32 columns, no swizzle (the backward's drain adds [32 queries][32 columns] boxes).
+cudaError_t make_tmap_acc(CUtensorMap* map, float* base, long long rows, int d);
 
 cudaError_t launch_fwd_bf16(const FwdArgs& a, cudaStream_t stream);
 cudaError_t launch_fwd_f32(const FwdArgs& a, cudaStream_t stream);

@@ -138,6 +138,16 @@ __device__ __forceinline__ void bulk_reduce_add_f32(float* dst, const void* src,
                  "r"(smem_addr(src)), "r"(bytes)
                  : "memory");
 }
+// Tiled tensor reduction shared -> global: the box at (c0, c1) of `map` += the box in shared
+// memory (fp32 add, done by the TMA unit; tracked by the bulk async-groups like bulk reductions).
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, const void* src, int c0,
+                                                  int c1) {
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];"
+        ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(src)), "r"(c0), "r"(c1)
+        : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

@@ -107,7 +107,7 @@ int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* ls
 /* Bytes of device workspace attn_bwd needs for these sizes: the D vector and the LSE·log2(e)
  * vector (B·H·n fp32 each, padded per head to a multiple of 128 rows) and the fp32 dQ accumulator
  * (B·H·n·d fp32, padded the same way), each rounded up to 256 bytes; with deterministic != 0 also
- * one int semaphore per 64 query rows. */
+ * four int semaphores per 64 query rows. */
 size_t attn_bwd_workspace_bytes(int B, int H, int n, int d, int deterministic);
 
 /* Masked and cross-length attention. Sliding window: "Attention Mechanism: Revolusi
