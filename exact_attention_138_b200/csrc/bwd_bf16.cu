@@ -295,17 +295,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
     } else if (warp == 9) {
         // ---------------------------------------------------------------- MMA issuer
-        // The whole warp runs this loop (warp-uniform state); one elected lane issues.
+        // The whole warp runs this loop (warp-uniform state) and waits together; one elected lane
+        // issues each batch of MMAs with its commits (a warp vote per tcgen05.mma would cost the
+        // issuing warp ~100 cycles per instruction).
         {
             auto vss = [](uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
-                if (elect_one()) mma_ss(d, a, b, id, acc);
+                mma_ss(d, a, b, id, acc);
             };
             auto vts = [](uint32_t d, uint32_t a, uint64_t b, uint32_t id, uint32_t acc) {
-                if (elect_one()) mma_ts(d, a, b, id, acc);
+                mma_ts(d, a, b, id, acc);
             };
-            auto vcommit = [](uint64_t* bar) {
-                if (elect_one()) mma_commit(bar);
-            };
+            auto vcommit = [](uint64_t* bar) { mma_commit(bar); };
             constexpr uint32_t idSS = idesc_bf16_f32(128, 128, 0, 0);    // K-major x K-major
             constexpr uint32_t idKN = idesc_bf16_f32(128, D, 0, 1);      // A K-major, B MN-major
             constexpr uint32_t idDQ = idesc_bf16_f32(128, D, 1, 1);      // dQ = dS · K    // dQ
@@ -347,16 +347,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (ok) ok = bounded_wait_warp(&bars->q_full[0], 0, abort, lim);
             tc_fence_after();
             if (ok) {
-                issue_s(0);
-                vcommit(&bars->s_full);
-                issue_dp(0);
-                vcommit(&bars->dp_full);
+                if (elect_one()) {
+                    issue_s(0);
+                    vcommit(&bars->s_full);
+                    issue_dp(0);
+                    vcommit(&bars->dp_full);
+                }
+                __syncwarp();
             }
             for (int it = 0; ok && it < NTT; ++it) {
                 const int st = it & 1;
                 if (!(ok = bounded_wait_warp(&bars->p_full, it & 1, abort, lim))) break;
                 tc_fence_after();
-                {   // dV_j += P^T · dO_i   (P^T in TMEM: queries 0-63 at S+0.., 64-127 at S+64..)
+                if (elect_one()) {   // dV_j += P^T · dO_i   (P^T in TMEM: queries 0-63 at S+0.., 64-127 at S+64..)
                     const SDesc bo = stage(dO_mn, st);
                     vts(tmem + COL_DV, tmem + COL_S, sdesc_at(bo, 0), idKN, it > 0 ? 1u : 0u);
 #pragma unroll
@@ -364,17 +367,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         vts(tmem + COL_DV, tmem + COL_S + (ks >> 2) * 64 + (ks & 3) * 8,
                                sdesc_at(bo, roff(ks)), idKN, 1u);
                 }
+                __syncwarp();
                 if (it + 1 < NTT) {
                     if (!(ok = bounded_wait_warp(&bars->q_full[(it + 1) & 1], ((it + 1) >> 1) & 1,
                                             abort, lim)))
                         break;
                     tc_fence_after();
-                    issue_s(it + 1);
-                    vcommit(&bars->s_full);
+                    if (elect_one()) {
+                        issue_s(it + 1);
+                        vcommit(&bars->s_full);
+                    }
+                    __syncwarp();
                 }
                 if (!(ok = bounded_wait_warp(&bars->ds_full, it & 1, abort, lim))) break;
                 tc_fence_after();
-                {   // dK_j += dS^T · Q_i   (A = dS^T K-major, B = Q_i MN-major)
+                if (elect_one()) {   // dK_j += dS^T · Q_i   (A = dS^T K-major, B = Q_i MN-major)
                     const SDesc bq = stage(Q_mn, st);
                     vss(tmem + COL_DK, sdesc_at(dS_k, 0), sdesc_at(bq, 0), idKN, it > 0 ? 1u : 0u);
 #pragma unroll
@@ -383,30 +390,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                sdesc_at(dS_k, static_cast<uint32_t>(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4)),
                                sdesc_at(bq, roff(ks)), idKN, 1u);
                 }
+                __syncwarp();
                 // dQ_i = dS · K_j into buffer it mod 2, once the partial of tile it-2 is drained
                 const int b2 = it & 1;
                 if (it >= 2) {
                     if (!(ok = bounded_wait_warp(&bars->dq_drained[b2], ((it - 2) >> 1) & 1, abort, lim))) break;
                     tc_fence_after();
                 }
+                if (elect_one()) {
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint64_t kd = sdesc_at(K_mn, roff(ks));
-                    const uint64_t sd = sdesc_at(dS_mn, static_cast<uint32_t>((ks * 2048) >> 4));
-                    vss(tmem + COL_DQ + b2 * 64, sd, kd, idDQ, ks > 0 ? 1u : 0u);
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint64_t kd = sdesc_at(K_mn, roff(ks));
+                        const uint64_t sd = sdesc_at(dS_mn, static_cast<uint32_t>((ks * 2048) >> 4));
+                        vss(tmem + COL_DQ + b2 * 64, sd, kd, idDQ, ks > 0 ? 1u : 0u);
+                    }
+                    vcommit(&bars->dq_full[b2]);
+                    vcommit(&bars->ds_free);
+                    vcommit(&bars->q_empty[st]);
+                    // dP^T(i+1): its columns were last read for dS^T(i) (ds_full(i)), and dO(i+1)
+                    // arrived before S^T(i+1)
+                    if (it + 1 < NTT) {
+                        issue_dp(it + 1);
+                        vcommit(&bars->dp_full);
+                    }
                 }
-                vcommit(&bars->dq_full[b2]);
-                vcommit(&bars->ds_free);
-                vcommit(&bars->q_empty[st]);
-                // dP^T(i+1): its columns were last read for dS^T(i) (ds_full(i)), and dO(i+1)
-                // arrived before S^T(i+1)
-                if (it + 1 < NTT) {
-                    issue_dp(it + 1);
-                    vcommit(&bars->dp_full);
-                }
+                __syncwarp();
             }
-            if (ok) vcommit(&bars->dkv_done);
-            vcommit(&bars->teardown);
+            if (elect_one()) {
+                if (ok) vcommit(&bars->dkv_done);
+                vcommit(&bars->teardown);
+            }
+            __syncwarp();
             drain_wait_bwd(&bars->teardown, 0, 100000000ull);
         }
         __syncwarp();

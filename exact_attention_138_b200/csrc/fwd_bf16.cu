@@ -259,21 +259,20 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap* tmQ_, const CUtensor
         }
     } else if (warp == 9) {
         // ---------------------------------------------------------------- MMA issuer
-        // The whole warp runs this loop (warp-uniform state); one elected lane issues.
+        // The whole warp runs this loop (warp-uniform state) and waits together; one elected
+        // lane issues each batch of MMAs with its commit. (A vote per instruction would cost the
+        // issuing warp ~100 cycles per tcgen05.mma, more than the tensor pipe needs for one.)
         {
             constexpr uint32_t idS = F8 ? idesc_e4m3_f32(128, 128, 0, 0) : idesc_bf16_f32(128, 128, 0, 0);
             constexpr uint32_t idPV = F8 ? idesc_e4m3_f32(128, D, 0, 1) : idesc_bf16_f32(128, D, 0, 1);
+            // issue helpers: called by the elected lane only
             auto mss = [](uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
-                if (elect_one()) {
-                    if constexpr (F8) mma_ss_f8(d, a, b, id, acc);
-                    else mma_ss(d, a, b, id, acc);
-                }
+                if constexpr (F8) mma_ss_f8(d, a, b, id, acc);
+                else mma_ss(d, a, b, id, acc);
             };
             auto mts = [](uint32_t d, uint32_t a, uint64_t b, uint32_t id, uint32_t acc) {
-                if (elect_one()) {
-                    if constexpr (F8) mma_ts_f8(d, a, b, id, acc);
-                    else mma_ts(d, a, b, id, acc);
-                }
+                if constexpr (F8) mma_ts_f8(d, a, b, id, acc);
+                else mma_ts(d, a, b, id, acc);
             };
             const uint32_t sQa = smem_addr(sQ), sKa = smem_addr(sK), sVa = smem_addr(sV);
             bool ok = U > 0 && bounded_wait_warp(&bars->q_full, 0, abort, lim);
@@ -291,16 +290,16 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap* tmQ_, const CUtensor
             // Lean issue path: descriptors per operand tile computed once, each k-step adds a
             // constant to the low word, loops fully unrolled. The issuing lane shares its SM
             // sub-partition with two busy softmax warps, so every instruction here costs.
-            SDesc dQ[2], dK[C::STAGES], dV[C::STAGES];
-#pragma unroll
-            for (int g = 0; g < 2; ++g) dQ[g] = sdesc(sQa + g * C::TILE, 16, 8 * C::SWB, C::SWZ);
-#pragma unroll
-            for (int st = 0; st < C::STAGES; ++st) {
-                dK[st] = sdesc(sKa + st * C::TILE, 16, 8 * C::SWB, C::SWZ);
-                dV[st] = sdesc(sVa + st * C::TILE, C::CHUNK, 8 * C::SWB, C::SWZ);
-            }
+            // (tile offsets are added to the start-address field: no descriptor arrays, so no
+            // local-memory indexing on the issue path)
+            const SDesc dQ0 = sdesc(sQa, 16, 8 * C::SWB, C::SWZ);
+            const SDesc dK0 = sdesc(sKa, 16, 8 * C::SWB, C::SWZ);
+            const SDesc dV0 = sdesc(sVa, C::CHUNK, 8 * C::SWB, C::SWZ);
+            auto tile_of = [](SDesc d, int idx) {
+                return SDesc{d.lo + static_cast<uint32_t>(idx) * (C::TILE >> 4), d.hi};
+            };
             auto issue_s = [&](int g, int u) {
-                const SDesc a = dQ[g], b = dK[u % C::STAGES];
+                const SDesc a = tile_of(dQ0, g), b = tile_of(dK0, u % C::STAGES);
                 const uint32_t d = tmem + 256 + g * 128;
 #pragma unroll
                 for (int ks = 0; ks < D / C::KSTEP; ++ks) {
@@ -310,7 +309,7 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap* tmQ_, const CUtensor
                 }
             };
             auto issue_pv = [&](int g, int u, bool accumulate) {
-                const SDesc b = dV[u % C::STAGES];
+                const SDesc b = tile_of(dV0, u % C::STAGES);
                 const uint32_t d = tmem + g * 128, a = tmem + 256 + g * 128;
                 // one instruction takes KSTEP keys: 8 TMEM columns of P, KSTEP rows of V
                 mts(d, a, sdesc_at(b, 0), idPV, accumulate ? 1u : 0u);
@@ -327,12 +326,15 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap* tmQ_, const CUtensor
             auto active = [&](int g, int u) { return T[g] > 0 && u >= s0[g] && u < s0[g] + T[g]; };
             if (ok) ok = wait_k(0);
             if (ok) {
-                for (int g = 0; g < 2; ++g)
-                    if (T[g] > 0 && s0[g] == 0) {
-                        issue_s(g, 0);
-                        FMMA_COMMIT(&bars->s_full[g]);
-                    }
-                FMMA_COMMIT(&bars->k_empty[0]);
+                if (elect_one()) {
+                    for (int g = 0; g < 2; ++g)
+                        if (T[g] > 0 && s0[g] == 0) {
+                            issue_s(g, 0);
+                            mma_commit(&bars->s_full[g]);
+                        }
+                    mma_commit(&bars->k_empty[0]);
+                }
+                __syncwarp();
             }
             for (int u = 0; ok && u < U; ++u) {
                 bool v_ready = false;
@@ -351,13 +353,19 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap* tmQ_, const CUtensor
                     if (!bounded_wait_warp(&bars->p_full[g], t & 1, abort, lim)) { ok = false; break; }
                     tc_fence_after();
                     if (!wait_v()) { ok = false; break; }
-                    issue_pv(g, u, t > 0);
-                    if (t + 1 < T[g]) {
+                    const bool more = t + 1 < T[g];
+                    if (elect_one()) {
+                        issue_pv(g, u, t > 0);
+                        if (!more) mma_commit(&bars->o_done[g]);
+                    }
+                    __syncwarp();
+                    if (more) {
                         if (!wait_k(u + 1)) { ok = false; break; }
-                        issue_s(g, u + 1);
-                        FMMA_COMMIT(&bars->s_full[g]);
-                    } else {
-                        FMMA_COMMIT(&bars->o_done[g]);
+                        if (elect_one()) {
+                            issue_s(g, u + 1);
+                            mma_commit(&bars->s_full[g]);
+                        }
+                        __syncwarp();
                     }
                 }
                 if (!ok) break;
@@ -365,8 +373,11 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap* tmQ_, const CUtensor
                     for (int g = 0; g < 2 && ok; ++g)
                         if (T[g] > 0 && s0[g] == u + 1) {      // first tile of g is the next one
                             if (!wait_k(u + 1)) { ok = false; break; }
-                            issue_s(g, u + 1);
-                            FMMA_COMMIT(&bars->s_full[g]);
+                            if (elect_one()) {
+                                issue_s(g, u + 1);
+                                mma_commit(&bars->s_full[g]);
+                            }
+                            __syncwarp();
                         }
                     if (!ok || !(ok = wait_k(u + 1))) break;
                 }
