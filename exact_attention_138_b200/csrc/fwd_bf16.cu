@@ -67,7 +67,7 @@ struct FwdCfg {
 struct FwdBars {
     uint64_t q_full;
     uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
-    uint64_t s_full[2], p_full[2], o_done[2];
+    uint64_t s_full[2], p_half[2], p_full[2], o_done[2];
     uint64_t teardown;
     uint32_t tmem_base;
     int abort;
@@ -193,6 +193,7 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap* tmQ_, const CUtensor
         }
         for (int g = 0; g < 2; ++g) {
             mbar_init(&bars->s_full[g], 1);
+            mbar_init(&bars->p_half[g], 128);
             mbar_init(&bars->p_full[g], 128);
             mbar_init(&bars->o_done[g], 1);
         }
@@ -308,15 +309,17 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap* tmQ_, const CUtensor
                     mss(d, sdesc_at(a, off), sdesc_at(b, off), idS, ks > 0 ? 1u : 0u);
                 }
             };
-            auto issue_pv = [&](int g, int u, bool accumulate) {
+            // O += P·V over keys [64·half, 64·half + 64) of the tile
+            auto issue_pv = [&](int g, int u, int half, bool accumulate) {
                 const SDesc b = tile_of(dV0, u % C::STAGES);
                 const uint32_t d = tmem + g * 128, a = tmem + 256 + g * 128;
+                constexpr int KH = C::BN / C::KSTEP / 2;   // instructions per half
                 // one instruction takes KSTEP keys: 8 TMEM columns of P, KSTEP rows of V
-                mts(d, a, sdesc_at(b, 0), idPV, accumulate ? 1u : 0u);
 #pragma unroll
-                for (int ks = 1; ks < C::BN / C::KSTEP; ++ks)
+                for (int ks = half * KH; ks < half * KH + KH; ++ks)
                     mts(d, a + ks * 8,
-                        sdesc_at(b, static_cast<uint32_t>((ks * C::KSTEP * C::SWB) >> 4)), idPV, 1u);
+                        sdesc_at(b, static_cast<uint32_t>((ks * C::KSTEP * C::SWB) >> 4)), idPV,
+                        (accumulate || ks > 0) ? 1u : 0u);
             };
             // Stream step u holds key tile Jmin + u. Query tile g uses steps [J0[g] - Jmin,
             // J0[g] - Jmin + T[g]); its S for step u+1 is issued during step u (or, for its first
@@ -350,12 +353,18 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap* tmQ_, const CUtensor
                 for (int g = 0; g < 2 && ok; ++g) {
                     if (!active(g, u)) continue;
                     const int t = u - s0[g];
-                    if (!bounded_wait_warp(&bars->p_full[g], t & 1, abort, lim)) { ok = false; break; }
+                    // the softmax hands over P in two halves of 64 keys: the first half's P·V
+                    // runs while the second half's exponentials are computed
+                    if (!bounded_wait_warp(&bars->p_half[g], t & 1, abort, lim)) { ok = false; break; }
                     tc_fence_after();
                     if (!wait_v()) { ok = false; break; }
+                    if (elect_one()) issue_pv(g, u, 0, t > 0);
+                    __syncwarp();
+                    if (!bounded_wait_warp(&bars->p_full[g], t & 1, abort, lim)) { ok = false; break; }
+                    tc_fence_after();
                     const bool more = t + 1 < T[g];
                     if (elect_one()) {
-                        issue_pv(g, u, t > 0);
+                        issue_pv(g, u, 1, true);
                         if (!more) mma_commit(&bars->o_done[g]);
                     }
                     __syncwarp();
@@ -481,29 +490,35 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap* tmQ_, const CUtensor
             const uint64_t nm2 = f2_pack(-m_use, -m_use);
             uint64_t rsa = f2_pack(0.f, 0.f), rsb = f2_pack(0.f, 0.f);
             // P = exp2(s·c - m) on the MUFU (masked -inf scores give exact zeros), two row-sum
-            // accumulators to shorten the add chain
+            // accumulators to shorten the add chain. P goes to TMEM in two halves of 64 keys
+            // (32 columns of bf16 pairs or 16 of E4M3 quadruples each), the first signalled as
+            // soon as it is stored so that its P·V overlaps the second half's exponentials.
+            constexpr int PW = F8 ? 16 : 32;                // P words per half
 #pragma unroll
-            for (int c = 0; c < 128; c += 2) {
-                float x0, x1;
-                f2_unpack(f2_fma(f2_pack(__uint_as_float(u[c]), __uint_as_float(u[c + 1])),
-                                 sl2x2, nm2), x0, x1);
-                const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-                if (c & 2) rsb = f2_add(rsb, f2_pack(p0, p1));
-                else rsa = f2_add(rsa, f2_pack(p0, p1));
-                store_p<F8>(u, c, p0, p1);
+            for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+                for (int c = 64 * hh; c < 64 * hh + 64; c += 2) {
+                    float x0, x1;
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(u[c]), __uint_as_float(u[c + 1])),
+                                     sl2x2, nm2), x0, x1);
+                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                    if (c & 2) rsb = f2_add(rsb, f2_pack(p0, p1));
+                    else rsa = f2_add(rsa, f2_pack(p0, p1));
+                    store_p<F8>(u, c, p0, p1);
+                }
+                if constexpr (F8)
+                    tmem_st16(tS + hh * PW, *reinterpret_cast<uint32_t(*)[16]>(&u[hh * PW]));
+                else
+                    tmem_st32(tS + hh * PW, *reinterpret_cast<uint32_t(*)[32]>(&u[hh * PW]));
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(hh == 0 ? &bars->p_half[g] : &bars->p_full[g]);
             }
             float ra0, ra1, rb0, rb1;
             f2_unpack(rsa, ra0, ra1);
             f2_unpack(rsb, rb0, rb1);
             const float rs0 = ra0 + rb0, rs1 = ra1 + rb1;
             l += rs0 + rs1;
-            // P: 64 columns of bf16 pairs, or 32 columns of E4M3 quadruples
-#pragma unroll
-            for (int h = 0; h < (F8 ? 1 : 2); ++h)
-                tmem_st32(tS + h * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[h * 32]));
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&bars->p_full[g]);
         }
         if constexpr (SPLIT) {
             // Partial of this share: unnormalised O (fp32, rows padded to D + 4 floats) and
