@@ -46,18 +46,40 @@ def rank_chunks(rank: int, world: int, zigzag: bool):
 
 
 class CudaOps:
-    """The per-chunk-pair operations, all in libattn.so."""
+    """The per-chunk-pair operations, all in libattn.so. One set of per-hop output buffers and one
+    backward workspace are kept and reused by every hop of a ring pass (each hop's partials are
+    folded into the running results on the same stream before the next hop overwrites them)."""
 
     def __init__(self):
         import exact_attention_138_b200 as ea
         self.ea = ea
+        self._bufs = {}
+
+    def _buf(self, key, shape, dtype, device):
+        t = self._bufs.get(key)
+        if t is None or tuple(t.shape) != tuple(shape) or t.dtype != dtype or t.device != device:
+            t = torch.empty(shape, dtype=dtype, device=device)
+            self._bufs[key] = t
+        return t
 
     def fwd(self, q, k, v, scale, window):
-        return self.ea.forward(q, k, v, scale=scale, window=window)
+        o = self._buf("o", q.shape, q.dtype, q.device)
+        lse = self._buf("lse", q.shape[:-1], torch.float32, q.device)
+        return self.ea.forward(q, k, v, scale=scale, window=window, out=o, lse=lse)
 
     def bwd(self, q, k, v, o, do, lse, scale, window, deterministic):
-        return self.ea.backward(q, k, v, o, do, lse, scale=scale, window=window,
-                                deterministic=deterministic)
+        """(dQ partial, dK and dV partials stacked as one (2, B, Hkv, n, d) tensor)."""
+        B, H, n, d = q.shape
+        dq = self._buf("dq", q.shape, q.dtype, q.device)
+        dkv = self._buf("dkv", (2,) + tuple(k.shape), k.dtype, k.device)
+        need = self.ea.attn_bwd_workspace_bytes(B, H, n, d, int(bool(deterministic)))
+        ws = self._bufs.get("ws")
+        if ws is None or ws.numel() < need or ws.device != q.device:
+            ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+            self._bufs["ws"] = ws
+        self.ea.backward(q, k, v, o, do, lse, scale=scale, window=window,
+                         deterministic=deterministic, dq=dq, dk=dkv[0], dv=dkv[1], workspace=ws)
+        return dq, dkv
 
     def merge(self, o_acc, lse_acc, o_part, lse_part, first, out):
         self.ea.ring_merge(o_acc, lse_acc, o_part, lse_part, first=first, out=out)
@@ -116,10 +138,9 @@ def _bwd_hop(ops, dq_acc, qs, q_ids, os_, dos, lses, kvs, kv_ids, dkv_acc, causa
             w = hop_window(q_ids[qi], kv_ids[ki], causal)
             if w is None:
                 continue
-            dq_p, dk_p, dv_p = ops.bwd(q, k, v, os_[qi], dos[qi], lses[qi], scale, w, det)
+            dq_p, dkv_p = ops.bwd(q, k, v, os_[qi], dos[qi], lses[qi], scale, w, det)
             ops.accumulate(dq_acc[qi], dq_p, False, None)
-            ops.accumulate(dkv_acc[ki][0], dk_p, False, None)
-            ops.accumulate(dkv_acc[ki][1], dv_p, False, None)
+            ops.accumulate(dkv_acc[ki], dkv_p, False, None)      # dK and dV in one pass
 
 
 def _convert(ops, accs, likes):
@@ -187,15 +208,15 @@ def ring_backward(q, k, v, o, do, lse, causal=False, scale=None, group=None, ops
     dq_acc = [torch.zeros(c.shape, dtype=torch.float32, device=c.device) for c in qs]
     ks, vs = _split(k, parts), _split(v, parts)
     cur = ks + vs
-    acc = [torch.zeros(c.shape, dtype=torch.float32, device=c.device) for c in ks + vs]
+    # per K/V chunk: its dK and dV accumulators stacked, (2, B, Hkv, chunk, d) fp32
+    acc = [torch.zeros((2,) + tuple(c.shape), dtype=torch.float32, device=c.device) for c in ks]
     for r in range(world):
         reqs = None
         if r < world - 1:
             nxt_kv, reqs = _exchange(cur, nxt, prv, group)
         kv_ids = rank_chunks((rank - r) % world, world, zigzag)
         kvs = list(zip(cur[:parts], cur[parts:]))
-        dkv = list(zip(acc[:parts], acc[parts:]))
-        _bwd_hop(ops, dq_acc, qs, q_ids, os_, dos, lses, kvs, kv_ids, dkv, causal, scale,
+        _bwd_hop(ops, dq_acc, qs, q_ids, os_, dos, lses, kvs, kv_ids, acc, causal, scale,
                  deterministic)
         # the dK / dV accumulators travel on with their chunks; after the last hop each rank
         # holds its own chunks'
@@ -205,8 +226,8 @@ def ring_backward(q, k, v, o, do, lse, causal=False, scale=None, group=None, ops
         if reqs is not None:
             cur = nxt_kv
         acc = nxt_acc
-    return (_convert(ops, dq_acc, qs), _convert(ops, acc[:parts], ks),
-            _convert(ops, acc[parts:], vs))
+    return (_convert(ops, dq_acc, qs), _convert(ops, [a[0] for a in acc], ks),
+            _convert(ops, [a[1] for a in acc], vs))
 
 
 def ring_forward_emulated(qs, ks, vs, causal=False, scale=None, ops=None, zigzag=False):
@@ -242,9 +263,8 @@ def ring_backward_emulated(qs, ks, vs, os_, dos, lses, causal=False, scale=None,
     kv_chunks = [list(zip(_split(k, parts), _split(v, parts))) for k, v in zip(ks, vs)]
     dq_acc = [[torch.zeros(c.shape, dtype=torch.float32, device=c.device) for c in qc]
               for qc in q_chunks]
-    dkv_acc = [[(torch.zeros(k.shape, dtype=torch.float32, device=k.device),
-                 torch.zeros(v.shape, dtype=torch.float32, device=v.device)) for k, v in kvc]
-               for kvc in kv_chunks]
+    dkv_acc = [[torch.zeros((2,) + tuple(k.shape), dtype=torch.float32, device=k.device)
+                for k, _ in kvc] for kvc in kv_chunks]
     for r in range(world):
         for p in range(world):
             s = (p - r) % world
@@ -254,6 +274,6 @@ def ring_backward_emulated(qs, ks, vs, os_, dos, lses, causal=False, scale=None,
     dqs, dks, dvs = [], [], []
     for p in range(world):
         dqs.append(_convert(ops, dq_acc[p], q_chunks[p]))
-        dks.append(_convert(ops, [a for a, _ in dkv_acc[p]], [k for k, _ in kv_chunks[p]]))
-        dvs.append(_convert(ops, [b for _, b in dkv_acc[p]], [v for _, v in kv_chunks[p]]))
+        dks.append(_convert(ops, [a[0] for a in dkv_acc[p]], [k for k, _ in kv_chunks[p]]))
+        dvs.append(_convert(ops, [a[1] for a in dkv_acc[p]], [v for _, v in kv_chunks[p]]))
     return dqs, dks, dvs

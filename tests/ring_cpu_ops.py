@@ -45,7 +45,7 @@ class CpuOps:
         B, _, n, d = dk.shape
         dk = dk.reshape(B, Hkv, H // Hkv, n, d).sum(2)
         dv = dv.reshape(B, Hkv, H // Hkv, n, d).sum(2)
-        return tuple(torch.from_numpy(x) for x in (dq, dk, dv))
+        return torch.from_numpy(dq), torch.from_numpy(np.stack((dk, dv)))
 
     def merge(self, o_acc, lse_acc, o_part, lse_part, first, out):
         la = np.full(lse_part.shape, -np.inf) if first else _np(lse_acc)
