@@ -1039,19 +1039,19 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
                              static_cast<long long>(i) * BQ, flo, fhi);
                 edge = !(flo <= j * 128LL && j * 128LL + 127 <= fhi);
             }
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t u[32];
-                tmem_ld32(tS + 32 * h, u);
+            {   // the whole S^T row of the tile (64 columns): two loads, one wait
+                uint32_t u[64];
+                tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+                tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
                 tmem_ld_wait();
-                reg_fence<32>(u);
+                reg_fence<64>(u);
 #pragma unroll
-                for (int c = 0; c < 32; c += 4) {
-                    const float4 l4 = *reinterpret_cast<const float4*>(L2 + 32 * h + c);
-                    pr[32 * h + c] = ex2_approx(fmaf(__uint_as_float(u[c]), sl2, -l4.x));
-                    pr[32 * h + c + 1] = ex2_approx(fmaf(__uint_as_float(u[c + 1]), sl2, -l4.y));
-                    pr[32 * h + c + 2] = ex2_approx(fmaf(__uint_as_float(u[c + 2]), sl2, -l4.z));
-                    pr[32 * h + c + 3] = ex2_approx(fmaf(__uint_as_float(u[c + 3]), sl2, -l4.w));
+                for (int c = 0; c < 64; c += 4) {
+                    const float4 l4 = *reinterpret_cast<const float4*>(L2 + c);
+                    pr[c] = ex2_approx(fmaf(__uint_as_float(u[c]), sl2, -l4.x));
+                    pr[c + 1] = ex2_approx(fmaf(__uint_as_float(u[c + 1]), sl2, -l4.y));
+                    pr[c + 2] = ex2_approx(fmaf(__uint_as_float(u[c + 2]), sl2, -l4.z));
+                    pr[c + 3] = ex2_approx(fmaf(__uint_as_float(u[c + 3]), sl2, -l4.w));
                 }
             }
             if (edge) {
@@ -1073,12 +1073,14 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
             if (!(ok = wait_all(&bars->dp_full[x], ph))) break;
             if (it >= 2 && !(ok = wait_all(&bars->ds_free[x], ph ^ 1u))) break;
             tc_fence_after();
+            uint32_t du[64];                                   // the dP^T row, one wait
+            tmem_ld32(tDP, *reinterpret_cast<uint32_t(*)[32]>(&du[0]));
+            tmem_ld32(tDP + 32, *reinterpret_cast<uint32_t(*)[32]>(&du[32]));
+            tmem_ld_wait();
+            reg_fence<64>(du);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                uint32_t u[32];
-                tmem_ld32(tDP + 32 * h, u);
-                tmem_ld_wait();
-                reg_fence<32>(u);
+                const uint32_t* u = du + 32 * h;
                 uint32_t w[16];
 #pragma unroll
                 for (int c = 0; c < 16; c += 2) {
