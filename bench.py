@@ -275,19 +275,28 @@ def fwd_case_query_tiles(w):
     return w.B * w.H * ((w.n + rows - 1) // rows)
 
 
-def time_forward_case(ea, w, dev, stream, iters, warmup, hbm_peak, fma_peak):
+def time_forward_case(ea, w, dev, stream, iters, warmup, hbm_peak, fma_peak, e4m3=False):
     """Median device time of one forward launch of workload `w` over `iters` launches, each
-    preceded by a write of a buffer larger than L2 so that q, k, v come from HBM."""
+    preceded by a write of a buffer larger than L2 so that q, k, v come from HBM. With e4m3 the
+    workload's inputs are quantised to E4M3 (descale 2^-4) and run through the FP8 forward."""
     import torch
     import attn_inputs
     q, k, v, _ = attn_inputs.workload_inputs(w)
     q, k, v = (t.to(dev) for t in (q, k, v))
-    o = torch.empty_like(q)
+    desc = 2.0 ** -4
+    if e4m3:
+        q, k, v = ((t.float() / desc).clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
+                   for t in (q, k, v))
+    o = torch.empty(q.shape, dtype=torch.bfloat16 if e4m3 else q.dtype, device=dev)
     lse = torch.empty((w.B, w.H, w.n), dtype=torch.float32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def fwd():
-        ea.forward(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse, stream=stream)
+        if e4m3:
+            ea.forward_fp8(q, k, v, desc, desc, desc, causal=w.causal, scale=w.scale, out=o,
+                           lse=lse, stream=stream)
+        else:
+            ea.forward(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse, stream=stream)
 
     for _ in range(warmup):
         fwd()
@@ -304,13 +313,13 @@ def time_forward_case(ea, w, dev, stream, iters, warmup, hbm_peak, fma_peak):
     if ea.device_status() != ea.ATTN_OK:
         raise SystemExit(f"device status not OK in the {w.name} forward timings")
     us = statistics.median(a.elapsed_time(b) * 1e3 for a, b in ev)
-    nbytes = fwd_case_bytes(w)
+    nbytes = fwd_case_bytes(w) if not e4m3 else 3 * q.numel() + 2 * q.numel() + 4 * lse.numel()
     flops = 4.0 * w.B * w.H * w.n * w.n * w.d * (0.5 if w.causal else 1.0)
     gbs = nbytes / (us * 1e-6) / 1e9
     tflops = flops / (us * 1e-6) / 1e12
     out = {"us": us, "launches": iters, "bytes": nbytes, "hbm_gbs": gbs,
            "hbm_frac": gbs / hbm_peak, "tflops": tflops, "query_tiles": fwd_case_query_tiles(w),
-           "sms": SM_COUNT, "dtype": w.dtype,
+           "sms": SM_COUNT, "dtype": "e4m3" if e4m3 else w.dtype,
            "l2": f"{L2_FLUSH_BYTES >> 20} MiB written before every launch"}
     if w.dtype == "fp32":
         out["fma_frac"] = tflops / fma_peak
@@ -613,6 +622,10 @@ def main():
         small = {name: time_forward_case(ea, attn_inputs.WORKLOADS[name], dev, stream,
                                          args.small_case_launches, args.warmup, hbm, fma)
                  for name in SMALL_CASES}
+        # the row-tiling case's bf16 inputs quantised to E4M3, through the FP8 forward
+        small["rowtile_e4m3_4096x64"] = time_forward_case(
+            ea, attn_inputs.WORKLOADS["rowtile_bf16_4096x64"], dev, stream,
+            args.small_case_launches, args.warmup, hbm, fma, e4m3=True)
         small["peaks"] = {"hbm_gbs": hbm, "fp32_fma_tflops": fma,
                           "fp32_fma_kind": "148 SMs x 128 lanes x 2 FLOP x 1965 MHz"}
 

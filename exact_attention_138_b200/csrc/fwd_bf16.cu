@@ -57,10 +57,17 @@ struct FwdCfg {
     static constexpr int CHUNK = 128 * SWB;              // bytes of one [128 rows x CW] chunk
     static constexpr int TILE = NCH * CHUNK;             // bytes of one 128 x D tile
     static constexpr int STAGES = TILE >= 32768 ? 2 : 3;
-    static constexpr int SMEM = (2 + 2 * STAGES) * TILE + 512;
-    // the split kernel's partials (bf16 only: 2 x 128 rows x (D + 4) fp32, then 256 x (m, l)) fit in the
-    // Q/K/V staging memory they overwrite
-    static_assert(F8 || (2 * BM * (D + 4) + 2 * 2 * BM) * 4 <= (2 + 2 * STAGES) * TILE, "partials");
+    static constexpr int STAGING = (2 + 2 * STAGES) * TILE;    // Q tiles, K and V rings
+    static constexpr int SMEM = STAGING + 512;
+    // The split kernels' partials (2 x 128 rows x (D + 4) fp32, then 256 x (m, l)) are written
+    // over the staging memory once every copy and MMA of the CTA is complete. bf16 staging always
+    // holds them; E4M3 staging (half the bytes) may not, so the split kernels place the barrier
+    // block after whichever is larger.
+    static constexpr int PARTIALS = (2 * BM * (D + 4) + 2 * 2 * BM) * 4;
+    static constexpr int BARS_SPLIT = STAGING > PARTIALS ? STAGING : PARTIALS;
+    static constexpr int SMEM_SPLIT = BARS_SPLIT + 512;
+    static_assert(F8 || PARTIALS <= STAGING, "bf16 partials fit in the staging memory");
+    static_assert(SMEM_SPLIT <= 232448, "dynamic shared memory per block");
     static_assert(SWB == 128 || SWB == 64, "tile rows of 64 or 128 bytes");
 };
 
@@ -135,7 +142,7 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap* tmQ_, const CUtensor
     uint8_t* sQ = smem;                                   // 2 tiles
     uint8_t* sK = smem + 2 * C::TILE;                     // STAGES tiles
     uint8_t* sV = sK + C::STAGES * C::TILE;               // STAGES tiles
-    FwdBars* bars = reinterpret_cast<FwdBars*>(sV + C::STAGES * C::TILE);
+    FwdBars* bars = reinterpret_cast<FwdBars*>(smem + (SPLIT ? C::BARS_SPLIT : C::STAGING));
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -664,14 +671,30 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     fwd_body<D, true, false>(&tmQ, &tmK, &tmV, p);
 }
 
-// Clusters of `split` CTAs of the split kernel that the GPU holds at once (each CTA takes a whole
+// E4M3 inputs on small grids: clusters of p.split CTAs as fwd_bf16_split_kernel.
+template <int D>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    fwd_fp8_split_kernel(const __grid_constant__ CUtensorMap tmQ,
+                         const __grid_constant__ CUtensorMap tmK,
+                         const __grid_constant__ CUtensorMap tmV, const FwdKParams p) {
+    fwd_body<D, true, true>(&tmQ, &tmK, &tmV, p);
+}
+
+// The split kernel of an input type.
+template <int D, bool F8>
+constexpr auto split_kernel() {
+    if constexpr (F8) return fwd_fp8_split_kernel<D>;
+    else return fwd_bf16_split_kernel<D>;
+}
+
+// Clusters of `split` CTAs of a split kernel that the GPU holds at once (each CTA takes a whole
 // SM, and a cluster must fit in one GPC); queried once per (device, d, split) and kept in a
 // per-device table of atomics, so concurrent host threads and GPUs of different layouts each see
 // their own device's answer. While `stream` is being captured into a graph the query is not made
 // and half of SMs / split is assumed.
 constexpr int kClusterCacheDevices = 64;
 
-template <int D>
+template <int D, bool F8>
 int max_active_clusters(int split, int sms, cudaStream_t stream) {
     static std::atomic<int> cache[kClusterCacheDevices][4];
     const int slot = split == 2 ? 0 : split == 4 ? 1 : split == 8 ? 2 : 3;
@@ -692,14 +715,15 @@ int max_active_clusters(int split, int sms, cudaStream_t stream) {
         return sms / (2 * split);
     }
     if (cap != cudaStreamCaptureStatusNone) return sms / (2 * split);
-    using C = FwdCfg<D, false>;
-    if (cudaFuncSetAttribute(fwd_bf16_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM) != cudaSuccess)
+    using C = FwdCfg<D, F8>;
+    constexpr auto kern = split_kernel<D, F8>();
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_SPLIT) !=
+        cudaSuccess)
         return 0;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(split * 256));
     cfg.blockDim = dim3(kFwdThreads);
-    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.dynamicSmemBytes = C::SMEM_SPLIT;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = static_cast<unsigned>(split);
@@ -708,7 +732,7 @@ int max_active_clusters(int split, int sms, cudaStream_t stream) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, fwd_bf16_split_kernel<D>, &cfg) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
         (void)cudaGetLastError();
         return 0;
     }
@@ -716,10 +740,10 @@ int max_active_clusters(int split, int sms, cudaStream_t stream) {
     return n;
 }
 
-// Key shares per tile pair for the bf16 forward: 1 when the pairs alone fill half the SMs, else the
+// Key shares per tile pair for the forward: 1 when the pairs alone fill half the SMs, else the
 // largest power of two (at most 8, at most the largest number of key tiles a query tile sees)
 // that keeps the grid within one CTA per SM and every cluster resident at once.
-template <int D>
+template <int D, bool F8>
 int choose_fwd_split(const MaskSpec& mk, int qtiles, long long pairs_total, cudaStream_t stream) {
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -738,7 +762,7 @@ int choose_fwd_split(const MaskSpec& mk, int qtiles, long long pairs_total, cuda
     }
     int s = 1;
     while (s < 8 && pairs_total * s * 2 <= sms && s * 2 <= max_tiles &&
-           pairs_total <= max_active_clusters<D>(s * 2, sms, stream))
+           pairs_total <= max_active_clusters<D, F8>(s * 2, sms, stream))
         s *= 2;
     return s;
 }
@@ -777,20 +801,20 @@ cudaError_t launch_fwd_d(const FwdArgs& a, cudaStream_t stream) {
     kp.o_scale = F8 ? a.v_descale : 1.f;
     kp.timeout_ns = a.timeout_ns;
     const long long pairs_total = static_cast<long long>(kp.n_pairs) * BH;
-    kp.split = F8 ? 1 : choose_fwd_split<D>(kp.mask, qtiles, pairs_total, stream);
+    kp.split = choose_fwd_split<D, F8>(kp.mask, qtiles, pairs_total, stream);
     const long long grid = pairs_total * kp.split;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     if (kp.split == 1) {
         kern<<<static_cast<unsigned>(grid), kFwdThreads, C::SMEM, stream>>>(mq, mk, mv, kp);
         return cudaGetLastError();
     }
-    e = cudaFuncSetAttribute(fwd_bf16_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM);
+    constexpr auto skern = split_kernel<D, F8>();
+    e = cudaFuncSetAttribute(skern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_SPLIT);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(kFwdThreads);
-    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.dynamicSmemBytes = C::SMEM_SPLIT;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -799,7 +823,7 @@ cudaError_t launch_fwd_d(const FwdArgs& a, cudaStream_t stream) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, fwd_bf16_split_kernel<D>, mq, mk, mv, kp);
+    return cudaLaunchKernelEx(&cfg, skern, mq, mk, mv, kp);
 }
 
 }  // namespace

@@ -100,3 +100,19 @@ def test_fp8_rejects_bad_arguments(cuda_device):
     y = torch.zeros((1, 1, 128, 32), dtype=torch.float8_e4m3fn, device="cuda:0")
     with pytest.raises(ea.AttnError):
         ea.forward_fp8(y, y, y)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_forward_small_grid_key_split(cuda_device, causal):
+    # 1x1x4096x64, the size of the row-tiling example: 16 pairs of query tiles on 148 SMs, so each
+    # pair's keys are split over a thread-block cluster and the shares merged on chip
+    (q8, k8, v8), (qd, kd, vd), desc = _case((1, 1, 4096, 64), (1, 1, 4096, 64), seed=77)
+    dev = torch.device("cuda:0")
+    o, lse = ea.forward_fp8(q8.to(dev), k8.to(dev), v8.to(dev), *desc, causal=causal)
+    torch.cuda.synchronize()
+    assert ea.device_status() == ea.ATTN_OK
+    ro, rlse = oracle.fwd(qd.numpy(), kd.numpy(), vd.numpy(), 1.0 / 8.0, causal)
+    got = to_np(o)
+    assert np.abs(got - ro).max() <= _bound(vd, ro)
+    assert np.linalg.norm(got - ro) / np.linalg.norm(ro) <= 3e-2
+    assert np.abs(to_np(lse) - rlse).max() <= TOL_LSE["bf16"]
