@@ -437,12 +437,15 @@ def time_variants(args, w, ea, q, k, v, do, ws, stream, causal_flops):
     per_rank = [[torch.cat([x[p], x[2 * ranks - 1 - p]], dim=2).contiguous() for p in range(ranks)]
                 for x in chunks]
     rq, rk, rv, rdo = per_rank
-    os_, lses = ring.ring_forward_emulated(rq, rk, rv, causal=True, scale=w.scale, zigzag=True)
+    ops = ring.CudaOps()        # one set of buffers and workspaces for every step
+    os_, lses = ring.ring_forward_emulated(rq, rk, rv, causal=True, scale=w.scale, zigzag=True,
+                                           ops=ops)
 
     def ring_step():
-        o_, l_ = ring.ring_forward_emulated(rq, rk, rv, causal=True, scale=w.scale, zigzag=True)
+        o_, l_ = ring.ring_forward_emulated(rq, rk, rv, causal=True, scale=w.scale, zigzag=True,
+                                            ops=ops)
         ring.ring_backward_emulated(rq, rk, rv, o_, rdo, l_, causal=True, scale=w.scale,
-                                    zigzag=True)
+                                    zigzag=True, ops=ops)
     ms = timed(ring_step)
     out["ring_zigzag_4"] = {"ms": ms, "tflops": causal_flops / (ms * 1e-3) / 1e12,
                             "config": "4 ranks emulated on one GPU (all ranks' hops in turn), "

@@ -66,6 +66,13 @@ _lib.attn_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
 _lib.attn_bwd.restype = _i
 _lib.attn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i,
                           _i, _i, _vp, _sz, _vp]
+_lib.attn_bwd_prepare.restype = _i
+_lib.attn_bwd_prepare.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]
+_lib.attn_bwd_accumulate.restype = _i
+_lib.attn_bwd_accumulate.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i,
+                                     _i, _i, _i, _vp, _sz, _vp]
+_lib.attn_bwd_finish.restype = _i
+_lib.attn_bwd_finish.argtypes = [_vp, _i, _i, _i, _i, _f, _i, _i, _vp, _sz, _vp]
 _lib.attn_get_device_status.restype = _i
 _lib.attn_get_device_status.argtypes = [_vp]
 _lib.attn_set_wait_timeout_us.restype = ctypes.c_uint
@@ -154,6 +161,25 @@ def attn_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, H, n, d, scale, causal, dtype, 
              workspace, ws_bytes, stream) -> int:
     return _lib.attn_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, H, n, d, scale, causal, dtype,
                          deterministic, workspace, ws_bytes, stream)
+
+
+def attn_bwd_prepare(o, dO, lse, B, H, nq, d, dtype, deterministic, workspace, ws_bytes,
+                     stream) -> int:
+    return _lib.attn_bwd_prepare(o, dO, lse, B, H, nq, d, dtype, deterministic, workspace,
+                                 ws_bytes, stream)
+
+
+def attn_bwd_accumulate(q, k, v, dO, dk_acc, dv_acc, B, H, Hkv, nq, nk, d, scale, window_left,
+                        window_right, dtype, deterministic, workspace, ws_bytes, stream) -> int:
+    return _lib.attn_bwd_accumulate(q, k, v, dO, dk_acc, dv_acc, B, H, Hkv, nq, nk, d, scale,
+                                    window_left, window_right, dtype, deterministic, workspace,
+                                    ws_bytes, stream)
+
+
+def attn_bwd_finish(dq, B, H, nq, d, scale, dtype, deterministic, workspace, ws_bytes,
+                    stream) -> int:
+    return _lib.attn_bwd_finish(dq, B, H, nq, d, scale, dtype, deterministic, workspace, ws_bytes,
+                                stream)
 
 
 def attn_get_device_status(stream=None) -> int:
@@ -299,6 +325,59 @@ def backward(q, k, v, o, do, lse, causal=False, scale=None, deterministic=False,
                           _stream_handle(stream))
     _check(rc, "attn_bwd")
     return dq, dk, dv
+
+
+class BackwardSum:
+    """The backward pass of one set of queries, summed over several key sets (attn_bwd_prepare /
+    attn_bwd_accumulate / attn_bwd_finish): construct with the final o, dO, lse of the queries,
+    call `add` once per key set (dK, dV added into fp32 arrays the caller zeroed), then `finish`
+    for dQ. The workspace it holds is reused by `reset` for another pass of the same sizes."""
+
+    def __init__(self, o, do, lse, deterministic=False, stream=None):
+        import torch
+        self.B, self.H, self.n, self.d = _dims(o)
+        self.det = int(bool(deterministic))
+        need = attn_bwd_workspace_bytes(self.B, self.H, self.n, self.d, self.det)
+        self.ws = torch.empty(need, dtype=torch.uint8, device=o.device)
+        self.reset(o, do, lse, stream)
+
+    def reset(self, o, do, lse, stream=None):
+        if _dims(o) != (self.B, self.H, self.n, self.d):
+            raise ValueError("reset needs the sizes the workspace was made for")
+        rc = attn_bwd_prepare(_ptr(o), _ptr(do), _ptr(lse), self.B, self.H, self.n, self.d,
+                              _dtype_code(o), self.det, _ptr(self.ws), self.ws.numel(),
+                              _stream_handle(stream))
+        _check(rc, "attn_bwd_prepare")
+
+    def add(self, q, k, v, do, dk_acc, dv_acc, scale=None, causal=False, window=None,
+            stream=None):
+        """dQ sum += and dk_acc, dv_acc (fp32, k's shape) += the gradients over keys k, v."""
+        Hkv, nk = _kv_heads(q, k, v)
+        for t in (dk_acc, dv_acc):
+            if t.shape != k.shape or t.dtype.itemsize != 4 or not t.is_floating_point():
+                raise ValueError("dk_acc, dv_acc must be fp32 with k's shape")
+        if scale is None:
+            scale = 1.0 / math.sqrt(self.d)
+        wl, wr = _window(causal, window)
+        rc = attn_bwd_accumulate(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dk_acc), _ptr(dv_acc),
+                                 self.B, self.H, Hkv, self.n, nk, self.d, float(scale), wl, wr,
+                                 _dtype_code(q), self.det, _ptr(self.ws), self.ws.numel(),
+                                 _stream_handle(stream))
+        _check(rc, "attn_bwd_accumulate")
+
+    def finish(self, dq=None, scale=None, stream=None):
+        """dQ (bf16, (B, H, n, d)) = scale · the dQ sum."""
+        import torch
+        if dq is None:
+            dq = torch.empty((self.B, self.H, self.n, self.d), dtype=torch.bfloat16,
+                             device=self.ws.device)
+        if scale is None:
+            scale = 1.0 / math.sqrt(self.d)
+        rc = attn_bwd_finish(_ptr(dq), self.B, self.H, self.n, self.d, float(scale),
+                             _dtype_code(dq), self.det, _ptr(self.ws), self.ws.numel(),
+                             _stream_handle(stream))
+        _check(rc, "attn_bwd_finish")
+        return dq
 
 
 def device_status(stream=None) -> int:

@@ -295,6 +295,97 @@ int attn_bwd_ex(const void* q, const void* k, const void* v, const void* o, cons
                     window_right, dtype, deterministic, workspace, ws_bytes, stream);
 }
 
+// Workspace arguments shared by the backward entry points: present, 256-byte aligned, large
+// enough for (B, H, nq, d, deterministic).
+static int check_ws(const void* workspace, size_t ws_bytes, int B, int H, int nq, int d,
+                    int deterministic, WsLayout* w) {
+    *w = ws_layout(B, H, nq, d, deterministic);
+    if (!workspace) return ATTN_ERR_INVALID;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_INVALID;
+    if (ws_bytes < w->total) return ATTN_ERR_WORKSPACE;
+    return ATTN_OK;
+}
+
+static void set_ws(BwdArgs& a, void* workspace, const WsLayout& w, int deterministic) {
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    a.Dvec = reinterpret_cast<float*>(ws + w.d_off);
+    a.L2vec = reinterpret_cast<float*>(ws + w.l2_off);
+    a.dq_acc = reinterpret_cast<float*>(ws + w.acc_off);
+    a.sems = deterministic ? reinterpret_cast<int*>(ws + w.sem_off) : nullptr;
+    a.timeout_ns = static_cast<uint64_t>(g_timeout_us.load()) * 1000ull;
+    a.phase_events = nullptr;
+}
+
+int attn_bwd_prepare(const void* o, const void* dO, const float* lse, int B, int H, int nq,
+                     int d, int dtype, int deterministic, void* workspace, size_t ws_bytes,
+                     void* stream) {
+    if (!o || !dO || !lse) return ATTN_ERR_INVALID;
+    int rc = validate_common(B, H, nq, d, 1.f, dtype);
+    if (rc) return rc;
+    if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(o) || !aligned16(dO) || !aligned16(lse)) return ATTN_ERR_INVALID;
+    WsLayout w;
+    if ((rc = check_ws(workspace, ws_bytes, B, H, nq, d, deterministic, &w))) return rc;
+    BwdArgs a = {};
+    a.o = o; a.dO = dO; a.lse = lse;
+    a.B = B; a.H = H; a.Hkv = H; a.nq = nq; a.nk = nq; a.d = d;
+    a.scale = 1.f;
+    a.wl = -1; a.wr = -1;
+    a.deterministic = deterministic ? 1 : 0;
+    set_ws(a, workspace, w, a.deterministic);
+    a.phases = 1;
+    return to_code(launch_bwd_bf16(a, static_cast<cudaStream_t>(stream)));
+}
+
+int attn_bwd_accumulate(const void* q, const void* k, const void* v, const void* dO,
+                        float* dk_acc, float* dv_acc, int B, int H, int Hkv, int nq, int nk, int d,
+                        float scale, int window_left, int window_right, int dtype,
+                        int deterministic, void* workspace, size_t ws_bytes, void* stream) {
+    if (!q || !k || !v || !dO || !dk_acc || !dv_acc) return ATTN_ERR_INVALID;
+    int rc = validate_common(B, H, nq, d, scale, dtype);
+    if (rc) return rc;
+    if (nk < 1 || nk > kMaxSeq) return ATTN_ERR_INVALID;
+    if (Hkv < 1 || H % Hkv != 0) return ATTN_ERR_INVALID;
+    if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+    const void* ptrs[] = {q, k, v, dO, dk_acc, dv_acc};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return ATTN_ERR_INVALID;
+    WsLayout w;
+    if ((rc = check_ws(workspace, ws_bytes, B, H, nq, d, deterministic, &w))) return rc;
+    BwdArgs a = {};
+    a.q = q; a.k = k; a.v = v; a.dO = dO;
+    a.B = B; a.H = H; a.Hkv = Hkv; a.nq = nq; a.nk = nk; a.d = d;
+    a.scale = scale;
+    a.wl = window_left < 0 ? -1 : window_left;
+    a.wr = window_right < 0 ? -1 : window_right;
+    a.deterministic = deterministic ? 1 : 0;
+    set_ws(a, workspace, w, a.deterministic);
+    a.phases = 2;
+    a.dk_acc32 = dk_acc;
+    a.dv_acc32 = dv_acc;
+    return to_code(launch_bwd_bf16(a, static_cast<cudaStream_t>(stream)));
+}
+
+int attn_bwd_finish(void* dq, int B, int H, int nq, int d, float scale, int dtype,
+                    int deterministic, void* workspace, size_t ws_bytes, void* stream) {
+    if (!dq) return ATTN_ERR_INVALID;
+    int rc = validate_common(B, H, nq, d, scale, dtype);
+    if (rc) return rc;
+    if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(dq)) return ATTN_ERR_INVALID;
+    WsLayout w;
+    if ((rc = check_ws(workspace, ws_bytes, B, H, nq, d, deterministic, &w))) return rc;
+    BwdArgs a = {};
+    a.dq = dq;
+    a.B = B; a.H = H; a.Hkv = H; a.nq = nq; a.nk = nq; a.d = d;
+    a.scale = scale;
+    a.wl = -1; a.wr = -1;
+    a.deterministic = deterministic ? 1 : 0;
+    set_ws(a, workspace, w, a.deterministic);
+    a.phases = 4;
+    return to_code(launch_bwd_bf16(a, static_cast<cudaStream_t>(stream)));
+}
+
 int attn_ring_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
                     long long rows, int d, int part_dtype, int first, void* o_out, int out_dtype,
                     void* stream) {

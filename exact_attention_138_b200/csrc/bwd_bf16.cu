@@ -74,6 +74,26 @@ struct BwdKParams {
     uint64_t timeout_ns;
 };
 
+// Accumulating launches (the backward in parts) add dK and dV in fp32 into these arrays
+// (B, Hkv, nk, d) instead of storing them; a kernel parameter of its own, used only by the
+// accumulating instantiation of each main kernel.
+struct AccOut {
+    float* dk;
+    float* dv;
+};
+
+// dst[0 .. N) += mul · (TMEM words u as fp32); dst 16-byte aligned. Vector reductions performed
+// in L2: nothing waits for them, and each element of dst gets one addition per launch (one CTA
+// owns each key row), so the sum does not depend on timing.
+template <int N>
+__device__ __forceinline__ void add_row_f32(float* dst, const uint32_t* u, float mul) {
+#pragma unroll
+    for (int c = 0; c < N / 4; ++c)
+        red_add_v4_f32(dst + 4 * c, __uint_as_float(u[4 * c]) * mul,
+                       __uint_as_float(u[4 * c + 1]) * mul, __uint_as_float(u[4 * c + 2]) * mul,
+                       __uint_as_float(u[4 * c + 3]) * mul);
+}
+
 __device__ __forceinline__ void drain_wait_bwd(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return;
     const uint64_t t0 = globaltimer_ns();
@@ -189,11 +209,11 @@ __global__ void __launch_bounds__(256) bwd_dq_convert_kernel(const float* __rest
 // softmax of the next overlap the dK/dQ MMAs. dQ has TMEM lane = query, and each thread adds
 // 16-byte pieces of its row to the fp32 accumulator with red.global.
 // ------------------------------------------------------------------------------------------
-template <int D>
+template <int D, bool ACC>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                    const BwdKParams p) {
+                    const BwdKParams p, const AccOut acc) {
     using C = BwdCfg<D>;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t* sK = smem;
@@ -599,7 +619,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (ok && NTT > 0) ok = drain(NTT - 1);
         if (ok && NTT == 0) {
             // no query sees these keys: dK = dV = 0
-            if (kidx < nk) {
+            if (kidx < nk && !ACC) {     // (accumulating: nothing to add)
                 const size_t orow = (static_cast<size_t>(kvbh) * nk + kidx) * D + g * (D / 2);
 #pragma unroll
                 for (int x = 0; x < D / 16; ++x) {
@@ -623,6 +643,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     uint32_t u[16];
                     tmem_ld16(tacc + cc, u);
                     tmem_ld_wait();
+                    if constexpr (ACC) {
+                        if (kidx < nk) add_row_f32<16>((which == 0 ? acc.dv : acc.dk) + orow + cc, u, mul);
+                        continue;
+                    }
                     uint32_t w[8];
 #pragma unroll
                     for (int x = 0; x < 8; ++x)
@@ -719,10 +743,12 @@ struct Bars {
 static_assert(sizeof(Bars) <= 256, "barrier block");
 }  // namespace q64
 
+template <bool ACC>
 __global__ void __launch_bounds__(q64::kThreads, 1)
     bwd_main_q64_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                        const __grid_constant__ CUtensorMap tmAcc, const BwdKParams p) {
+                        const __grid_constant__ CUtensorMap tmAcc, const BwdKParams p,
+                        const AccOut acc) {
     using namespace q64;
     constexpr int D = 128;
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -1104,7 +1130,7 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
         // ---- epilogue: warpgroup x writes head-dim columns 64x .. 64x+63 of dV and dK
         if (ok && NTT == 0) {
             // no query sees these keys: dK = dV = 0
-            if (kidx < nk) {
+            if (kidx < nk && !ACC) {     // (accumulating: nothing to add)
                 const size_t orow = (static_cast<size_t>(kvbh) * nk + kidx) * D + x * 64;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
@@ -1129,6 +1155,10 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
                     tmem_ld32(tacc + cc, u);
                     tmem_ld_wait();
                     reg_fence<32>(u);
+                    if constexpr (ACC) {
+                        if (kidx < nk) add_row_f32<32>((which == 0 ? acc.dv : acc.dk) + orow + cc, u, mul);
+                        continue;
+                    }
                     uint32_t w[16];
 #pragma unroll
                     for (int c = 0; c < 16; ++c)
@@ -1175,7 +1205,7 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
     const cudaEvent_t* ev = a.phase_events;
     if (ev && ev[0] && (e = cudaEventRecord(ev[0], stream)) != cudaSuccess) return e;
     // 1. preprocess
-    {
+    if (a.phases & 1) {
         const long long rows = static_cast<long long>(BH) * n_pad;
         const int rpw = 32 / (D / 8);
         long long blocks = (rows + (8 * rpw) - 1) / (8 * rpw);
@@ -1188,54 +1218,62 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     // 2. main
-    BwdKParams kp;
-    kp.lse = a.lse;
-    kp.Dvec = a.Dvec;
-    kp.L2vec = a.L2vec;
-    kp.dq_acc = a.dq_acc;
-    kp.sems = a.sems;
-    kp.dk = static_cast<__nv_bfloat16*>(a.dk);
-    kp.dv = static_cast<__nv_bfloat16*>(a.dv);
-    kp.n_pad = n_pad;
-    kp.BH = BHkv;
-    kp.nkt = nkt;
-    kp.kv_group = kvg;
-    kp.deterministic = a.deterministic;
-    kp.group = group;
-    kp.mask = MaskSpec{a.nq, a.nk, a.wl, a.wr, static_cast<long long>(a.nk) - a.nq};
-    kp.scale = a.scale;
-    kp.scale_log2 = a.scale * kBwdLog2e;
-    kp.timeout_ns = a.timeout_ns;
-    const long long grid = static_cast<long long>(nkt) * BHkv;
-    if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    const int qbox = D == 128 ? q64::BQ : 128;
-    CUtensorMap mq, mk, mv, mdo;
-    if ((e = make_tmap_bf16(&mq, a.q, BH, a.nq, D, qbox)) != cudaSuccess) return e;
-    if ((e = make_tmap_bf16(&mk, a.k, BHkv, a.nk, D)) != cudaSuccess) return e;
-    if ((e = make_tmap_bf16(&mv, a.v, BHkv, a.nk, D)) != cudaSuccess) return e;
-    if ((e = make_tmap_bf16(&mdo, a.dO, BH, a.nq, D, qbox)) != cudaSuccess) return e;
-    if constexpr (D == 128) {
-        CUtensorMap macc;   // the fp32 dQ accumulator as (B·H·n_pad) rows x 128 columns
-        if ((e = make_tmap_acc(&macc, a.dq_acc, static_cast<long long>(BH) * n_pad, D)) != cudaSuccess)
-            return e;
-        e = cudaFuncSetAttribute(bwd_main_q64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 q64::SMEM);
-        if (e != cudaSuccess) return e;
-        if (ev && ev[1] && (e = cudaEventRecord(ev[1], stream)) != cudaSuccess) return e;
-        bwd_main_q64_kernel<<<static_cast<unsigned>(grid), q64::kThreads, q64::SMEM, stream>>>(
-            mq, mk, mv, mdo, macc, kp);
-    } else {
-        e = cudaFuncSetAttribute(bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::SMEM);
-        if (e != cudaSuccess) return e;
-        if (ev && ev[1] && (e = cudaEventRecord(ev[1], stream)) != cudaSuccess) return e;
-        bwd_main_kernel<D><<<static_cast<unsigned>(grid), kBwdThreads, C::SMEM, stream>>>(
-            mq, mk, mv, mdo, kp);
+    if (a.phases & 2) {
+        if (a.deterministic && !(a.phases & 1)) {
+            // the semaphores count this launch's partials from zero (the accumulator keeps its sums)
+            const size_t n_sems = static_cast<size_t>(BH) * (n_pad / 64) * 4;
+            if ((e = cudaMemsetAsync(a.sems, 0, n_sems * sizeof(int), stream)) != cudaSuccess) return e;
+        }
+        const AccOut acc{a.dk_acc32, a.dv_acc32};
+        BwdKParams kp;
+        kp.lse = a.lse;
+        kp.Dvec = a.Dvec;
+        kp.L2vec = a.L2vec;
+        kp.dq_acc = a.dq_acc;
+        kp.sems = a.sems;
+        kp.dk = static_cast<__nv_bfloat16*>(a.dk);
+        kp.dv = static_cast<__nv_bfloat16*>(a.dv);
+        kp.n_pad = n_pad;
+        kp.BH = BHkv;
+        kp.nkt = nkt;
+        kp.kv_group = kvg;
+        kp.deterministic = a.deterministic;
+        kp.group = group;
+        kp.mask = MaskSpec{a.nq, a.nk, a.wl, a.wr, static_cast<long long>(a.nk) - a.nq};
+        kp.scale = a.scale;
+        kp.scale_log2 = a.scale * kBwdLog2e;
+        kp.timeout_ns = a.timeout_ns;
+        const long long grid = static_cast<long long>(nkt) * BHkv;
+        if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+        const int qbox = D == 128 ? q64::BQ : 128;
+        CUtensorMap mq, mk, mv, mdo;
+        if ((e = make_tmap_bf16(&mq, a.q, BH, a.nq, D, qbox)) != cudaSuccess) return e;
+        if ((e = make_tmap_bf16(&mk, a.k, BHkv, a.nk, D)) != cudaSuccess) return e;
+        if ((e = make_tmap_bf16(&mv, a.v, BHkv, a.nk, D)) != cudaSuccess) return e;
+        if ((e = make_tmap_bf16(&mdo, a.dO, BH, a.nq, D, qbox)) != cudaSuccess) return e;
+        if constexpr (D == 128) {
+            CUtensorMap macc;   // the fp32 dQ accumulator as (B·H·n_pad) rows x 128 columns
+            if ((e = make_tmap_acc(&macc, a.dq_acc, static_cast<long long>(BH) * n_pad, D)) != cudaSuccess)
+                return e;
+            const auto kern = acc.dk ? bwd_main_q64_kernel<true> : bwd_main_q64_kernel<false>;
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, q64::SMEM);
+            if (e != cudaSuccess) return e;
+            if (ev && ev[1] && (e = cudaEventRecord(ev[1], stream)) != cudaSuccess) return e;
+            kern<<<static_cast<unsigned>(grid), q64::kThreads, q64::SMEM, stream>>>(
+                mq, mk, mv, mdo, macc, kp, acc);
+        } else {
+            const auto kern = acc.dk ? bwd_main_kernel<D, true> : bwd_main_kernel<D, false>;
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+            if (e != cudaSuccess) return e;
+            if (ev && ev[1] && (e = cudaEventRecord(ev[1], stream)) != cudaSuccess) return e;
+            kern<<<static_cast<unsigned>(grid), kBwdThreads, C::SMEM, stream>>>(mq, mk, mv, mdo, kp,
+                                                                                acc);
+        }
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if (ev && ev[2] && (e = cudaEventRecord(ev[2], stream)) != cudaSuccess) return e;
     }
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if (ev && ev[2] && (e = cudaEventRecord(ev[2], stream)) != cudaSuccess) return e;
     // 3. dQ convert
-    {
+    if (a.phases & 4) {
         const long long total8 = static_cast<long long>(BH) * a.nq * (D / 8);
         long long blocks = (total8 + 255) / 256;
         if (blocks > 148 * 16) blocks = 148 * 16;

@@ -110,6 +110,12 @@ struct BwdArgs {
     int* sems;        // workspace: B*H*(n_pad/64)*4, deterministic mode only
     uint64_t timeout_ns;
     const cudaEvent_t* phase_events;   // 4 events or nullptr (measurement hook)
+    // Kernels to run: 1 the preprocess (D, LSE·log2 e, zeroed dQ accumulator and semaphores),
+    // 2 the main kernel, 4 the dQ conversion. With dk_acc32 / dv_acc32 set, the main kernel adds
+    // dK and dV (fp32, (B, Hkv, nk, d)) into them instead of writing dk, dv.
+    int phases = 7;
+    float* dk_acc32 = nullptr;
+    float* dv_acc32 = nullptr;
 };
 
 // Encodes a 3-D tensor map over a (B*H, n, d) tensor of `esize`-byte elements (2: bf16, 1: 8-bit)

@@ -178,6 +178,40 @@ int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
                      int B, int H, int n, int d, float scale, int causal, int dtype,
                      int deterministic, void* stream);
 
+/* The backward pass in three parts, for gradients summed over several key sets with the same
+ * queries (ring attention: one call of attn_bwd_accumulate per hop, each with the K/V chunk that
+ * the hop holds; "Attention Mechanism: Revolusi Representasi Sequence", §16 "Long Context
+ * Training", Ring Attention). Because P = exp(scale·q·k - LSE) uses the final LSE over all keys and
+ * D = rowsum(dO∘O) the final O (the recomputation of "Flash Attention Nedir?", Recomputation),
+ * each key set's contribution to dQ, dK and dV is independent of the others and the sums are the
+ * gradients of attention over all keys together. bf16 inputs only (else ATTN_ERR_UNSUPPORTED).
+ * The workspace is attn_bwd_workspace_bytes(B, H, nq, d, deterministic), 256-byte aligned; it
+ * carries D, LSE·log2(e) and the fp32 dQ sum from one call to the next, so the calls of one
+ * sequence use the same workspace, sizes and deterministic flag, in stream order.
+ *
+ * attn_bwd_prepare: o, dO (B, H, nq, d) bf16 and lse (B, H, nq) fp32 of the whole forward pass;
+ *   computes D and LSE·log2(e) and zeroes the dQ sum.
+ * attn_bwd_accumulate: adds the gradients of attention of q, dO (B, H, nq, d) over the keys
+ *   k, v (B, Hkv, nk, d) with the visible window of attn_fwd_ex: dQ into the workspace's fp32
+ *   sum, and dK, dV (scale included, summed over the query heads of each K/V head) into the
+ *   caller's fp32 arrays dk_acc, dv_acc (B, Hkv, nk, d), which the caller zeroes before the first
+ *   call. Keys that no query sees add nothing. deterministic != 0: each call adds a query tile's
+ *   partials in decreasing key-tile order, so the whole sequence of calls repeats bit for bit.
+ * attn_bwd_finish: writes dq (B, H, nq, d) bf16 = scale · the dQ sum.
+ * Errors: null or misaligned (16-byte) pointer, or sizes as attn_bwd_ex -> ATTN_ERR_INVALID; a
+ *   workspace that is null or not 256-byte aligned -> ATTN_ERR_INVALID, too small ->
+ *   ATTN_ERR_WORKSPACE; a failed launch -> ATTN_ERR_CUDA. Arguments are checked before anything
+ *   is launched. */
+int attn_bwd_prepare(const void* o, const void* dO, const float* lse, int B, int H, int nq, int d,
+                     int dtype, int deterministic, void* workspace, size_t ws_bytes,
+                     void* stream);
+int attn_bwd_accumulate(const void* q, const void* k, const void* v, const void* dO,
+                        float* dk_acc, float* dv_acc, int B, int H, int Hkv, int nq, int nk, int d,
+                        float scale, int window_left, int window_right, int dtype,
+                        int deterministic, void* workspace, size_t ws_bytes, void* stream);
+int attn_bwd_finish(void* dq, int B, int H, int nq, int d, float scale, int dtype,
+                    int deterministic, void* workspace, size_t ws_bytes, void* stream);
+
 /* Synchronises `stream`, then returns and clears the sticky device status word: ATTN_OK, or
  * ATTN_ERR_TIMEOUT if a kernel's bounded wait expired since the last call, or ATTN_ERR_CUDA if
  * the synchronisation itself failed. */

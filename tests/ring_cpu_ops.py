@@ -1,7 +1,8 @@
-"""CPU stand-ins (fp64 numpy) for the four per-hop operations of the ring schedule, so that the
+"""CPU stand-ins (fp64 numpy) for the per-hop operations of the ring schedule, so that the
 multi-rank schedule and its point-to-point exchanges can run as gloo ranks on the CPU. The hop
 forward is the oracle's masked definition; the hop backward uses the global LSE and O (as the
-CUDA hop kernel does): P = exp(scale·q·k - LSE), D = rowsum(dO∘O), dS = P∘(dP - D)."""
+CUDA kernels do): P = exp(scale·q·k - LSE), D = rowsum(dO∘O), dS = P∘(dP - D), with dQ summed in
+the query chunk's state and dK, dV added into the travelling fp32 accumulators."""
 import numpy as np
 import torch
 
@@ -24,28 +25,36 @@ def _visible(nq, nk, wl, wr):
 
 
 class CpuOps:
-    def fwd(self, q, k, v, scale, window):
+    def fwd(self, q, k, v, scale, window, slot=0):
         o, lse = oracle.fwd_ex(q.float().numpy(), k.float().numpy(), v.float().numpy(), scale,
                                window[0], window[1])
         return torch.from_numpy(o), torch.from_numpy(lse)
 
-    def bwd(self, q, k, v, o, do, lse, scale, window, deterministic):
-        Q, K, V, O, dO, L = (_np(x) for x in (q, k, v, o, do, lse))
+    def bwd_begin(self, key, o, do, lse, deterministic):
+        """State of one query chunk: D = rowsum(dO∘O), the global LSE and a zero dQ sum."""
+        O, dO, L = _np(o), _np(do), _np(lse)
+        return {"D": (dO * O).sum(-1), "L": L, "dq": np.zeros(O.shape)}
+
+    def bwd_add(self, st, q, k, v, do, dkv_acc, scale, window):
+        Q, K, V, dO = (_np(x) for x in (q, k, v, do))
         H, Hkv = Q.shape[1], K.shape[1]
         K, V = np.repeat(K, H // Hkv, axis=1), np.repeat(V, H // Hkv, axis=1)
         vis = _visible(Q.shape[2], K.shape[2], *window)
         S = np.einsum("bhid,bhjd->bhij", Q, K) * scale
-        P = np.where(vis, np.exp(S - L[..., None]), 0.0)
+        P = np.where(vis, np.exp(S - st["L"][..., None]), 0.0)
         dP = np.einsum("bhid,bhjd->bhij", dO, V)
-        D = (dO * O).sum(-1)
-        dS = P * (dP - D[..., None])
-        dq = scale * np.einsum("bhij,bhjd->bhid", dS, K)
+        dS = P * (dP - st["D"][..., None])
+        st["dq"] += np.einsum("bhij,bhjd->bhid", dS, K)
         dk = scale * np.einsum("bhij,bhid->bhjd", dS, Q)
         dv = np.einsum("bhij,bhid->bhjd", P, dO)
         B, _, n, d = dk.shape
         dk = dk.reshape(B, Hkv, H // Hkv, n, d).sum(2)
         dv = dv.reshape(B, Hkv, H // Hkv, n, d).sum(2)
-        return torch.from_numpy(dq), torch.from_numpy(np.stack((dk, dv)))
+        dkv_acc.copy_(torch.from_numpy(_np(dkv_acc) + np.stack((dk, dv))))
+
+    def bwd_finish(self, st, out, scale):
+        out.copy_(torch.from_numpy(scale * st["dq"]))
+        return out
 
     def merge(self, o_acc, lse_acc, o_part, lse_part, first, out):
         la = np.full(lse_part.shape, -np.inf) if first else _np(lse_acc)

@@ -168,3 +168,47 @@ def test_noalloc_validates_before_touching_the_device():
     assert call(ok, scale=0.0) == ea.ATTN_ERR_INVALID
     assert ea.attn_bwd_workspace_bytes(1, 64, 8192, 128, 0) > (32 << 20)
     assert call(ok, B=1, H=64, n=8192) == ea.ATTN_ERR_WORKSPACE
+
+
+def _parts(which, **kw):
+    """One of the three backward-part entry points with valid fake arguments, `kw` overriding."""
+    a = dict(B=1, H=2, Hkv=1, nq=300, nk=500, d=128, scale=0.1, wl=-1, wr=0,
+             dtype=ea.ATTN_BF16, det=1)
+    a.update(kw)
+    need = (ea.attn_bwd_workspace_bytes(a["B"], a["H"], a["nq"], a["d"], a["det"])
+            if a["B"] > 0 and a["nq"] > 0 else 0)
+    ws = ctypes.c_void_p(kw.get("ws", FAKE))
+    ws_bytes = kw.get("ws_bytes", need)
+    P = lambda name: ctypes.c_void_p(kw.get(name, FAKE))
+    if which == "prepare":
+        return ea.attn_bwd_prepare(P("o"), P("dO"), P("lse"), a["B"], a["H"], a["nq"], a["d"],
+                                   a["dtype"], a["det"], ws, ws_bytes, None)
+    if which == "accumulate":
+        return ea.attn_bwd_accumulate(P("q"), P("k"), P("v"), P("dO"), P("dk_acc"), P("dv_acc"),
+                                      a["B"], a["H"], a["Hkv"], a["nq"], a["nk"], a["d"],
+                                      a["scale"], a["wl"], a["wr"], a["dtype"], a["det"], ws,
+                                      ws_bytes, None)
+    return ea.attn_bwd_finish(P("dq"), a["B"], a["H"], a["nq"], a["d"], a["scale"], a["dtype"],
+                              a["det"], ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("which,kw,code", [
+    ("prepare", dict(o=0), ea.ATTN_ERR_INVALID),
+    ("prepare", dict(lse=FAKE + 4), ea.ATTN_ERR_INVALID),
+    ("prepare", dict(dtype=ea.ATTN_FP32), ea.ATTN_ERR_UNSUPPORTED),
+    ("prepare", dict(ws_bytes=1000), ea.ATTN_ERR_WORKSPACE),
+    ("prepare", dict(ws=FAKE + 16), ea.ATTN_ERR_INVALID),
+    ("accumulate", dict(dk_acc=0), ea.ATTN_ERR_INVALID),
+    ("accumulate", dict(dv_acc=FAKE + 8), ea.ATTN_ERR_INVALID),
+    ("accumulate", dict(Hkv=3), ea.ATTN_ERR_INVALID),          # H not a multiple of Hkv
+    ("accumulate", dict(nk=0), ea.ATTN_ERR_INVALID),
+    ("accumulate", dict(scale=-1.0), ea.ATTN_ERR_INVALID),
+    ("accumulate", dict(d=48), ea.ATTN_ERR_UNSUPPORTED),
+    ("accumulate", dict(ws=0), ea.ATTN_ERR_INVALID),
+    ("accumulate", dict(ws_bytes=4096), ea.ATTN_ERR_WORKSPACE),
+    ("finish", dict(dq=0), ea.ATTN_ERR_INVALID),
+    ("finish", dict(nq=0), ea.ATTN_ERR_INVALID),
+    ("finish", dict(det=0, ws_bytes=100), ea.ATTN_ERR_WORKSPACE),
+])
+def test_backward_parts_reject_bad_arguments(which, kw, code):
+    assert _parts(which, **kw) == code
