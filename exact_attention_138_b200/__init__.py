@@ -66,6 +66,9 @@ _lib.attn_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
 _lib.attn_bwd.restype = _i
 _lib.attn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i,
                           _i, _i, _vp, _sz, _vp]
+_lib.attn_fwd_accumulate.restype = _i
+_lib.attn_fwd_accumulate.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i,
+                                     _i, _vp]
 _lib.attn_bwd_prepare.restype = _i
 _lib.attn_bwd_prepare.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]
 _lib.attn_bwd_accumulate.restype = _i
@@ -161,6 +164,12 @@ def attn_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, H, n, d, scale, causal, dtype, 
              workspace, ws_bytes, stream) -> int:
     return _lib.attn_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, H, n, d, scale, causal, dtype,
                          deterministic, workspace, ws_bytes, stream)
+
+
+def attn_fwd_accumulate(q, k, v, o_acc, lse_acc, B, H, Hkv, nq, nk, d, scale, window_left,
+                        window_right, first, stream) -> int:
+    return _lib.attn_fwd_accumulate(q, k, v, o_acc, lse_acc, B, H, Hkv, nq, nk, d, scale,
+                                    window_left, window_right, first, stream)
 
 
 def attn_bwd_prepare(o, dO, lse, B, H, nq, d, dtype, deterministic, workspace, ws_bytes,
@@ -289,6 +298,24 @@ def forward(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None, 
                           float(scale), int(bool(causal)), _dtype_code(q), _stream_handle(stream))
     _check(rc, "attn_fwd")
     return out, lse
+
+
+def forward_accumulate(q, k, v, o_acc, lse_acc, first=False, causal=False, scale=None,
+                       window=None, stream=None):
+    """Fold attention of q (bf16) over the keys k, v into the running fp32 o_acc (q's shape) and
+    lse_acc ((B, H, nq), natural log) in place (attn_fwd_accumulate); first=True initialises
+    them. Masks as `forward`."""
+    import torch
+    B, H, n, d = _dims(q)
+    Hkv, nk = _kv_heads(q, k, v)
+    if o_acc.shape != q.shape or o_acc.dtype != torch.float32 or lse_acc.dtype != torch.float32:
+        raise ValueError("o_acc must be fp32 with q's shape, lse_acc fp32 (B, H, nq)")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    wl, wr = _window(causal, window)
+    rc = attn_fwd_accumulate(_ptr(q), _ptr(k), _ptr(v), _ptr(o_acc), _ptr(lse_acc), B, H, Hkv, n,
+                             nk, d, float(scale), wl, wr, int(bool(first)), _stream_handle(stream))
+    _check(rc, "attn_fwd_accumulate")
 
 
 def backward(q, k, v, o, do, lse, causal=False, scale=None, deterministic=False, dq=None,

@@ -212,6 +212,28 @@ int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse
                     stream);
 }
 
+int attn_fwd_accumulate(const void* q, const void* k, const void* v, float* o_acc, float* lse_acc,
+                        int B, int H, int Hkv, int nq, int nk, int d, float scale,
+                        int window_left, int window_right, int first, void* stream) {
+    if (!q || !k || !v || !o_acc || !lse_acc) return ATTN_ERR_INVALID;
+    int rc = validate_common(B, H, nq, d, scale, ATTN_BF16);
+    if (rc) return rc;
+    if (nk < 1 || nk > kMaxSeq) return ATTN_ERR_INVALID;
+    if (Hkv < 1 || H % Hkv != 0) return ATTN_ERR_INVALID;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o_acc) || !aligned16(lse_acc))
+        return ATTN_ERR_INVALID;
+    FwdArgs a;
+    a.q = q; a.k = k; a.v = v; a.o = o_acc; a.lse = lse_acc;
+    a.B = B; a.H = H; a.nq = nq; a.nk = nk; a.d = d; a.Hkv = Hkv;
+    a.scale = scale;
+    a.wl = window_left < 0 ? -1 : window_left;
+    a.wr = window_right < 0 ? -1 : window_right;
+    a.q_descale = a.k_descale = a.v_descale = 1.f;
+    a.timeout_ns = static_cast<uint64_t>(g_timeout_us.load()) * 1000ull;
+    a.acc_first = first ? 1 : 0;
+    return to_code(launch_fwd_bf16(a, static_cast<cudaStream_t>(stream)));
+}
+
 int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                  int Hkv, int nq, int nk, int d, float scale, int window_left, int window_right,
                  float q_descale, float k_descale, float v_descale, void* stream) {

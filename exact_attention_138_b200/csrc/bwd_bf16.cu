@@ -645,17 +645,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     tmem_ld_wait();
                     if constexpr (ACC) {
                         if (kidx < nk) add_row_f32<16>((which == 0 ? acc.dv : acc.dk) + orow + cc, u, mul);
-                        continue;
-                    }
-                    uint32_t w[8];
+                    } else {
+                        uint32_t w[8];
 #pragma unroll
-                    for (int x = 0; x < 8; ++x)
-                        w[x] = pack_bf16x2(__uint_as_float(u[2 * x]) * mul,
-                                           __uint_as_float(u[2 * x + 1]) * mul);
-                    if (kidx < nk) {
-                        uint4* o = reinterpret_cast<uint4*>(dst + cc);
-                        o[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                        o[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                        for (int x = 0; x < 8; ++x)
+                            w[x] = pack_bf16x2(__uint_as_float(u[2 * x]) * mul,
+                                               __uint_as_float(u[2 * x + 1]) * mul);
+                        if (kidx < nk) {
+                            uint4* o = reinterpret_cast<uint4*>(dst + cc);
+                            o[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                            o[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                        }
                     }
                 }
             }
@@ -1157,18 +1157,18 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
                     reg_fence<32>(u);
                     if constexpr (ACC) {
                         if (kidx < nk) add_row_f32<32>((which == 0 ? acc.dv : acc.dk) + orow + cc, u, mul);
-                        continue;
-                    }
-                    uint32_t w[16];
+                    } else {
+                        uint32_t w[16];
 #pragma unroll
-                    for (int c = 0; c < 16; ++c)
-                        w[c] = pack_bf16x2(__uint_as_float(u[2 * c]) * mul,
-                                           __uint_as_float(u[2 * c + 1]) * mul);
-                    if (kidx < nk) {
-                        uint4* o = reinterpret_cast<uint4*>(dst + cc);
+                        for (int c = 0; c < 16; ++c)
+                            w[c] = pack_bf16x2(__uint_as_float(u[2 * c]) * mul,
+                                               __uint_as_float(u[2 * c + 1]) * mul);
+                        if (kidx < nk) {
+                            uint4* o = reinterpret_cast<uint4*>(dst + cc);
 #pragma unroll
-                        for (int c = 0; c < 4; ++c)
-                            o[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+                            for (int c = 0; c < 4; ++c)
+                                o[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+                        }
                     }
                 }
             }

@@ -131,10 +131,14 @@ __device__ __forceinline__ void store_p(uint32_t* u, int c, float p0, float p1) 
 // SPLIT: the CTAs of a cluster share the key tiles of one tile pair (small grids); each keeps its
 // unnormalised O and (m, l) for its share, and the cluster merges them through distributed
 // shared memory with the rule that joins two softmax blocks (weights 2^(m_s - M)).
-template <int D, bool F8, bool SPLIT>
+// ACC: p.o and p.lse are a running fp32 result (o_acc, and lse_acc in natural log) over earlier
+// key sets, into which this launch folds its own (acc_first: initialised instead of read).
+template <int D, bool F8, bool SPLIT, bool ACC = false>
 __device__ __forceinline__ void fwd_body(const CUtensorMap* tmQ_, const CUtensorMap* tmK_,
-                                         const CUtensorMap* tmV_, const FwdKParams& p) {
+                                         const CUtensorMap* tmV_, const FwdKParams& p,
+                                         int acc_first = 0) {
     using C = FwdCfg<D, F8>;
+    static_assert(!(ACC && (F8 || SPLIT)), "accumulating launches: bf16 without key split");
     const CUtensorMap& tmQ = *tmQ_;
     const CUtensorMap& tmK = *tmK_;
     const CUtensorMap& tmV = *tmV_;
@@ -598,6 +602,63 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap* tmQ_, const CUtensor
                         Lsum > 0.f ? (M + __log2f(Lsum)) * kLn2 : -INFINITY;
             }
             cluster_sync_all();   // peers may still be reading this CTA's shared memory
+        } else if constexpr (ACC) {
+            // Fold this launch's rows into the running result: with la the running LSE and lb
+            // this launch's (natural log, -inf where no key was seen), L = log(e^la + e^lb),
+            // o_acc = e^(la-L)·o_acc + e^(lb-L)·O/l, lse_acc = L; acc_first: la = -inf.
+            float* oacc = static_cast<float*>(p.o) + (static_cast<size_t>(bh) * nq + qidx) * D;
+            const bool row = qidx < nq;
+            float a[D];                                 // running row, loaded before O is ready
+            if (row && !acc_first) {
+#pragma unroll
+                for (int x = 0; x < D / 4; ++x) {
+                    const float4 t = reinterpret_cast<const float4*>(oacc)[x];
+                    a[4 * x] = t.x; a[4 * x + 1] = t.y; a[4 * x + 2] = t.z; a[4 * x + 3] = t.w;
+                }
+            }
+            const bool have = ok && T[g] > 0;
+            if (have) {
+                ok = bounded_wait(&bars->o_done[g], 0, abort, lim);
+                ok = __all_sync(0xffffffffu, ok);
+            }
+            if (ok && have) tc_fence_after();
+            const bool seen = ok && have && l > 0.f;
+            const float lb = seen ? (m + __log2f(l)) * kLn2 : -INFINITY;
+            const float la = (!row || acc_first) ? -INFINITY : p.lse[static_cast<size_t>(bh) * nq + qidx];
+            const float mx = fmaxf(la, lb);
+            float L = -INFINITY, wa = 0.f, wb = 0.f;
+            if (mx != -INFINITY) {
+                const float ea = expf(la - mx), eb = expf(lb - mx);
+                L = mx + logf(ea + eb);
+                wa = ea / (ea + eb);
+                wb = seen ? eb / (ea + eb) / l : 0.f;   // includes the 1/l of O/l
+            }
+            if (ok && (have || acc_first)) {
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t u[32];
+                    if (have) {
+                        tmem_ld32(tO + c * 32, u);
+                        tmem_ld_wait();
+                    }
+                    if (row) {
+                        float4* dst = reinterpret_cast<float4*>(oacc + c * 32);
+#pragma unroll
+                        for (int x = 0; x < 8; ++x) {
+                            float v4[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int k = c * 32 + 4 * x + e;
+                                const float pa = (wa == 0.f || acc_first) ? 0.f : wa * a[k];
+                                const float pb = wb == 0.f ? 0.f : wb * __uint_as_float(u[4 * x + e]);
+                                v4[e] = pa + pb;
+                            }
+                            dst[x] = make_float4(v4[0], v4[1], v4[2], v4[3]);
+                        }
+                    }
+                }
+                if (row) p.lse[static_cast<size_t>(bh) * nq + qidx] = L;
+            }
         } else if (ok && T[g] > 0) {
             ok = bounded_wait(&bars->o_done[g], 0, abort, lim);
             ok = __all_sync(0xffffffffu, ok);
@@ -652,6 +713,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdKParams p) {
     fwd_body<D, false, false>(&tmQ, &tmK, &tmV, p);
+}
+
+// Folds its result into a running fp32 (o_acc, lse_acc) over earlier key sets (see fwd_body).
+template <int D>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    fwd_bf16_acc_kernel(const __grid_constant__ CUtensorMap tmQ,
+                        const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const FwdKParams p, int first) {
+    fwd_body<D, false, false, true>(&tmQ, &tmK, &tmV, p, first);
 }
 
 // Small grids: launched in clusters of p.split CTAs that share each tile pair's key tiles.
@@ -801,6 +871,18 @@ cudaError_t launch_fwd_d(const FwdArgs& a, cudaStream_t stream) {
     kp.o_scale = F8 ? a.v_descale : 1.f;
     kp.timeout_ns = a.timeout_ns;
     const long long pairs_total = static_cast<long long>(kp.n_pairs) * BH;
+    if constexpr (!F8) {
+        if (a.acc_first >= 0) {      // accumulating launch: one CTA per tile pair
+            kp.split = 1;
+            if (pairs_total > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+            constexpr auto akern = fwd_bf16_acc_kernel<D>;
+            e = cudaFuncSetAttribute(akern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+            if (e != cudaSuccess) return e;
+            akern<<<static_cast<unsigned>(pairs_total), kFwdThreads, C::SMEM, stream>>>(
+                mq, mk, mv, kp, a.acc_first);
+            return cudaGetLastError();
+        }
+    }
     kp.split = choose_fwd_split<D, F8>(kp.mask, qtiles, pairs_total, stream);
     const long long grid = pairs_total * kp.split;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;

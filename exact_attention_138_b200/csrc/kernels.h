@@ -85,6 +85,9 @@ struct FwdArgs {
     int wl, wr;       // visible window (see MaskSpec)
     float q_descale, k_descale, v_descale;   // E4M3 inputs only: real value = stored · descale
     uint64_t timeout_ns;
+    // >= 0: o and lse are a running fp32 result (o_acc, lse_acc) that the launch folds its own
+    // into (bf16 inputs); 1: the first such launch (initialise, do not read)
+    int acc_first = -1;
 };
 
 struct BwdArgs {

@@ -16,10 +16,10 @@ locally (in the fp32 sum of the query chunk's backward workspace), and the fp32 
 accumulators travel with their chunks, are added to in place by every hop, and arrive back at
 their owner after the last hop.
 
-Every arithmetic step runs in the library's CUDA kernels (attn_fwd_ex and attn_ring_merge per
-chunk pair forward; attn_bwd_prepare once per query chunk, attn_bwd_accumulate per chunk pair and
-attn_bwd_finish at the end backward; attn_ring_accumulate for the final conversions); this module
-only schedules them and
+Every arithmetic step runs in the library's CUDA kernels: forward, attn_fwd_accumulate per
+chunk pair (it folds the pair into the running result inside the forward kernel); backward,
+attn_bwd_prepare once per query chunk, attn_bwd_accumulate per chunk pair and attn_bwd_finish at
+the end; attn_ring_accumulate for the final conversions. This module only schedules them and
 moves chunks with torch.distributed point-to-point operations (NCCL on GPUs), which run on NCCL's
 stream and overlap the current hop's kernels. `ring_forward_emulated` / `ring_backward_emulated`
 run the same schedule for N ranks inside one process (chunks are indexed instead of sent), which
@@ -96,6 +96,16 @@ class CudaOps:
     def merge(self, o_acc, lse_acc, o_part, lse_part, first, out):
         self.ea.ring_merge(o_acc, lse_acc, o_part, lse_part, first=first, out=out)
 
+    def fwd_fold(self, o_acc, lse_acc, first, q, k, v, scale, window, slot=0):
+        """Fold one chunk pair into the running (o_acc, lse_acc): inside the forward kernel for
+        bf16 inputs, else a forward into this slot's buffers and a merge."""
+        if q.dtype == torch.bfloat16:
+            self.ea.forward_accumulate(q, k, v, o_acc, lse_acc, first=first, scale=scale,
+                                       window=window)
+            return
+        o_p, l_p = self.fwd(q, k, v, scale, window, slot)
+        self.merge(o_acc, lse_acc, o_p, l_p, first, None)
+
     def accumulate(self, acc, part, first, out):
         self.ea.ring_accumulate(acc, part, first=first, out=out)
 
@@ -139,9 +149,8 @@ def _fwd_hop(ops, states, qs, q_ids, kvs, kv_ids, causal, scale, slot=0):
             w = hop_window(q_ids[qi], kv_ids[ki], causal)
             if w is None:
                 continue
-            o_p, l_p = ops.fwd(q, k, v, scale, w, slot)
             st = states[qi]
-            ops.merge(st.o_acc, st.lse, o_p, l_p, st.first, None)
+            ops.fwd_fold(st.o_acc, st.lse, st.first, q, k, v, scale, w, slot)
             st.first = False
 
 

@@ -84,6 +84,22 @@ int attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* ls
                  int B, int H, int Hkv, int n, int d, float scale, int causal, int dtype,
                  void* stream);
 
+/* Forward pass over one key set folded into a running result over earlier key sets (ring
+ * attention: one call per hop; "Attention Mechanism: Revolusi Representasi Sequence", §16 "Long
+ * Context Training", Ring Attention). The launch computes this key set's O_b, LSE_b exactly as
+ * attn_fwd_ex (q, k, v bf16; same shapes and masks) and, in the same kernel, combines them with
+ * the running o_acc (B, H, nq, d) fp32 and lse_acc (B, H, nq) fp32 (natural log), row by row:
+ *     L = log(exp(lse_acc) + exp(LSE_b)),
+ *     o_acc = exp(lse_acc - L)·o_acc + exp(LSE_b - L)·O_b,   lse_acc = L,
+ * which is exact because each result is normalised by its own exp(LSE) (the rule of
+ * attn_ring_merge, without the rounding of O_b to bf16). first != 0: o_acc and lse_acc are not
+ * read (they are set to this key set's result). A row that sees no key in any call so far has
+ * o_acc = 0, lse_acc = -inf. Errors as attn_fwd_ex; null or misaligned (16-byte) o_acc / lse_acc
+ * -> ATTN_ERR_INVALID. */
+int attn_fwd_accumulate(const void* q, const void* k, const void* v, float* o_acc, float* lse_acc,
+                        int B, int H, int Hkv, int nq, int nk, int d, float scale,
+                        int window_left, int window_right, int first, void* stream);
+
 /* FP8 forward pass ("Flash Attention Nedir?" and "Apa itu FlashAttention": FlashAttention-3 runs
  * the method in FP8 on Hopper). q, k, v hold E4M3 bytes (OCP FP8 E4M3: 1 sign, 4 exponent bits
  * with bias 7, 3 mantissa bits, no infinities, max 448) in the layouts of attn_fwd_ex; the real

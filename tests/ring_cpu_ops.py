@@ -70,6 +70,10 @@ class CpuOps:
         if out is not None:
             out.copy_(torch.from_numpy(o))
 
+    def fwd_fold(self, o_acc, lse_acc, first, q, k, v, scale, window, slot=0):
+        o_p, l_p = self.fwd(q, k, v, scale, window)
+        self.merge(o_acc, lse_acc, o_p, l_p, first, None)
+
     def accumulate(self, acc, part, first, out):
         a = np.zeros(acc.shape) if first else _np(acc)
         if part is not None:

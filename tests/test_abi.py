@@ -212,3 +212,20 @@ def _parts(which, **kw):
 ])
 def test_backward_parts_reject_bad_arguments(which, kw, code):
     assert _parts(which, **kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(o_acc=0), ea.ATTN_ERR_INVALID),
+    (dict(lse_acc=FAKE + 4), ea.ATTN_ERR_INVALID),
+    (dict(nk=0), ea.ATTN_ERR_INVALID),
+    (dict(Hkv=3), ea.ATTN_ERR_INVALID),
+    (dict(d=96), ea.ATTN_ERR_UNSUPPORTED),
+    (dict(scale=0.0), ea.ATTN_ERR_INVALID),
+])
+def test_forward_accumulate_rejects_bad_arguments(kw, code):
+    a = dict(B=1, H=2, Hkv=1, nq=300, nk=500, d=128, scale=0.1)
+    a.update(kw)
+    P = lambda name: ctypes.c_void_p(kw.get(name, FAKE))
+    assert ea.attn_fwd_accumulate(P("q"), P("k"), P("v"), P("o_acc"), P("lse_acc"), a["B"], a["H"],
+                                  a["Hkv"], a["nq"], a["nk"], a["d"], a["scale"], -1, 0, 1,
+                                  None) == code
