@@ -448,8 +448,10 @@ def time_variants(args, w, ea, q, k, v, do, ws, stream, causal_flops):
                                     zigzag=True, ops=ops)
     ms = timed(ring_step)
     out["ring_zigzag_4"] = {"ms": ms, "tflops": causal_flops / (ms * 1e-3) / 1e12,
-                            "config": "4 ranks emulated on one GPU (all ranks' hops in turn), "
-                                      "zigzag chunks of 1024 rows; same FLOPs as the bench step"}
+                            "config": "4 ranks emulated on one GPU, each on its own CUDA "
+                                      "stream (hop r+1 of rank p waits for hop r of rank p-1), "
+                                      "zigzag chunks of 1024 rows, one launch per hop; same "
+                                      "FLOPs as the bench step"}
     return out
 
 

@@ -67,13 +67,13 @@ _lib.attn_bwd.restype = _i
 _lib.attn_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i,
                           _i, _i, _vp, _sz, _vp]
 _lib.attn_fwd_accumulate.restype = _i
-_lib.attn_fwd_accumulate.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i, _i,
-                                     _i, _vp]
+_lib.attn_fwd_accumulate.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _ll, _ll, _f,
+                                     _i, _i, _i, _vp]
 _lib.attn_bwd_prepare.restype = _i
 _lib.attn_bwd_prepare.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]
 _lib.attn_bwd_accumulate.restype = _i
-_lib.attn_bwd_accumulate.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _f, _i,
-                                     _i, _i, _i, _vp, _sz, _vp]
+_lib.attn_bwd_accumulate.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _ll,
+                                     _ll, _i, _i, _f, _i, _i, _i, _i, _vp, _sz, _vp]
 _lib.attn_bwd_finish.restype = _i
 _lib.attn_bwd_finish.argtypes = [_vp, _i, _i, _i, _i, _f, _i, _i, _vp, _sz, _vp]
 _lib.attn_get_device_status.restype = _i
@@ -166,10 +166,10 @@ def attn_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, H, n, d, scale, causal, dtype, 
                          deterministic, workspace, ws_bytes, stream)
 
 
-def attn_fwd_accumulate(q, k, v, o_acc, lse_acc, B, H, Hkv, nq, nk, d, scale, window_left,
-                        window_right, first, stream) -> int:
-    return _lib.attn_fwd_accumulate(q, k, v, o_acc, lse_acc, B, H, Hkv, nq, nk, d, scale,
-                                    window_left, window_right, first, stream)
+def attn_fwd_accumulate(q, k, v, o_acc, lse_acc, B, H, Hkv, nq, nk, d, q_head_rows,
+                        kv_head_rows, scale, window_left, window_right, first, stream) -> int:
+    return _lib.attn_fwd_accumulate(q, k, v, o_acc, lse_acc, B, H, Hkv, nq, nk, d, q_head_rows,
+                                    kv_head_rows, scale, window_left, window_right, first, stream)
 
 
 def attn_bwd_prepare(o, dO, lse, B, H, nq, d, dtype, deterministic, workspace, ws_bytes,
@@ -178,9 +178,11 @@ def attn_bwd_prepare(o, dO, lse, B, H, nq, d, dtype, deterministic, workspace, w
                                  ws_bytes, stream)
 
 
-def attn_bwd_accumulate(q, k, v, dO, dk_acc, dv_acc, B, H, Hkv, nq, nk, d, scale, window_left,
-                        window_right, dtype, deterministic, workspace, ws_bytes, stream) -> int:
-    return _lib.attn_bwd_accumulate(q, k, v, dO, dk_acc, dv_acc, B, H, Hkv, nq, nk, d, scale,
+def attn_bwd_accumulate(q, k, v, dO, dk_acc, dv_acc, B, H, Hkv, nq, nk, d, q_head_rows,
+                        kv_head_rows, ws_rows, q_row0, scale, window_left, window_right, dtype,
+                        deterministic, workspace, ws_bytes, stream) -> int:
+    return _lib.attn_bwd_accumulate(q, k, v, dO, dk_acc, dv_acc, B, H, Hkv, nq, nk, d,
+                                    q_head_rows, kv_head_rows, ws_rows, q_row0, scale,
                                     window_left, window_right, dtype, deterministic, workspace,
                                     ws_bytes, stream)
 
@@ -238,6 +240,29 @@ def _stream_handle(stream):
     import torch
     s = stream if stream is not None else torch.cuda.current_stream()
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def _head_rows(*ts):
+    """Rows between consecutive heads shared by (B, H, n, d) tensors / (B, H, n) row vectors that
+    may be views of rows of longer sequences (0 when packed); raises for other layouts."""
+    rows = None
+    for t in ts:
+        if t.dim() == 4:
+            B, H, n, d = t.shape
+            ok = t.stride(3) == 1 and t.stride(2) == d and t.stride(1) % d == 0
+            r = t.stride(1) // d if ok else -1
+            ok = ok and (B == 1 or t.stride(0) == H * t.stride(1))
+        else:
+            B, H, n = t.shape
+            r = t.stride(1)
+            ok = t.stride(2) == 1 and (B == 1 or t.stride(0) == H * r)
+        if H == 1 and B == 1:
+            r = n if rows is None else rows
+        if not ok or r < n or (rows is not None and r != rows):
+            raise ValueError("expected packed (B, H, n, d) tensors or views of rows of a longer "
+                             "sequence with one layout")
+        rows = r
+    return 0 if rows is None or rows == ts[0].shape[2] else rows
 
 
 def _check(rc, where):
@@ -313,8 +338,10 @@ def forward_accumulate(q, k, v, o_acc, lse_acc, first=False, causal=False, scale
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     wl, wr = _window(causal, window)
+    q_rows, kv_rows = _head_rows(q, o_acc, lse_acc), _head_rows(k, v)
     rc = attn_fwd_accumulate(_ptr(q), _ptr(k), _ptr(v), _ptr(o_acc), _ptr(lse_acc), B, H, Hkv, n,
-                             nk, d, float(scale), wl, wr, int(bool(first)), _stream_handle(stream))
+                             nk, d, q_rows, kv_rows, float(scale), wl, wr, int(bool(first)),
+                             _stream_handle(stream))
     _check(rc, "attn_fwd_accumulate")
 
 
@@ -377,8 +404,10 @@ class BackwardSum:
         _check(rc, "attn_bwd_prepare")
 
     def add(self, q, k, v, do, dk_acc, dv_acc, scale=None, causal=False, window=None,
-            stream=None):
-        """dQ sum += and dk_acc, dv_acc (fp32, k's shape) += the gradients over keys k, v."""
+            stream=None, q_row0=0):
+        """dQ sum += and dk_acc, dv_acc (fp32, k's shape) += the gradients over keys k, v. q, dO
+        may be rows [q_row0, q_row0 + nq) of the queries (views of them), k, v, dk_acc, dv_acc
+        views of rows of longer key sequences."""
         Hkv, nk = _kv_heads(q, k, v)
         for t in (dk_acc, dv_acc):
             if t.shape != k.shape or t.dtype.itemsize != 4 or not t.is_floating_point():
@@ -386,10 +415,12 @@ class BackwardSum:
         if scale is None:
             scale = 1.0 / math.sqrt(self.d)
         wl, wr = _window(causal, window)
+        nq = q.shape[2]
+        q_rows, kv_rows = _head_rows(q, do), _head_rows(k, v, dk_acc, dv_acc)
         rc = attn_bwd_accumulate(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dk_acc), _ptr(dv_acc),
-                                 self.B, self.H, Hkv, self.n, nk, self.d, float(scale), wl, wr,
-                                 _dtype_code(q), self.det, _ptr(self.ws), self.ws.numel(),
-                                 _stream_handle(stream))
+                                 self.B, self.H, Hkv, nq, nk, self.d, q_rows, kv_rows, self.n,
+                                 int(q_row0), float(scale), wl, wr, _dtype_code(q), self.det,
+                                 _ptr(self.ws), self.ws.numel(), _stream_handle(stream))
         _check(rc, "attn_bwd_accumulate")
 
     def finish(self, dq=None, scale=None, stream=None):

@@ -88,14 +88,16 @@ int validate_common(int B, int H, int n, int d, float scale, int dtype) {
 }  // namespace
 
 cudaError_t make_tmap(CUtensorMap* map, const void* base, int esize, int BH, int n, int d,
-                      int box_rows) {
+                      int box_rows, long long head_rows) {
+    if (head_rows <= 0) head_rows = n;
+    if (head_rows < n) return cudaErrorInvalidValue;
     auto fn = encode_fn();
     if (!fn) return cudaErrorNotSupported;
     const int chunk = d * esize >= 128 ? 128 / esize : d;
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n),
                           static_cast<cuuint64_t>(BH)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * esize,
-                             static_cast<cuuint64_t>(d) * esize * static_cast<cuuint64_t>(n)};
+                             static_cast<cuuint64_t>(d) * esize * static_cast<cuuint64_t>(head_rows)};
     cuuint32_t box[3] = {static_cast<cuuint32_t>(chunk), static_cast<cuuint32_t>(box_rows), 1u};
     cuuint32_t estr[3] = {1u, 1u, 1u};
     const int chunk_bytes = chunk * esize;
@@ -213,13 +215,17 @@ int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse
 }
 
 int attn_fwd_accumulate(const void* q, const void* k, const void* v, float* o_acc, float* lse_acc,
-                        int B, int H, int Hkv, int nq, int nk, int d, float scale,
-                        int window_left, int window_right, int first, void* stream) {
+                        int B, int H, int Hkv, int nq, int nk, int d, long long q_head_rows,
+                        long long kv_head_rows, float scale, int window_left, int window_right,
+                        int first, void* stream) {
     if (!q || !k || !v || !o_acc || !lse_acc) return ATTN_ERR_INVALID;
     int rc = validate_common(B, H, nq, d, scale, ATTN_BF16);
     if (rc) return rc;
     if (nk < 1 || nk > kMaxSeq) return ATTN_ERR_INVALID;
     if (Hkv < 1 || H % Hkv != 0) return ATTN_ERR_INVALID;
+    if ((q_head_rows != 0 && q_head_rows < nq) || (kv_head_rows != 0 && kv_head_rows < nk) ||
+        q_head_rows < 0 || kv_head_rows < 0 || q_head_rows > kMaxSeq || kv_head_rows > kMaxSeq)
+        return ATTN_ERR_INVALID;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o_acc) || !aligned16(lse_acc))
         return ATTN_ERR_INVALID;
     FwdArgs a;
@@ -231,6 +237,8 @@ int attn_fwd_accumulate(const void* q, const void* k, const void* v, float* o_ac
     a.q_descale = a.k_descale = a.v_descale = 1.f;
     a.timeout_ns = static_cast<uint64_t>(g_timeout_us.load()) * 1000ull;
     a.acc_first = first ? 1 : 0;
+    a.q_rows = q_head_rows;
+    a.kv_rows = kv_head_rows;
     return to_code(launch_fwd_bf16(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -361,6 +369,7 @@ int attn_bwd_prepare(const void* o, const void* dO, const float* lse, int B, int
 
 int attn_bwd_accumulate(const void* q, const void* k, const void* v, const void* dO,
                         float* dk_acc, float* dv_acc, int B, int H, int Hkv, int nq, int nk, int d,
+                        long long q_head_rows, long long kv_head_rows, int ws_rows, int q_row0,
                         float scale, int window_left, int window_right, int dtype,
                         int deterministic, void* workspace, size_t ws_bytes, void* stream) {
     if (!q || !k || !v || !dO || !dk_acc || !dv_acc) return ATTN_ERR_INVALID;
@@ -372,8 +381,16 @@ int attn_bwd_accumulate(const void* q, const void* k, const void* v, const void*
     const void* ptrs[] = {q, k, v, dO, dk_acc, dv_acc};
     for (const void* p : ptrs)
         if (!aligned16(p)) return ATTN_ERR_INVALID;
+    if (ws_rows == 0) ws_rows = nq;
+    if ((q_head_rows != 0 && q_head_rows < nq) || (kv_head_rows != 0 && kv_head_rows < nk) ||
+        q_head_rows < 0 || kv_head_rows < 0 || q_head_rows > kMaxSeq || kv_head_rows > kMaxSeq)
+        return ATTN_ERR_INVALID;
+    // the rows after this launch's last query tile are padding of the workspace, or there are none
+    if (ws_rows < 1 || ws_rows > kMaxSeq || q_row0 < 0 || q_row0 > ws_rows - nq ||
+        (q_row0 + nq != ws_rows && nq % 128 != 0))
+        return ATTN_ERR_INVALID;
     WsLayout w;
-    if ((rc = check_ws(workspace, ws_bytes, B, H, nq, d, deterministic, &w))) return rc;
+    if ((rc = check_ws(workspace, ws_bytes, B, H, ws_rows, d, deterministic, &w))) return rc;
     BwdArgs a = {};
     a.q = q; a.k = k; a.v = v; a.dO = dO;
     a.B = B; a.H = H; a.Hkv = Hkv; a.nq = nq; a.nk = nk; a.d = d;
@@ -385,6 +402,10 @@ int attn_bwd_accumulate(const void* q, const void* k, const void* v, const void*
     a.phases = 2;
     a.dk_acc32 = dk_acc;
     a.dv_acc32 = dv_acc;
+    a.q_rows = q_head_rows;
+    a.kv_rows = kv_head_rows;
+    a.ws_rows = ws_rows;
+    a.q_row0 = q_row0;
     return to_code(launch_bwd_bf16(a, static_cast<cudaStream_t>(stream)));
 }
 

@@ -80,6 +80,7 @@ struct BwdKParams {
 struct AccOut {
     float* dk;
     float* dv;
+    long long rows;   // rows between consecutive K/V heads of dk, dv
 };
 
 // dst[0 .. N) += mul · (TMEM words u as fp32); dst 16-byte aligned. Vector reductions performed
@@ -644,7 +645,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     tmem_ld16(tacc + cc, u);
                     tmem_ld_wait();
                     if constexpr (ACC) {
-                        if (kidx < nk) add_row_f32<16>((which == 0 ? acc.dv : acc.dk) + orow + cc, u, mul);
+                        if (kidx < nk)
+                            add_row_f32<16>((which == 0 ? acc.dv : acc.dk) +
+                                                (static_cast<size_t>(kvbh) * acc.rows + kidx) * D +
+                                                g * (D / 2) + cc,
+                                            u, mul);
                     } else {
                         uint32_t w[8];
 #pragma unroll
@@ -1156,7 +1161,11 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
                     tmem_ld_wait();
                     reg_fence<32>(u);
                     if constexpr (ACC) {
-                        if (kidx < nk) add_row_f32<32>((which == 0 ? acc.dv : acc.dk) + orow + cc, u, mul);
+                        if (kidx < nk)
+                            add_row_f32<32>((which == 0 ? acc.dv : acc.dk) +
+                                                (static_cast<size_t>(kvbh) * acc.rows + kidx) * D +
+                                                x * 64 + cc,
+                                            u, mul);
                     } else {
                         uint32_t w[16];
 #pragma unroll
@@ -1187,7 +1196,8 @@ template <int D>
 cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
     using C = BwdCfg<D>;
     const int BH = a.B * a.H;
-    const int n_pad = (a.nq + 127) / 128 * 128;
+    // query rows per head in the workspace (this launch's rows start at a.q_row0 within them)
+    const int n_pad = ((a.ws_rows > 0 ? a.ws_rows : a.nq) + 127) / 128 * 128;
     const int nkt = (a.nk + 127) / 128;
     const int nk_pad = nkt * 128;
     // Main-kernel CTAs run per K/V head. Heads per group: a K/V head's K and V (4·nk·d bytes) and
@@ -1224,13 +1234,14 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
             const size_t n_sems = static_cast<size_t>(BH) * (n_pad / 64) * 4;
             if ((e = cudaMemsetAsync(a.sems, 0, n_sems * sizeof(int), stream)) != cudaSuccess) return e;
         }
-        const AccOut acc{a.dk_acc32, a.dv_acc32};
+        const AccOut acc{a.dk_acc32, a.dv_acc32, a.kv_rows > 0 ? a.kv_rows : a.nk};
         BwdKParams kp;
         kp.lse = a.lse;
-        kp.Dvec = a.Dvec;
-        kp.L2vec = a.L2vec;
-        kp.dq_acc = a.dq_acc;
-        kp.sems = a.sems;
+        // the workspace rows of this launch's first query, in every head
+        kp.Dvec = a.Dvec + a.q_row0;
+        kp.L2vec = a.L2vec + a.q_row0;
+        kp.dq_acc = a.dq_acc + static_cast<size_t>(a.q_row0) * D;
+        kp.sems = a.sems ? a.sems + (a.q_row0 / 64) * 4 : nullptr;
         kp.dk = static_cast<__nv_bfloat16*>(a.dk);
         kp.dv = static_cast<__nv_bfloat16*>(a.dv);
         kp.n_pad = n_pad;
@@ -1247,13 +1258,14 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
         if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
         const int qbox = D == 128 ? q64::BQ : 128;
         CUtensorMap mq, mk, mv, mdo;
-        if ((e = make_tmap_bf16(&mq, a.q, BH, a.nq, D, qbox)) != cudaSuccess) return e;
-        if ((e = make_tmap_bf16(&mk, a.k, BHkv, a.nk, D)) != cudaSuccess) return e;
-        if ((e = make_tmap_bf16(&mv, a.v, BHkv, a.nk, D)) != cudaSuccess) return e;
-        if ((e = make_tmap_bf16(&mdo, a.dO, BH, a.nq, D, qbox)) != cudaSuccess) return e;
+        if ((e = make_tmap_bf16(&mq, a.q, BH, a.nq, D, qbox, a.q_rows)) != cudaSuccess) return e;
+        if ((e = make_tmap_bf16(&mk, a.k, BHkv, a.nk, D, 128, a.kv_rows)) != cudaSuccess) return e;
+        if ((e = make_tmap_bf16(&mv, a.v, BHkv, a.nk, D, 128, a.kv_rows)) != cudaSuccess) return e;
+        if ((e = make_tmap_bf16(&mdo, a.dO, BH, a.nq, D, qbox, a.q_rows)) != cudaSuccess) return e;
         if constexpr (D == 128) {
             CUtensorMap macc;   // the fp32 dQ accumulator as (B·H·n_pad) rows x 128 columns
-            if ((e = make_tmap_acc(&macc, a.dq_acc, static_cast<long long>(BH) * n_pad, D)) != cudaSuccess)
+            if ((e = make_tmap_acc(&macc, kp.dq_acc,
+                                   static_cast<long long>(BH) * n_pad - a.q_row0, D)) != cudaSuccess)
                 return e;
             const auto kern = acc.dk ? bwd_main_q64_kernel<true> : bwd_main_q64_kernel<false>;
             e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, q64::SMEM);

@@ -132,11 +132,12 @@ __device__ __forceinline__ void store_p(uint32_t* u, int c, float p0, float p1) 
 // unnormalised O and (m, l) for its share, and the cluster merges them through distributed
 // shared memory with the rule that joins two softmax blocks (weights 2^(m_s - M)).
 // ACC: p.o and p.lse are a running fp32 result (o_acc, and lse_acc in natural log) over earlier
-// key sets, into which this launch folds its own (acc_first: initialised instead of read).
+// key sets, into which this launch folds its own (acc_first: initialised instead of read); their
+// heads start acc_rows rows apart.
 template <int D, bool F8, bool SPLIT, bool ACC = false>
 __device__ __forceinline__ void fwd_body(const CUtensorMap* tmQ_, const CUtensorMap* tmK_,
                                          const CUtensorMap* tmV_, const FwdKParams& p,
-                                         int acc_first = 0) {
+                                         int acc_first = 0, long long acc_rows = 0) {
     using C = FwdCfg<D, F8>;
     static_assert(!(ACC && (F8 || SPLIT)), "accumulating launches: bf16 without key split");
     const CUtensorMap& tmQ = *tmQ_;
@@ -606,7 +607,8 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap* tmQ_, const CUtensor
             // Fold this launch's rows into the running result: with la the running LSE and lb
             // this launch's (natural log, -inf where no key was seen), L = log(e^la + e^lb),
             // o_acc = e^(la-L)·o_acc + e^(lb-L)·O/l, lse_acc = L; acc_first: la = -inf.
-            float* oacc = static_cast<float*>(p.o) + (static_cast<size_t>(bh) * nq + qidx) * D;
+            const size_t arow = static_cast<size_t>(bh) * acc_rows + qidx;
+            float* oacc = static_cast<float*>(p.o) + arow * D;
             const bool row = qidx < nq;
             float a[D];                                 // running row, loaded before O is ready
             if (row && !acc_first) {
@@ -624,7 +626,7 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap* tmQ_, const CUtensor
             if (ok && have) tc_fence_after();
             const bool seen = ok && have && l > 0.f;
             const float lb = seen ? (m + __log2f(l)) * kLn2 : -INFINITY;
-            const float la = (!row || acc_first) ? -INFINITY : p.lse[static_cast<size_t>(bh) * nq + qidx];
+            const float la = (!row || acc_first) ? -INFINITY : p.lse[arow];
             const float mx = fmaxf(la, lb);
             float L = -INFINITY, wa = 0.f, wb = 0.f;
             if (mx != -INFINITY) {
@@ -657,7 +659,7 @@ __device__ __forceinline__ void fwd_body(const CUtensorMap* tmQ_, const CUtensor
                         }
                     }
                 }
-                if (row) p.lse[static_cast<size_t>(bh) * nq + qidx] = L;
+                if (row) p.lse[arow] = L;
             }
         } else if (ok && T[g] > 0) {
             ok = bounded_wait(&bars->o_done[g], 0, abort, lim);
@@ -716,12 +718,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 }
 
 // Folds its result into a running fp32 (o_acc, lse_acc) over earlier key sets (see fwd_body).
+struct FwdAccP {
+    int first;
+    long long rows;   // rows between consecutive heads of o_acc and lse_acc
+};
+
 template <int D>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fwd_bf16_acc_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
-                        const __grid_constant__ CUtensorMap tmV, const FwdKParams p, int first) {
-    fwd_body<D, false, false, true>(&tmQ, &tmK, &tmV, p, first);
+                        const __grid_constant__ CUtensorMap tmV, const FwdKParams p,
+                        const FwdAccP acc) {
+    fwd_body<D, false, false, true>(&tmQ, &tmK, &tmV, p, acc.first, acc.rows);
 }
 
 // Small grids: launched in clusters of p.split CTAs that share each tile pair's key tiles.
@@ -844,10 +852,10 @@ cudaError_t launch_fwd_d(const FwdArgs& a, cudaStream_t stream) {
     const int BH = a.B * a.H;
     const int esize = F8 ? 1 : 2;
     cudaError_t e;
-    if ((e = make_tmap(&mq, a.q, esize, BH, a.nq, D)) != cudaSuccess) return e;
+    if ((e = make_tmap(&mq, a.q, esize, BH, a.nq, D, 128, a.q_rows)) != cudaSuccess) return e;
     const int BHkv = a.B * a.Hkv;
-    if ((e = make_tmap(&mk, a.k, esize, BHkv, a.nk, D)) != cudaSuccess) return e;
-    if ((e = make_tmap(&mv, a.v, esize, BHkv, a.nk, D)) != cudaSuccess) return e;
+    if ((e = make_tmap(&mk, a.k, esize, BHkv, a.nk, D, 128, a.kv_rows)) != cudaSuccess) return e;
+    if ((e = make_tmap(&mv, a.v, esize, BHkv, a.nk, D, 128, a.kv_rows)) != cudaSuccess) return e;
     void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const FwdKParams);
     if constexpr (F8) kern = fwd_fp8_kernel<D>;
     else kern = fwd_bf16_kernel<D>;
@@ -878,8 +886,9 @@ cudaError_t launch_fwd_d(const FwdArgs& a, cudaStream_t stream) {
             constexpr auto akern = fwd_bf16_acc_kernel<D>;
             e = cudaFuncSetAttribute(akern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
             if (e != cudaSuccess) return e;
+            const FwdAccP acc{a.acc_first, a.q_rows > 0 ? a.q_rows : a.nq};
             akern<<<static_cast<unsigned>(pairs_total), kFwdThreads, C::SMEM, stream>>>(
-                mq, mk, mv, kp, a.acc_first);
+                mq, mk, mv, kp, acc);
             return cudaGetLastError();
         }
     }

@@ -88,6 +88,9 @@ struct FwdArgs {
     // >= 0: o and lse are a running fp32 result (o_acc, lse_acc) that the launch folds its own
     // into (bf16 inputs); 1: the first such launch (initialise, do not read)
     int acc_first = -1;
+    // rows between consecutive heads of q (and, accumulating, of o_acc / lse_acc) and of k, v;
+    // 0: nq / nk (packed)
+    long long q_rows = 0, kv_rows = 0;
 };
 
 struct BwdArgs {
@@ -119,16 +122,22 @@ struct BwdArgs {
     int phases = 7;
     float* dk_acc32 = nullptr;
     float* dv_acc32 = nullptr;
+    // Views (main kernel only): rows between consecutive heads of q, dO and of k, v, dk_acc32,
+    // dv_acc32 (0: nq / nk); the workspace holds ws_rows query rows per head (0: nq) and this
+    // launch's queries are its rows [q_row0, q_row0 + nq) (q_row0 a multiple of 64).
+    long long q_rows = 0, kv_rows = 0;
+    int ws_rows = 0, q_row0 = 0;
 };
 
 // Encodes a 3-D tensor map over a (B*H, n, d) tensor of `esize`-byte elements (2: bf16, 1: 8-bit)
 // with a box of (chunk, box_rows, 1), chunk = min(d, 128 / esize) elements, and the swizzle that
-// matches the chunk's bytes (128: 128-byte, 64: 64-byte).
+// matches the chunk's bytes (128: 128-byte, 64: 64-byte). Consecutive heads start head_rows rows
+// apart (0: n, packed; a view of rows of a longer sequence otherwise).
 cudaError_t make_tmap(CUtensorMap* map, const void* base, int esize, int BH, int n, int d,
-                      int box_rows = 128);
+                      int box_rows = 128, long long head_rows = 0);
 inline cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int BH, int n, int d,
-                                  int box_rows = 128) {
-    return make_tmap(map, base, 2, BH, n, d, box_rows);
+                                  int box_rows = 128, long long head_rows = 0) {
+    return make_tmap(map, base, 2, BH, n, d, box_rows, head_rows);
 }
 
 // Encodes a 2-D tensor map over the fp32 dQ accumulator: `rows` rows of `d` fp32 values, box of

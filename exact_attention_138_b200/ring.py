@@ -8,18 +8,21 @@ Layouts. With N ranks the sequence is cut into equal chunks:
               after the other). Under a causal mask every rank then sees the same amount of work
               (the contiguous layout gives rank N-1 N times the work of rank 0).
 In hop r a rank attends its query chunks to the K/V chunks of rank (p - r) mod N, which arrived
-from rank p - 1, while sending the chunks it holds on to rank p + 1; the partial results of each
-query chunk are folded together with the log-sum-exp rule (attn_ring_merge). Under a causal mask
-a (query chunk, key chunk) pair is unmasked (earlier key chunk), causal (same chunk) or skipped
-(later key chunk). The backward pass walks the same ring with the final O and LSE: dQ accumulates
-locally (in the fp32 sum of the query chunk's backward workspace), and the fp32 dK / dV
-accumulators travel with their chunks, are added to in place by every hop, and arrive back at
-their owner after the last hop.
+from rank p - 1, while sending the chunks it holds on to rank p + 1; the partial results are
+folded together with the log-sum-exp rule (attn_ring_merge). Under a causal mask a (query chunk,
+key chunk) pair is unmasked (earlier key chunk), causal (same chunk) or skipped (later key
+chunk). The visible pairs of a hop are joined into as few launches as the masks allow, each on
+row ranges (views) of the rank's whole tensors: with zigzag chunks every hop is one launch (the
+rank's own chunks: the causal mask of their concatenation; an earlier rank's: all queries
+against its first chunk; a later rank's: the second query chunk against both). The backward
+pass walks the same ring with the final O and LSE: dQ accumulates locally (in the fp32 sum of
+the rank's backward workspace), and the fp32 dK / dV accumulators travel with their chunks, are
+added to in place by every hop, and arrive back at their owner after the last hop.
 
 Every arithmetic step runs in the library's CUDA kernels: forward, attn_fwd_accumulate per
-chunk pair (it folds the pair into the running result inside the forward kernel); backward,
-attn_bwd_prepare once per query chunk, attn_bwd_accumulate per chunk pair and attn_bwd_finish at
-the end; attn_ring_accumulate for the final conversions. This module only schedules them and
+launch (it folds the launch into the running result inside the forward kernel); backward,
+attn_bwd_prepare once per rank, attn_bwd_accumulate per launch and attn_bwd_finish at the end;
+attn_ring_accumulate for the final conversions. This module only schedules them and
 moves chunks with torch.distributed point-to-point operations (NCCL on GPUs), which run on NCCL's
 stream and overlap the current hop's kernels. `ring_forward_emulated` / `ring_backward_emulated`
 run the same schedule for N ranks inside one process (chunks are indexed instead of sent), which
@@ -48,34 +51,51 @@ def rank_chunks(rank: int, world: int, zigzag: bool):
     return [rank, 2 * world - 1 - rank] if zigzag else [rank]
 
 
+def hop_launches(q_ids, kv_ids, causal):
+    """The launches of one hop, as (first query chunk, end, first key chunk, end, window) over the
+    rank's chunk order: the visible (query chunk, key chunk) pairs, joined into one launch when
+    they form the causal mask of the concatenated chunks or a block with no mask, else one
+    launch per pair."""
+    W = [[hop_window(a, b, causal) for b in kv_ids] for a in q_ids]
+    full = (-1, -1)
+    if causal and q_ids == kv_ids and q_ids == sorted(q_ids):
+        return [(0, len(q_ids), 0, len(kv_ids), (-1, 0))]
+    rows = [a for a in range(len(q_ids)) if any(w is not None for w in W[a])]
+    cols = [b for b in range(len(kv_ids)) if any(W[a][b] is not None for a in range(len(q_ids)))]
+    if (rows and rows == list(range(rows[0], rows[-1] + 1))
+            and cols == list(range(cols[0], cols[-1] + 1))
+            and all(W[a][b] == full for a in rows for b in cols)):
+        return [(rows[0], rows[-1] + 1, cols[0], cols[-1] + 1, full)]
+    return [(a, a + 1, b, b + 1, W[a][b]) for a in range(len(q_ids)) for b in range(len(kv_ids))
+            if W[a][b] is not None]
+
+
 class CudaOps:
-    """The per-chunk-pair operations, all in libattn.so. One set of per-hop forward output buffers
-    is reused by every hop (each partial is merged on the same stream before the next hop
-    overwrites it), and one backward workspace per query chunk (keyed by the caller) is kept for
-    the next pass of the same sizes, so an instance passed to every step allocates nothing after
-    the first."""
+    """The per-hop operations, all in libattn.so: the forward folded into a running result, and
+    the backward in parts (one workspace per rank, kept for the next pass of the same sizes, so
+    an instance passed to every step allocates nothing after the first)."""
 
     def __init__(self):
         import exact_attention_138_b200 as ea
         self.ea = ea
-        self._bufs = {}
         self._sums = {}
 
-    def _buf(self, key, shape, dtype, device):
-        t = self._bufs.get(key)
-        if t is None or tuple(t.shape) != tuple(shape) or t.dtype != dtype or t.device != device:
-            t = torch.empty(shape, dtype=dtype, device=device)
-            self._bufs[key] = t
-        return t
-
-    def fwd(self, q, k, v, scale, window, slot=0):
-        """O and LSE of one chunk pair, in buffers of `slot` (one per concurrent caller)."""
-        o = self._buf(("o", slot), q.shape, q.dtype, q.device)
-        lse = self._buf(("lse", slot), q.shape[:-1], torch.float32, q.device)
-        return self.ea.forward(q, k, v, scale=scale, window=window, out=o, lse=lse)
+    def fwd_fold(self, o_acc, lse_acc, first, q, k, v, scale, window, slot=0):
+        """Fold attention of q over k, v into the running (o_acc, lse_acc) (views allowed)."""
+        if q.dtype == torch.bfloat16:
+            self.ea.forward_accumulate(q, k, v, o_acc, lse_acc, first=first, scale=scale,
+                                       window=window)
+            return
+        # other input types: a forward on copies and a merge into copies of the running rows
+        o_p, l_p = self.ea.forward(q.contiguous(), k.contiguous(), v.contiguous(), scale=scale,
+                                   window=window)
+        oa, la = o_acc.contiguous(), lse_acc.contiguous()
+        self.ea.ring_merge(oa, la, o_p, l_p, first=first)
+        o_acc.copy_(oa)
+        lse_acc.copy_(la)
 
     def bwd_begin(self, key, o, do, lse, deterministic):
-        """Backward state of one query chunk (o, dO, lse of the whole forward pass)."""
+        """Backward state of the rank's queries (o, dO, lse of the whole forward pass)."""
         st = self._sums.get(key)
         if (st is None or st.det != int(bool(deterministic)) or st.ws.device != o.device
                 or (st.B, st.H, st.n, st.d) != tuple(o.shape)):
@@ -85,26 +105,13 @@ class CudaOps:
             st.reset(o, do, lse)
         return st
 
-    def bwd_add(self, st, q, k, v, do, dkv_acc, scale, window):
-        """dQ sum of `st` and dkv_acc (fp32 (2, B, Hkv, n_k, d): dK, dV) += this pair's part."""
-        st.add(q, k, v, do, dkv_acc[0], dkv_acc[1], scale=scale, window=window)
+    def bwd_add(self, st, q, k, v, do, dk_acc, dv_acc, scale, window, q_row0):
+        """dQ sum of `st` (its rows from q_row0) and dk_acc, dv_acc += this launch's part."""
+        st.add(q, k, v, do, dk_acc, dv_acc, scale=scale, window=window, q_row0=q_row0)
 
     def bwd_finish(self, st, out, scale):
-        """Writes dQ of `st` into `out` (the query chunk's dtype and shape) and returns it."""
+        """Writes dQ of `st` into `out` and returns it."""
         return st.finish(out, scale=scale)
-
-    def merge(self, o_acc, lse_acc, o_part, lse_part, first, out):
-        self.ea.ring_merge(o_acc, lse_acc, o_part, lse_part, first=first, out=out)
-
-    def fwd_fold(self, o_acc, lse_acc, first, q, k, v, scale, window, slot=0):
-        """Fold one chunk pair into the running (o_acc, lse_acc): inside the forward kernel for
-        bf16 inputs, else a forward into this slot's buffers and a merge."""
-        if q.dtype == torch.bfloat16:
-            self.ea.forward_accumulate(q, k, v, o_acc, lse_acc, first=first, scale=scale,
-                                       window=window)
-            return
-        o_p, l_p = self.fwd(q, k, v, scale, window, slot)
-        self.merge(o_acc, lse_acc, o_p, l_p, first, None)
 
     def accumulate(self, acc, part, first, out):
         self.ea.ring_accumulate(acc, part, first=first, out=out)
@@ -114,71 +121,39 @@ def _scale(q, scale):
     return 1.0 / math.sqrt(q.shape[-1]) if scale is None else float(scale)
 
 
-def _wide(x):
-    """x viewed with 8-byte elements when its rows allow (copies then move 4x fewer elements)."""
-    if x.is_contiguous() and x.dim() == 4 and (x.shape[-1] * x.element_size()) % 8 == 0:
-        return x.view(torch.int64)
-    return x
+def _rows(x, lo, hi, c):
+    """Rows [lo·c, hi·c) of a (.., n, d) tensor or (.., n) vector: a view, no copy."""
+    return x[:, :, lo * c:hi * c]
 
 
-def _split(x, parts):
-    """The chunks of a rank's (B, H, parts·c, d) tensor as contiguous tensors."""
-    if parts == 1:
-        return [x.contiguous()]
-    w = _wide(x)
-    return [c.contiguous().view(x.dtype) for c in torch.chunk(w, parts, dim=2)]
+def _chunk_len(q, parts):
+    n = q.shape[2]
+    if n % parts:
+        raise ValueError("a zigzag rank holds two chunks of equal length")
+    return n // parts
 
 
-def _join(chunks):
-    if len(chunks) == 1:
-        return chunks[0]
-    return torch.cat([_wide(c) for c in chunks], dim=2).view(chunks[0].dtype)
+def _fwd_hop(ops, o_acc, lse_acc, init, q, k, v, q_ids, kv_ids, causal, scale, slot=0):
+    """Fold one hop into the rank's running (o_acc, lse_acc); init[a]: query chunk a has been
+    initialised by an earlier launch."""
+    c = _chunk_len(q, len(q_ids))
+    for a0, a1, b0, b1, w in hop_launches(q_ids, kv_ids, causal):
+        first = not init[a0]
+        if any(init[a] != init[a0] for a in range(a0, a1)):
+            raise RuntimeError("a launch over query chunks in different states")
+        ops.fwd_fold(_rows(o_acc, a0, a1, c), _rows(lse_acc, a0, a1, c), first,
+                     _rows(q, a0, a1, c), _rows(k, b0, b1, c), _rows(v, b0, b1, c), scale, w,
+                     slot)
+        for a in range(a0, a1):
+            init[a] = True
 
 
-class _FwdState:
-    def __init__(self, q):
-        self.o_acc = torch.empty(q.shape, dtype=torch.float32, device=q.device)
-        self.lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
-        self.first = True
-
-
-def _fwd_hop(ops, states, qs, q_ids, kvs, kv_ids, causal, scale, slot=0):
-    """Fold every visible (query chunk, key chunk) pair of one hop into the running results."""
-    for qi, q in enumerate(qs):
-        for ki, (k, v) in enumerate(kvs):
-            w = hop_window(q_ids[qi], kv_ids[ki], causal)
-            if w is None:
-                continue
-            st = states[qi]
-            ops.fwd_fold(st.o_acc, st.lse, st.first, q, k, v, scale, w, slot)
-            st.first = False
-
-
-def _fwd_outputs(ops, states, qs):
-    outs = []
-    for st, q in zip(states, qs):
-        out = torch.empty_like(q)
-        ops.accumulate(st.o_acc, None, False, out)    # fp32 running output -> q's dtype
-        outs.append(out)
-    return _join(outs), _join([st.lse for st in states])
-
-
-def _bwd_hop(ops, sums, qs, q_ids, dos, kvs, kv_ids, dkv_acc, causal, scale):
-    for qi, q in enumerate(qs):
-        for ki, (k, v) in enumerate(kvs):
-            w = hop_window(q_ids[qi], kv_ids[ki], causal)
-            if w is None:
-                continue
-            ops.bwd_add(sums[qi], q, k, v, dos[qi], dkv_acc[ki], scale, w)
-
-
-def _convert(ops, accs, likes):
-    outs = []
-    for acc, like in zip(accs, likes):
-        out = torch.empty_like(like)
-        ops.accumulate(acc, None, False, out)
-        outs.append(out)
-    return _join(outs)
+def _bwd_hop(ops, st, q, do, k, v, dkv_acc, q_ids, kv_ids, causal, scale):
+    c = _chunk_len(q, len(q_ids))
+    for a0, a1, b0, b1, w in hop_launches(q_ids, kv_ids, causal):
+        ops.bwd_add(st, _rows(q, a0, a1, c), _rows(k, b0, b1, c), _rows(v, b0, b1, c),
+                    _rows(do, a0, a1, c), _rows(dkv_acc[0], b0, b1, c),
+                    _rows(dkv_acc[1], b0, b1, c), scale, w, a0 * c)
 
 
 def _peers(group):
@@ -204,23 +179,24 @@ def ring_forward(q, k, v, causal=False, scale=None, group=None, ops=None, zigzag
     ops = ops or CudaOps()
     scale = _scale(q, scale)
     rank, world, nxt, prv = _peers(group)
-    parts = 2 if zigzag else 1
     q_ids = rank_chunks(rank, world, zigzag)
-    qs = _split(q, parts)
-    states = [_FwdState(c) for c in qs]
-    cur = _split(k, parts) + _split(v, parts)          # k chunks, then v chunks
+    o_acc = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    lse_acc = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
+    init = [False] * len(q_ids)
+    cur = [k.contiguous(), v.contiguous()]
     for r in range(world):
         reqs = None
         if r < world - 1:
             nxt_kv, reqs = _exchange(cur, nxt, prv, group)
         kv_ids = rank_chunks((rank - r) % world, world, zigzag)
-        kvs = list(zip(cur[:parts], cur[parts:]))
-        _fwd_hop(ops, states, qs, q_ids, kvs, kv_ids, causal, scale)
+        _fwd_hop(ops, o_acc, lse_acc, init, q, cur[0], cur[1], q_ids, kv_ids, causal, scale)
         if reqs is not None:
             for req in reqs:
                 req.wait()
             cur = nxt_kv
-    return _fwd_outputs(ops, states, qs)
+    out = torch.empty_like(q)
+    ops.accumulate(o_acc, None, False, out)            # fp32 running output -> q's dtype
+    return out, lse_acc
 
 
 def ring_backward(q, k, v, o, do, lse, causal=False, scale=None, group=None, ops=None,
@@ -230,33 +206,29 @@ def ring_backward(q, k, v, o, do, lse, causal=False, scale=None, group=None, ops
     ops = ops or CudaOps()
     scale = _scale(q, scale)
     rank, world, nxt, prv = _peers(group)
-    parts = 2 if zigzag else 1
     q_ids = rank_chunks(rank, world, zigzag)
-    qs, os_, dos = _split(q, parts), _split(o, parts), _split(do, parts)
-    lses = [c.contiguous() for c in torch.chunk(lse, parts, dim=2)]
-    sums = [ops.bwd_begin(("local", i), os_[i], dos[i], lses[i], deterministic)
-            for i in range(parts)]
-    ks, vs = _split(k, parts), _split(v, parts)
-    cur = ks + vs
-    # per K/V chunk: its dK and dV accumulators stacked, (2, B, Hkv, chunk, d) fp32
-    acc = [torch.zeros((2,) + tuple(c.shape), dtype=torch.float32, device=c.device) for c in ks]
+    st = ops.bwd_begin("local", o, do, lse, deterministic)
+    cur = [k.contiguous(), v.contiguous()]
+    # dK and dV accumulators of the chunks held, stacked: (2, B, Hkv, n, d) fp32
+    acc = torch.zeros((2,) + tuple(k.shape), dtype=torch.float32, device=k.device)
     for r in range(world):
         reqs = None
         if r < world - 1:
             nxt_kv, reqs = _exchange(cur, nxt, prv, group)
         kv_ids = rank_chunks((rank - r) % world, world, zigzag)
-        kvs = list(zip(cur[:parts], cur[parts:]))
-        _bwd_hop(ops, sums, qs, q_ids, dos, kvs, kv_ids, acc, causal, scale)
+        _bwd_hop(ops, st, q, do, cur[0], cur[1], acc, q_ids, kv_ids, causal, scale)
         # the dK / dV accumulators travel on with their chunks; after the last hop each rank
         # holds its own chunks'
-        nxt_acc, acc_reqs = _exchange(acc, nxt, prv, group)
+        (nxt_acc,), acc_reqs = _exchange([acc], nxt, prv, group)
         for req in (reqs or []) + acc_reqs:
             req.wait()
         if reqs is not None:
             cur = nxt_kv
         acc = nxt_acc
-    return (_join([ops.bwd_finish(st, torch.empty_like(c), scale) for st, c in zip(sums, qs)]),
-            _convert(ops, [a[0] for a in acc], ks), _convert(ops, [a[1] for a in acc], vs))
+    dk, dv = torch.empty_like(k), torch.empty_like(v)
+    ops.accumulate(acc[0], None, False, dk)
+    ops.accumulate(acc[1], None, False, dv)
+    return ops.bwd_finish(st, torch.empty_like(q), scale), dk, dv
 
 
 class _Lanes:
@@ -305,25 +277,24 @@ def ring_forward_emulated(qs, ks, vs, causal=False, scale=None, ops=None, zigzag
     ops = ops or CudaOps()
     world = len(qs)
     scale = _scale(qs[0], scale)
-    parts = 2 if zigzag else 1
-    q_chunks = [_split(q, parts) for q in qs]
-    kv_chunks = [list(zip(_split(k, parts), _split(v, parts))) for k, v in zip(ks, vs)]
-    states = [[_FwdState(c) for c in qc] for qc in q_chunks]
-    outs = [[torch.empty_like(c) for c in qc] for qc in q_chunks]
+    o_acc = [torch.empty(q.shape, dtype=torch.float32, device=q.device) for q in qs]
+    lse_acc = [torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device) for q in qs]
+    outs = [torch.empty_like(q) for q in qs]
+    kvs = [(k.contiguous(), v.contiguous()) for k, v in zip(ks, vs)]
+    init = [[False] * (2 if zigzag else 1) for _ in range(world)]
     lanes = _Lanes(world, qs[0].device)
     for r in range(world):
         for p in range(world):
             s = (p - r) % world      # the rank whose chunks rank p holds in hop r
             with lanes.rank(p):
-                _fwd_hop(ops, states[p], q_chunks[p], rank_chunks(p, world, zigzag),
-                         kv_chunks[s], rank_chunks(s, world, zigzag), causal, scale, slot=p)
+                _fwd_hop(ops, o_acc[p], lse_acc[p], init[p], qs[p], kvs[s][0], kvs[s][1],
+                         rank_chunks(p, world, zigzag), rank_chunks(s, world, zigzag), causal,
+                         scale, slot=p)
     for p in range(world):
         with lanes.rank(p):
-            for st, out in zip(states[p], outs[p]):
-                ops.accumulate(st.o_acc, None, False, out)
+            ops.accumulate(o_acc[p], None, False, outs[p])
     lanes.join()
-    return ([_join(outs[p]) for p in range(world)],
-            [_join([st.lse for st in states[p]]) for p in range(world)])
+    return outs, lse_acc
 
 
 def ring_backward_emulated(qs, ks, vs, os_, dos, lses, causal=False, scale=None, ops=None,
@@ -334,19 +305,13 @@ def ring_backward_emulated(qs, ks, vs, os_, dos, lses, causal=False, scale=None,
     ops = ops or CudaOps()
     world = len(qs)
     scale = _scale(qs[0], scale)
-    parts = 2 if zigzag else 1
-    q_chunks = [_split(q, parts) for q in qs]
-    o_chunks = [_split(o, parts) for o in os_]
-    do_chunks = [_split(x, parts) for x in dos]
-    l_chunks = [[c.contiguous() for c in torch.chunk(x, parts, dim=2)] for x in lses]
-    kv_chunks = [list(zip(_split(k, parts), _split(v, parts))) for k, v in zip(ks, vs)]
-    sums = [[ops.bwd_begin((p, i), o_chunks[p][i], do_chunks[p][i], l_chunks[p][i],
-                           deterministic) for i in range(parts)] for p in range(world)]
-    dkv_acc = [[torch.zeros((2,) + tuple(k.shape), dtype=torch.float32, device=k.device)
-                for k, _ in kvc] for kvc in kv_chunks]
-    dq_out = [[torch.empty_like(c) for c in qc] for qc in q_chunks]
-    dk_out = [[torch.empty_like(k) for k, _ in kvc] for kvc in kv_chunks]
-    dv_out = [[torch.empty_like(v) for _, v in kvc] for kvc in kv_chunks]
+    kvs = [(k.contiguous(), v.contiguous()) for k, v in zip(ks, vs)]
+    sums = [ops.bwd_begin(p, os_[p], dos[p], lses[p], deterministic) for p in range(world)]
+    dkv_acc = [torch.zeros((2,) + tuple(k.shape), dtype=torch.float32, device=k.device)
+               for k in ks]
+    dq_out = [torch.empty_like(q) for q in qs]
+    dk_out = [torch.empty_like(k) for k in ks]
+    dv_out = [torch.empty_like(v) for v in vs]
     lanes = _Lanes(world, qs[0].device)
     for r in range(world):
         for p in range(world):
@@ -354,18 +319,17 @@ def ring_backward_emulated(qs, ks, vs, os_, dos, lses, causal=False, scale=None,
             with lanes.rank(p):
                 if r > 0:
                     lanes.after_previous(p)
-                _bwd_hop(ops, sums[p], q_chunks[p], rank_chunks(p, world, zigzag), do_chunks[p],
-                         kv_chunks[s], rank_chunks(s, world, zigzag), dkv_acc[s], causal, scale)
+                _bwd_hop(ops, sums[p], qs[p], dos[p], kvs[s][0], kvs[s][1], dkv_acc[s],
+                         rank_chunks(p, world, zigzag), rank_chunks(s, world, zigzag), causal,
+                         scale)
         for p in range(world):
             lanes.hop_done(p)
     # the last addition to rank p's own chunks' sums is rank p - 1's in the last hop
     for p in range(world):
         with lanes.rank(p):
             lanes.after_previous(p)
-            for st, out in zip(sums[p], dq_out[p]):
-                ops.bwd_finish(st, out, scale)
-            for acc, dk, dv in zip(dkv_acc[p], dk_out[p], dv_out[p]):
-                ops.accumulate(acc[0], None, False, dk)
-                ops.accumulate(acc[1], None, False, dv)
+            ops.bwd_finish(sums[p], dq_out[p], scale)
+            ops.accumulate(dkv_acc[p][0], None, False, dk_out[p])
+            ops.accumulate(dkv_acc[p][1], None, False, dv_out[p])
     lanes.join()
-    return ([_join(x) for x in dq_out], [_join(x) for x in dk_out], [_join(x) for x in dv_out])
+    return dq_out, dk_out, dv_out

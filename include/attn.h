@@ -94,11 +94,17 @@ int attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* ls
  * which is exact because each result is normalised by its own exp(LSE) (the rule of
  * attn_ring_merge, without the rounding of O_b to bf16). first != 0: o_acc and lse_acc are not
  * read (they are set to this key set's result). A row that sees no key in any call so far has
- * o_acc = 0, lse_acc = -inf. Errors as attn_fwd_ex; null or misaligned (16-byte) o_acc / lse_acc
- * -> ATTN_ERR_INVALID. */
+ * o_acc = 0, lse_acc = -inf.
+ *   Views of longer sequences: the heads of q, o_acc and lse_acc start q_head_rows rows apart and
+ *   those of k and v kv_head_rows rows apart (0: nq / nk, the packed layouts); so rows
+ *   [r0, r0 + nq) of (B, H, N, d) tensors are passed as the pointers to row r0 with
+ *   q_head_rows = N.
+ * Errors as attn_fwd_ex; null or misaligned (16-byte) o_acc / lse_acc, or head_rows below the
+ * row count -> ATTN_ERR_INVALID. */
 int attn_fwd_accumulate(const void* q, const void* k, const void* v, float* o_acc, float* lse_acc,
-                        int B, int H, int Hkv, int nq, int nk, int d, float scale,
-                        int window_left, int window_right, int first, void* stream);
+                        int B, int H, int Hkv, int nq, int nk, int d, long long q_head_rows,
+                        long long kv_head_rows, float scale, int window_left, int window_right,
+                        int first, void* stream);
 
 /* FP8 forward pass ("Flash Attention Nedir?" and "Apa itu FlashAttention": FlashAttention-3 runs
  * the method in FP8 on Hopper). q, k, v hold E4M3 bytes (OCP FP8 E4M3: 1 sign, 4 exponent bits
@@ -213,6 +219,10 @@ int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
  *   caller's fp32 arrays dk_acc, dv_acc (B, Hkv, nk, d), which the caller zeroes before the first
  *   call. Keys that no query sees add nothing. deterministic != 0: each call adds a query tile's
  *   partials in decreasing key-tile order, so the whole sequence of calls repeats bit for bit.
+ *   Views: the heads of q and dO start q_head_rows rows apart, those of k, v, dk_acc and dv_acc
+ *   kv_head_rows apart (0: nq / nk, packed). The workspace was prepared for ws_rows query rows
+ *   (0: nq) and this call's queries are its rows [q_row0, q_row0 + nq); either they end at
+ *   ws_rows or nq is a multiple of 128 (else ATTN_ERR_INVALID).
  * attn_bwd_finish: writes dq (B, H, nq, d) bf16 = scale · the dQ sum.
  * Errors: null or misaligned (16-byte) pointer, or sizes as attn_bwd_ex -> ATTN_ERR_INVALID; a
  *   workspace that is null or not 256-byte aligned -> ATTN_ERR_INVALID, too small ->
@@ -223,6 +233,7 @@ int attn_bwd_prepare(const void* o, const void* dO, const float* lse, int B, int
                      void* stream);
 int attn_bwd_accumulate(const void* q, const void* k, const void* v, const void* dO,
                         float* dk_acc, float* dv_acc, int B, int H, int Hkv, int nq, int nk, int d,
+                        long long q_head_rows, long long kv_head_rows, int ws_rows, int q_row0,
                         float scale, int window_left, int window_right, int dtype,
                         int deterministic, void* workspace, size_t ws_bytes, void* stream);
 int attn_bwd_finish(void* dq, int B, int H, int nq, int d, float scale, int dtype,

@@ -173,10 +173,11 @@ def test_noalloc_validates_before_touching_the_device():
 def _parts(which, **kw):
     """One of the three backward-part entry points with valid fake arguments, `kw` overriding."""
     a = dict(B=1, H=2, Hkv=1, nq=300, nk=500, d=128, scale=0.1, wl=-1, wr=0,
-             dtype=ea.ATTN_BF16, det=1)
+             dtype=ea.ATTN_BF16, det=1, q_rows=0, kv_rows=0, ws_rows=0, q_row0=0)
     a.update(kw)
-    need = (ea.attn_bwd_workspace_bytes(a["B"], a["H"], a["nq"], a["d"], a["det"])
-            if a["B"] > 0 and a["nq"] > 0 else 0)
+    ws_rows = a["ws_rows"] or a["nq"]
+    need = (ea.attn_bwd_workspace_bytes(a["B"], a["H"], ws_rows, a["d"], a["det"])
+            if a["B"] > 0 and ws_rows > 0 else 0)
     ws = ctypes.c_void_p(kw.get("ws", FAKE))
     ws_bytes = kw.get("ws_bytes", need)
     P = lambda name: ctypes.c_void_p(kw.get(name, FAKE))
@@ -186,6 +187,7 @@ def _parts(which, **kw):
     if which == "accumulate":
         return ea.attn_bwd_accumulate(P("q"), P("k"), P("v"), P("dO"), P("dk_acc"), P("dv_acc"),
                                       a["B"], a["H"], a["Hkv"], a["nq"], a["nk"], a["d"],
+                                      a["q_rows"], a["kv_rows"], a["ws_rows"], a["q_row0"],
                                       a["scale"], a["wl"], a["wr"], a["dtype"], a["det"], ws,
                                       ws_bytes, None)
     return ea.attn_bwd_finish(P("dq"), a["B"], a["H"], a["nq"], a["d"], a["scale"], a["dtype"],
@@ -206,6 +208,11 @@ def _parts(which, **kw):
     ("accumulate", dict(d=48), ea.ATTN_ERR_UNSUPPORTED),
     ("accumulate", dict(ws=0), ea.ATTN_ERR_INVALID),
     ("accumulate", dict(ws_bytes=4096), ea.ATTN_ERR_WORKSPACE),
+    ("accumulate", dict(q_rows=299), ea.ATTN_ERR_INVALID),     # heads closer than nq rows
+    ("accumulate", dict(kv_rows=499), ea.ATTN_ERR_INVALID),
+    ("accumulate", dict(ws_rows=600, q_row0=301), ea.ATTN_ERR_INVALID),   # past the workspace
+    ("accumulate", dict(ws_rows=600, q_row0=0), ea.ATTN_ERR_INVALID),     # ragged, not at the end
+    ("accumulate", dict(q_row0=-1), ea.ATTN_ERR_INVALID),
     ("finish", dict(dq=0), ea.ATTN_ERR_INVALID),
     ("finish", dict(nq=0), ea.ATTN_ERR_INVALID),
     ("finish", dict(det=0, ws_bytes=100), ea.ATTN_ERR_WORKSPACE),
@@ -221,11 +228,13 @@ def test_backward_parts_reject_bad_arguments(which, kw, code):
     (dict(Hkv=3), ea.ATTN_ERR_INVALID),
     (dict(d=96), ea.ATTN_ERR_UNSUPPORTED),
     (dict(scale=0.0), ea.ATTN_ERR_INVALID),
+    (dict(q_rows=100), ea.ATTN_ERR_INVALID),
+    (dict(kv_rows=-5), ea.ATTN_ERR_INVALID),
 ])
 def test_forward_accumulate_rejects_bad_arguments(kw, code):
-    a = dict(B=1, H=2, Hkv=1, nq=300, nk=500, d=128, scale=0.1)
+    a = dict(B=1, H=2, Hkv=1, nq=300, nk=500, d=128, scale=0.1, q_rows=0, kv_rows=0)
     a.update(kw)
     P = lambda name: ctypes.c_void_p(kw.get(name, FAKE))
     assert ea.attn_fwd_accumulate(P("q"), P("k"), P("v"), P("o_acc"), P("lse_acc"), a["B"], a["H"],
-                                  a["Hkv"], a["nq"], a["nk"], a["d"], a["scale"], -1, 0, 1,
-                                  None) == code
+                                  a["Hkv"], a["nq"], a["nk"], a["d"], a["q_rows"], a["kv_rows"],
+                                  a["scale"], -1, 0, 1, None) == code

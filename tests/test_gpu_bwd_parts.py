@@ -84,3 +84,44 @@ def test_parts_match_the_single_call(cuda_device):
     assert torch.equal(dq, rq)
     assert torch.equal(dk.to(torch.bfloat16), rk)
     assert torch.equal(dv.to(torch.bfloat16), rv)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_parts_on_views_of_the_whole_sequence(cuda_device, d):
+    """Query and key row ranges passed as views (no copies): the first 256 queries against each
+    key half, the last 256 against all keys (workspace rows from 256), unmasked; the sums equal
+    the whole gradient, and the folded forward on the same views equals the whole forward."""
+    n = 512
+    q, k, v, do = attn_inputs.random_draws((2, 2, n, d), seed=90 + d, count=4)
+    dev = torch.device("cuda:0")
+    gq, gk, gv, gdo = (x.to(dev) for x in (q, k, v, do))
+    scale = 1.0 / math.sqrt(d)
+    o_acc = torch.empty(gq.shape, dtype=torch.float32, device=dev)
+    lse_acc = torch.empty(gq.shape[:3], dtype=torch.float32, device=dev)
+    h = n // 2
+    plan = [(0, h, 0, h), (0, h, h, n), (h, n, 0, n)]
+    first = {0: True, h: True}
+    for a0, a1, b0, b1 in plan:
+        ea.forward_accumulate(gq[:, :, a0:a1], gk[:, :, b0:b1], gv[:, :, b0:b1],
+                              o_acc[:, :, a0:a1], lse_acc[:, :, a0:a1], first=first[a0],
+                              scale=scale)
+        first[a0] = False
+    torch.cuda.synchronize()
+    ro, rlse = oracle.fwd_ex(q, k, v, scale, -1, -1)
+    assert np.abs(to_np(o_acc) - ro).max() <= 1e-2
+    assert np.abs(to_np(lse_acc) - rlse).max() <= 1e-3
+    o = o_acc.to(torch.bfloat16)
+    for det in (False, True):
+        bs = ea.BackwardSum(o, gdo, lse_acc, deterministic=det)
+        dk = torch.zeros(gk.shape, dtype=torch.float32, device=dev)
+        dv = torch.zeros_like(dk)
+        for a0, a1, b0, b1 in plan:
+            bs.add(gq[:, :, a0:a1], gk[:, :, b0:b1], gv[:, :, b0:b1], gdo[:, :, a0:a1],
+                   dk[:, :, b0:b1], dv[:, :, b0:b1], scale=scale, q_row0=a0)
+        dq = bs.finish(scale=scale)
+        torch.cuda.synchronize()
+        assert ea.device_status() == ea.ATTN_OK
+        rq, rk, rv = oracle.bwd_ex(q, k, v, do, scale, -1, -1)
+        assert grad_close(to_np(dq), rq)
+        assert grad_close(to_np(dk), rk)
+        assert grad_close(to_np(dv), rv)

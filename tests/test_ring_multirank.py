@@ -115,3 +115,35 @@ def test_zigzag_layout_balances_causal_work():
                         pairs += 0 if w is None else (0.5 if w == (-1, 0) else 1.0)
             work.append(pairs)
         assert (len(set(work)) == 1) == balanced, work
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("causal", [True, False])
+def test_hop_launches_cover_the_visible_pairs_once(world, causal):
+    """Each hop's launches, expanded back to (query chunk, key chunk) pairs with the mask each
+    pair gets, must be exactly the visible pairs with their own windows; with zigzag chunks every
+    hop is a single launch."""
+    from exact_attention_138_b200 import ring
+    for zigzag in (False, True):
+        for p in range(world):
+            q_ids = ring.rank_chunks(p, world, zigzag)
+            for r in range(world):
+                kv_ids = ring.rank_chunks((p - r) % world, world, zigzag)
+                launches = ring.hop_launches(q_ids, kv_ids, causal)
+                got = {}
+                for a0, a1, b0, b1, w in launches:
+                    for a in range(a0, a1):
+                        for b in range(b0, b1):
+                            assert (a, b) not in got
+                            if w == (-1, 0) and (a1 - a0) > 1:
+                                # the causal mask of the concatenation, on this pair
+                                qa, kb = q_ids[a], kv_ids[b]
+                                got[(a, b)] = (-1, 0) if qa == kb else ((-1, -1) if kb < qa else None)
+                            else:
+                                got[(a, b)] = w
+                want = {(a, b): ring.hop_window(qa, kb, causal)
+                        for a, qa in enumerate(q_ids) for b, kb in enumerate(kv_ids)}
+                for key, w in want.items():
+                    assert got.get(key) == w, (p, r, key)
+                if zigzag and any(w is not None for w in want.values()):
+                    assert len(launches) == 1
