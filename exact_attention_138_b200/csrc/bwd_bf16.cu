@@ -907,23 +907,24 @@ __global__ void __launch_bounds__(q64::kThreads, 1)
             const int x = it & 1, st = it % STAGES;
             const SDesc bq = shift(Q_mn, st * QTILE);
             const SDesc a_ds = shift(dS_k, x * DS_BYTES), b_ds = shift(dS_mn, x * DS_BYTES);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_ss(tmem + COL_DK, sdesc_at(a_ds, static_cast<uint32_t>((ks * 32) >> 4)),
-                       sdesc_at(bq, static_cast<uint32_t>((ks * 2048) >> 4)), idKV,
-                       (it > 0 || ks > 0) ? 1u : 0u);
+            // dQ^T first: the drain, and through it the next S^T of this parity, waits for it
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
                 mma_ss(tmem + COL_DP + 64 * x, sdesc_at(K_mn, static_cast<uint32_t>((ks * 2048) >> 4)),
                        sdesc_at(b_ds, static_cast<uint32_t>((ks * 2048) >> 4)), idQ, ks > 0 ? 1u : 0u);
             mma_commit(&bars->dq_full[x]);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_ss(tmem + COL_DK, sdesc_at(a_ds, static_cast<uint32_t>((ks * 32) >> 4)),
+                       sdesc_at(bq, static_cast<uint32_t>((ks * 2048) >> 4)), idKV,
+                       (it > 0 || ks > 0) ? 1u : 0u);
             mma_commit(&bars->ds_free[x]);
             mma_commit(&bars->q_empty[st]);
         };
         bool ok = NTT > 0;
         if (warp == 9) {
             // S^T(i), dP^T(i): tile i takes the columns of tile i-2, free once the drain has read
-            // dQ^T(i-2) (which also means dV(i-2), dK(i-2) and dQ^T(i-2) are complete)
+            // dQ^T(i-2) (which also means dV(i-2), the last reader of P^T(i-2), is complete)
             if (ok) ok = bounded_wait_warp(&bars->kv_full, 0, abort, lim);
             for (int it = 0; ok && it < NTT; ++it) {
                 const int x = it & 1;
