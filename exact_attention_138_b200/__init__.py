@@ -249,15 +249,20 @@ def _head_rows(*ts):
     for t in ts:
         if t.dim() == 4:
             B, H, n, d = t.shape
-            ok = t.stride(3) == 1 and t.stride(2) == d and t.stride(1) % d == 0
-            r = t.stride(1) // d if ok else -1
-            ok = ok and (B == 1 or t.stride(0) == H * t.stride(1))
+            e = d                                   # elements per row
+            ok = t.stride(3) == 1 and t.stride(2) == d
         else:
             B, H, n = t.shape
-            r = t.stride(1)
-            ok = t.stride(2) == 1 and (B == 1 or t.stride(0) == H * r)
-        if H == 1 and B == 1:
-            r = n if rows is None else rows
+            e = 1
+            ok = t.stride(2) == 1
+        # rows between heads: from the head stride, or from the batch stride when H == 1 (the
+        # stride of a dimension of size 1 carries no layout)
+        hs = t.stride(1) if H > 1 else (t.stride(0) if B > 1 else None)
+        if hs is None:
+            r = n if rows is None else rows         # a single head: any row count fits
+        else:
+            ok = ok and hs % e == 0 and (B == 1 or H == 1 or t.stride(0) == H * hs)
+            r = hs // e
         if not ok or r < n or (rows is not None and r != rows):
             raise ValueError("expected packed (B, H, n, d) tensors or views of rows of a longer "
                              "sequence with one layout")

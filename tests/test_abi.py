@@ -238,3 +238,18 @@ def test_forward_accumulate_rejects_bad_arguments(kw, code):
     assert ea.attn_fwd_accumulate(P("q"), P("k"), P("v"), P("o_acc"), P("lse_acc"), a["B"], a["H"],
                                   a["Hkv"], a["nq"], a["nk"], a["d"], a["q_rows"], a["kv_rows"],
                                   a["scale"], -1, 0, 1, None) == code
+
+
+def test_head_rows_of_views():
+    """Rows between heads that the binding passes for views of longer sequences (0 = packed)."""
+    import torch
+    x = torch.zeros(2, 4, 100, 64)
+    assert ea._head_rows(x) == 0
+    assert ea._head_rows(x[:, :, 50:]) == 100
+    assert ea._head_rows(x[:, :, :30], torch.zeros(2, 4, 100)[:, :, :30]) == 100
+    assert ea._head_rows(torch.zeros(3, 1, 100, 32)[:, :, 10:20]) == 100    # H = 1: batch stride
+    assert ea._head_rows(torch.zeros(1, 1, 7, 32)) == 0
+    for bad in ((x.transpose(1, 2),), (x[:, :, 50:], x[:, :, :30].contiguous()),
+                (x[..., :32],)):
+        with pytest.raises(ValueError):
+            ea._head_rows(*bad)
