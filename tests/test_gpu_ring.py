@@ -65,17 +65,27 @@ def test_emulated_ring_equals_full_attention(cuda_device, world, causal, H, Hkv,
     assert grad_close(to_np(dv), rv)
 
 
-def test_emulated_ring_deterministic_is_bitwise_repeatable(cuda_device):
+@pytest.mark.parametrize("zigzag", [False, True])
+def test_emulated_ring_deterministic_is_bitwise_repeatable(cuda_device, zigzag):
     world, n_chunk, d = 4, 256, 128
     q, k, v, do = attn_inputs.random_draws((1, 2, world * n_chunk, d), seed=5, count=4)
     dev = torch.device("cuda:0")
-    qs, ks, vs, dos = (_split(x.to(dev), world) for x in (q, k, v, do))
-    os_, lses = ring.ring_forward_emulated(qs, ks, vs, causal=True)
-    first = ring.ring_backward_emulated(qs, ks, vs, os_, dos, lses, causal=True, deterministic=True)
-    again = ring.ring_backward_emulated(qs, ks, vs, os_, dos, lses, causal=True, deterministic=True)
+    qs, ks, vs, dos = (_split(x.to(dev), world, zigzag) for x in (q, k, v, do))
+    os_, lses = ring.ring_forward_emulated(qs, ks, vs, causal=True, zigzag=zigzag)
+    first = ring.ring_backward_emulated(qs, ks, vs, os_, dos, lses, causal=True, deterministic=True,
+                                        zigzag=zigzag)
+    again = ring.ring_backward_emulated(qs, ks, vs, os_, dos, lses, causal=True, deterministic=True,
+                                        zigzag=zigzag)
     for a_list, b_list in zip(first, again):
         for a, b in zip(a_list, b_list):
             assert torch.equal(a, b)
+    # and the deterministic sums are the gradients (against the oracle over the whole sequence)
+    scale = 1.0 / math.sqrt(d)
+    dq, dk, dv = (_unsplit(x, world, zigzag) for x in first)
+    rq, rk, rv = oracle.bwd_ex(q, k, v, do, scale, -1, 0)
+    assert grad_close(to_np(dq), rq)
+    assert grad_close(to_np(dk), rk)
+    assert grad_close(to_np(dv), rv)
 
 
 @pytest.mark.parametrize("d", [32, 64, 128])
