@@ -1,6 +1,6 @@
-"""Forward parity on grids that fill the GPU (more query tiles than the SMs can hold at once),
-where the library runs one query tile per CTA with two CTAs per SM; smaller grids take the
-kernels that split each tile's keys over a cluster, which the other forward tests cover. Whole
+"""Forward parity on grids that fill the GPU (more tile pairs than the SMs hold at once), where
+the library runs one CTA per pair of query tiles with no key split; most of the other forward
+tests have small grids, which take the kernels that split each pair's keys over a cluster. Whole
 tensors against the oracle, element by element, with the masks and head layouts of the pages
 ("Attention Mechanism ...", §4.2, §4.4, §4.5, §12)."""
 import math
