@@ -270,6 +270,42 @@ def _head_rows(*ts):
     return 0 if rows is None or rows == ts[0].shape[2] else rows
 
 
+def _packed(where, *ts):
+    """The entry points without view support take packed CUDA tensors on one device: a host
+    tensor's pointer must never reach a kernel, and a strided one would be read as packed."""
+    dev = None
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError(f"{where}: tensors must be on a CUDA device")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{where}: tensors must be on one device")
+        if not t.is_contiguous():
+            raise ValueError(f"{where}: tensors must be contiguous")
+
+
+def _shaped(where, pairs):
+    """(tensor, expected shape, expected dtype or None) triples: a buffer the kernels write or read
+    must have the size they assume (the C ABI only sees pointers)."""
+    for t, shape, dtype in pairs:
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{where}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+        if dtype is not None and t.dtype != dtype:
+            raise ValueError(f"{where}: expected {dtype}, got {t.dtype}")
+
+
+def _on_device(where, dev, *ts):
+    """Views are allowed (their layout is checked by _head_rows), host tensors are not."""
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError(f"{where}: tensors must be on a CUDA device")
+        if t.device != dev:
+            raise ValueError(f"{where}: tensors must be on one device ({dev})")
+
+
 def _check(rc, where):
     if rc != ATTN_OK:
         raise AttnError(rc, where)
@@ -316,6 +352,9 @@ def forward(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None, 
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, n), dtype=torch.float32, device=q.device)
+    _packed("forward", q, k, v, out, lse)
+    _shaped("forward", [(out, q.shape, q.dtype), (lse, (B, H, n) if q.dim() == 4 else (n,),
+                                                  torch.float32)])
     if nk != n or window is not None:
         wl, wr = _window(causal, window)
         rc = attn_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Hkv, n, nk, d,
@@ -343,6 +382,7 @@ def forward_accumulate(q, k, v, o_acc, lse_acc, first=False, causal=False, scale
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     wl, wr = _window(causal, window)
+    _on_device("forward_accumulate", q.device, q, k, v, o_acc, lse_acc)
     q_rows, kv_rows = _head_rows(q, o_acc, lse_acc), _head_rows(k, v)
     rc = attn_fwd_accumulate(_ptr(q), _ptr(k), _ptr(v), _ptr(o_acc), _ptr(lse_acc), B, H, Hkv, n,
                              nk, d, q_rows, kv_rows, float(scale), wl, wr, int(bool(first)),
@@ -366,6 +406,11 @@ def backward(q, k, v, o, do, lse, causal=False, scale=None, deterministic=False,
     need = attn_bwd_workspace_bytes(B, H, n, d, int(bool(deterministic)))
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _packed("backward", q, k, v, o, do, lse, dq, dk, dv, workspace)
+    lse_shape = (B, H, n) if q.dim() == 4 else (n,)
+    _shaped("backward", [(o, q.shape, q.dtype), (do, q.shape, q.dtype),
+                         (lse, lse_shape, torch.float32), (dq, q.shape, q.dtype),
+                         (dk, k.shape, k.dtype), (dv, v.shape, v.dtype)])
     ws_bytes = workspace.numel() * workspace.element_size()
     if nk != n or window is not None:
         wl, wr = _window(causal, window)
@@ -401,8 +446,11 @@ class BackwardSum:
         self.reset(o, do, lse, stream)
 
     def reset(self, o, do, lse, stream=None):
+        import torch
         if _dims(o) != (self.B, self.H, self.n, self.d):
             raise ValueError("reset needs the sizes the workspace was made for")
+        _packed("BackwardSum", o, do, lse, self.ws)
+        _shaped("BackwardSum", [(do, o.shape, o.dtype), (lse, o.shape[:-1], torch.float32)])
         rc = attn_bwd_prepare(_ptr(o), _ptr(do), _ptr(lse), self.B, self.H, self.n, self.d,
                               _dtype_code(o), self.det, _ptr(self.ws), self.ws.numel(),
                               _stream_handle(stream))
@@ -413,10 +461,16 @@ class BackwardSum:
         """dQ sum += and dk_acc, dv_acc (fp32, k's shape) += the gradients over keys k, v. q, dO
         may be rows [q_row0, q_row0 + nq) of the queries (views of them), k, v, dk_acc, dv_acc
         views of rows of longer key sequences."""
+        import torch
         Hkv, nk = _kv_heads(q, k, v)
         for t in (dk_acc, dv_acc):
-            if t.shape != k.shape or t.dtype.itemsize != 4 or not t.is_floating_point():
+            if t.shape != k.shape or t.dtype != torch.float32:
                 raise ValueError("dk_acc, dv_acc must be fp32 with k's shape")
+        if (q.dim() != 4 or q.shape[0] != self.B or q.shape[1] != self.H or q.shape[3] != self.d
+                or q.shape[2] + int(q_row0) > self.n or int(q_row0) < 0):
+            raise ValueError("q must be (B, H, nq, d) rows of the queries this sum was made for")
+        _shaped("BackwardSum.add", [(do, q.shape, q.dtype)])
+        _on_device("BackwardSum.add", self.ws.device, q, k, v, do, dk_acc, dv_acc)
         if scale is None:
             scale = 1.0 / math.sqrt(self.d)
         wl, wr = _window(causal, window)
@@ -436,6 +490,8 @@ class BackwardSum:
                              device=self.ws.device)
         if scale is None:
             scale = 1.0 / math.sqrt(self.d)
+        _packed("BackwardSum.finish", dq, self.ws)
+        _shaped("BackwardSum.finish", [(dq, (self.B, self.H, self.n, self.d), torch.bfloat16)])
         rc = attn_bwd_finish(_ptr(dq), self.B, self.H, self.n, self.d, float(scale),
                              _dtype_code(dq), self.det, _ptr(self.ws), self.ws.numel(),
                              _stream_handle(stream))
@@ -451,8 +507,14 @@ def device_status(stream=None) -> int:
 def ring_merge(o_acc, lse_acc, o_part, lse_part, first=False, out=None, stream=None):
     """Fold a partial (o_part, lse_part) into the running fp32 (o_acc, lse_acc) in place; with
     `out` also write the merged output there (see attn_ring_merge)."""
+    import torch
     d = o_acc.shape[-1]
     rows = lse_acc.numel()
+    _packed("ring_merge", o_acc, lse_acc, o_part, lse_part, out)
+    _shaped("ring_merge", [(o_acc, tuple(lse_acc.shape) + (d,), torch.float32),
+                           (lse_acc, lse_acc.shape, torch.float32), (o_part, o_acc.shape, None),
+                           (lse_part, lse_acc.shape, torch.float32)]
+            + ([(out, o_acc.shape, None)] if out is not None else []))
     rc = attn_ring_merge(_ptr(o_acc), _ptr(lse_acc), _ptr(o_part), _ptr(lse_part), rows, d,
                          _dtype_code(o_part), int(bool(first)),
                          _ptr(out) if out is not None else None,
@@ -463,6 +525,10 @@ def ring_merge(o_acc, lse_acc, o_part, lse_part, first=False, out=None, stream=N
 
 def ring_accumulate(acc, part=None, first=False, out=None, stream=None):
     """acc (fp32) = (0 if first else acc) + part; with `out` also write the sum there."""
+    import torch
+    _packed("ring_accumulate", acc, part, out)
+    _shaped("ring_accumulate", [(acc, acc.shape, torch.float32)]
+            + [(t, acc.shape, None) for t in (part, out) if t is not None])
     rc = attn_ring_accumulate(_ptr(acc), _ptr(part) if part is not None else None, acc.numel(),
                               _dtype_code(part) if part is not None else ATTN_BF16,
                               int(bool(first)), _ptr(out) if out is not None else None,
@@ -491,6 +557,9 @@ def forward_fp8(q, k, v, q_descale=1.0, k_descale=1.0, v_descale=1.0, causal=Fal
         out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty((B, H, n), dtype=torch.float32, device=q.device)
+    _packed("forward_fp8", q, k, v, out, lse)
+    _shaped("forward_fp8", [(out, q.shape, torch.bfloat16),
+                            (lse, (B, H, n) if q.dim() == 4 else (n,), torch.float32)])
     wl, wr = _window(causal, window)
     rc = attn_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Hkv, n, nk, d,
                       float(scale), wl, wr, float(q_descale), float(k_descale), float(v_descale),

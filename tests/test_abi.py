@@ -253,3 +253,36 @@ def test_head_rows_of_views():
                 (x[..., :32],)):
         with pytest.raises(ValueError):
             ea._head_rows(*bad)
+
+
+def test_bindings_refuse_host_and_strided_tensors():
+    """The binding stops host tensors (a host pointer must never reach a kernel), strided tensors
+    where the entry point takes packed ones, and buffers of the wrong size, before any C call."""
+    import torch
+    q = torch.zeros(1, 2, 64, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        ea.forward(q, q, q)
+    with pytest.raises(ValueError, match="CUDA"):
+        ea.backward(q, q, q, q, q, torch.zeros(1, 2, 64))
+    with pytest.raises(ValueError, match="CUDA"):
+        ea.forward_accumulate(q, q, q, torch.zeros(1, 2, 64, 64), torch.zeros(1, 2, 64))
+    with pytest.raises(ValueError):
+        ea.ring_accumulate(torch.zeros(16), torch.zeros(8))
+    with pytest.raises(ValueError):
+        ea.forward_fp8(q.to(torch.uint8), q.to(torch.uint8), q.to(torch.uint8))
+    # the layout and size checks themselves
+    with pytest.raises(ValueError, match="contiguous"):
+        ea._packed("t", torch.zeros(4, 4).t().cuda() if torch.cuda.is_available() else _FakeCuda())
+    with pytest.raises(ValueError, match="shape"):
+        ea._shaped("t", [(torch.zeros(2, 3), (3, 2), None)])
+    with pytest.raises(ValueError, match="expected torch.float32"):
+        ea._shaped("t", [(torch.zeros(2, 3, dtype=torch.bfloat16), (2, 3), torch.float32)])
+
+
+class _FakeCuda:
+    """A stand-in with the attributes _packed reads: on a CUDA device, not contiguous."""
+    is_cuda = True
+    device = "cuda:0"
+
+    def is_contiguous(self):
+        return False
