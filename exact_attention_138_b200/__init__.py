@@ -459,15 +459,15 @@ class BackwardSum:
     def add(self, q, k, v, do, dk_acc, dv_acc, scale=None, causal=False, window=None,
             stream=None, q_row0=0):
         """dQ sum += and dk_acc, dv_acc (fp32, k's shape) += the gradients over keys k, v. q, dO
-        may be rows [q_row0, q_row0 + nq) of the queries (views of them), k, v, dk_acc, dv_acc
-        views of rows of longer key sequences."""
+        may be rows [q_row0, q_row0 + nq) of the queries (views of them; q_row0 a multiple of
+        64), k, v, dk_acc, dv_acc views of rows of longer key sequences."""
         import torch
         Hkv, nk = _kv_heads(q, k, v)
         for t in (dk_acc, dv_acc):
             if t.shape != k.shape or t.dtype != torch.float32:
                 raise ValueError("dk_acc, dv_acc must be fp32 with k's shape")
         if (q.dim() != 4 or q.shape[0] != self.B or q.shape[1] != self.H or q.shape[3] != self.d
-                or q.shape[2] + int(q_row0) > self.n or int(q_row0) < 0):
+                or q.shape[2] + int(q_row0) > self.n or int(q_row0) < 0 or int(q_row0) % 64):
             raise ValueError("q must be (B, H, nq, d) rows of the queries this sum was made for")
         _shaped("BackwardSum.add", [(do, q.shape, q.dtype)])
         _on_device("BackwardSum.add", self.ws.device, q, k, v, do, dk_acc, dv_acc)

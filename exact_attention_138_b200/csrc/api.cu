@@ -385,9 +385,10 @@ int attn_bwd_accumulate(const void* q, const void* k, const void* v, const void*
     if ((q_head_rows != 0 && q_head_rows < nq) || (kv_head_rows != 0 && kv_head_rows < nk) ||
         q_head_rows < 0 || kv_head_rows < 0 || q_head_rows > kMaxSeq || kv_head_rows > kMaxSeq)
         return ATTN_ERR_INVALID;
-    // the rows after this launch's last query tile are padding of the workspace, or there are none
-    if (ws_rows < 1 || ws_rows > kMaxSeq || q_row0 < 0 || q_row0 > ws_rows - nq ||
-        (q_row0 + nq != ws_rows && nq % 128 != 0))
+    // the first query sits on a 64-row boundary of the workspace (its fp32 rows are moved by bulk
+    // copies), and the rows after this launch's last query tile are padding or there are none
+    if (ws_rows < 1 || ws_rows > kMaxSeq || q_row0 < 0 || q_row0 % 64 != 0 ||
+        q_row0 > ws_rows - nq || (q_row0 + nq != ws_rows && nq % 128 != 0))
         return ATTN_ERR_INVALID;
     WsLayout w;
     if ((rc = check_ws(workspace, ws_bytes, B, H, ws_rows, d, deterministic, &w))) return rc;

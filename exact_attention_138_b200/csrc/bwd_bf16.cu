@@ -510,8 +510,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             float* acc_tile = p.dq_acc + (static_cast<size_t>(qbh) * p.n_pad + i * 128) * D;
             {
-                // lane r = query row; columns = head-dim g*D/2 .. (g+1)*D/2-1
+                // lane r = query row; columns = head-dim g*D/2 .. (g+1)*D/2-1; rows past the
+                // launch's last query add nothing (they may lie outside its workspace rows)
                 const uint32_t tDQ = tmem + lane_base + COL_DQ + b2 * 64 + g * (D / 2);
+                const bool live = i * 128 + r < mk.nq;
                 float* row = acc_tile + r * D + g * (D / 2);
                 if constexpr (D / 2 == 32) {
                     uint32_t u[32];
@@ -519,7 +521,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     tmem_ld_wait();
 #pragma unroll
                     for (int x = 0; x < 8; ++x)
-                        red_add_v4_f32(row + 4 * x, __uint_as_float(u[4 * x]), __uint_as_float(u[4 * x + 1]),
+                        if (live) red_add_v4_f32(row + 4 * x, __uint_as_float(u[4 * x]), __uint_as_float(u[4 * x + 1]),
                                        __uint_as_float(u[4 * x + 2]), __uint_as_float(u[4 * x + 3]));
                 } else {
                     uint32_t u[16];
@@ -527,7 +529,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     tmem_ld_wait();
 #pragma unroll
                     for (int x = 0; x < 4; ++x)
-                        red_add_v4_f32(row + 4 * x, __uint_as_float(u[4 * x]), __uint_as_float(u[4 * x + 1]),
+                        if (live) red_add_v4_f32(row + 4 * x, __uint_as_float(u[4 * x]), __uint_as_float(u[4 * x + 1]),
                                        __uint_as_float(u[4 * x + 2]), __uint_as_float(u[4 * x + 3]));
                 }
             }
@@ -547,11 +549,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             float* sL = sStat + (g * 2 + (it & 1)) * 128;
             float* sD = sL + 64;
             {
-                const size_t qq = static_cast<size_t>(qbh) * p.n_pad + i * 128 + cb + (t & 63);
+                // rows past the launch's last query (a 128-row tile that starts 64 rows into a
+                // workspace block runs into the next head's rows) read as padding: P = dS = 0
+                const int qr = i * 128 + cb + (t & 63);
+                const size_t qq = static_cast<size_t>(qbh) * p.n_pad + qr;
                 if (t < 64)
-                    sL[t] = p.L2vec[qq];
+                    sL[t] = qr < mk.nq ? p.L2vec[qq] : INFINITY;
                 else
-                    sD[t - 64] = p.Dvec[qq];
+                    sD[t - 64] = qr < mk.nq ? p.Dvec[qq] : 0.f;
             }
             wg_bar();
             // ---- P^T = exp2(S^T·scale·log2e - LSE·log2e), masked; bf16 copy into TMEM
@@ -1242,7 +1247,9 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t stream) {
         kp.Dvec = a.Dvec + a.q_row0;
         kp.L2vec = a.L2vec + a.q_row0;
         kp.dq_acc = a.dq_acc + static_cast<size_t>(a.q_row0) * D;
-        kp.sems = a.sems ? a.sems + (a.q_row0 / 64) * 4 : nullptr;
+        // semaphores count one launch's partials (zeroed by the preprocess or just above), so
+        // every launch indexes them from its own first query tile
+        kp.sems = a.sems;
         kp.dk = static_cast<__nv_bfloat16*>(a.dk);
         kp.dv = static_cast<__nv_bfloat16*>(a.dv);
         kp.n_pad = n_pad;

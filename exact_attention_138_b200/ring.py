@@ -14,10 +14,12 @@ key chunk) pair is unmasked (earlier key chunk), causal (same chunk) or skipped 
 chunk). The visible pairs of a hop are joined into as few launches as the masks allow, each on
 row ranges (views) of the rank's whole tensors: with zigzag chunks every hop is one launch (the
 rank's own chunks: the causal mask of their concatenation; an earlier rank's: all queries
-against its first chunk; a later rank's: the second query chunk against both). The backward
-pass walks the same ring with the final O and LSE: dQ accumulates locally (in the fp32 sum of
-the rank's backward workspace), and the fp32 dK / dV accumulators travel with their chunks, are
-added to in place by every hop, and arrive back at their owner after the last hop.
+against its first chunk; a later rank's: the second query chunk against both; the backward's
+launches start their queries on 64-row boundaries, so causal zigzag chunks on GPUs are multiples
+of 64 rows). The backward pass walks the same ring with the final O and LSE: dQ accumulates
+locally (in the fp32 sum of the rank's backward workspace), and the fp32 dK / dV accumulators
+travel with their chunks, are added to in place by every hop, and arrive back at their owner
+after the last hop.
 
 Every arithmetic step runs in the library's CUDA kernels: forward, attn_fwd_accumulate per
 launch (it folds the launch into the running result inside the forward kernel); backward,
@@ -107,6 +109,9 @@ class CudaOps:
 
     def bwd_add(self, st, q, k, v, do, dk_acc, dv_acc, scale, window, q_row0):
         """dQ sum of `st` (its rows from q_row0) and dk_acc, dv_acc += this launch's part."""
+        if q_row0 % 64:
+            raise ValueError("the backward adds query rows from 64-row boundaries: the chunks of "
+                             "a causal zigzag ring must be multiples of 64 rows long")
         st.add(q, k, v, do, dk_acc, dv_acc, scale=scale, window=window, q_row0=q_row0)
 
     def bwd_finish(self, st, out, scale):

@@ -221,8 +221,8 @@ int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
  *   partials in decreasing key-tile order, so the whole sequence of calls repeats bit for bit.
  *   Views: the heads of q and dO start q_head_rows rows apart, those of k, v, dk_acc and dv_acc
  *   kv_head_rows apart (0: nq / nk, packed). The workspace was prepared for ws_rows query rows
- *   (0: nq) and this call's queries are its rows [q_row0, q_row0 + nq); either they end at
- *   ws_rows or nq is a multiple of 128 (else ATTN_ERR_INVALID).
+ *   (0: nq) and this call's queries are its rows [q_row0, q_row0 + nq), q_row0 a multiple of
+ *   64; either they end at ws_rows or nq is a multiple of 128 (else ATTN_ERR_INVALID).
  * attn_bwd_finish: writes dq (B, H, nq, d) bf16 = scale · the dQ sum.
  * Errors: null or misaligned (16-byte) pointer, or sizes as attn_bwd_ex -> ATTN_ERR_INVALID; a
  *   workspace that is null or not 256-byte aligned -> ATTN_ERR_INVALID, too small ->

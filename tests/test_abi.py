@@ -213,6 +213,7 @@ def _parts(which, **kw):
     ("accumulate", dict(ws_rows=600, q_row0=301), ea.ATTN_ERR_INVALID),   # past the workspace
     ("accumulate", dict(ws_rows=600, q_row0=0), ea.ATTN_ERR_INVALID),     # ragged, not at the end
     ("accumulate", dict(q_row0=-1), ea.ATTN_ERR_INVALID),
+    ("accumulate", dict(ws_rows=332, q_row0=32), ea.ATTN_ERR_INVALID),    # off a 64-row boundary
     ("finish", dict(dq=0), ea.ATTN_ERR_INVALID),
     ("finish", dict(nq=0), ea.ATTN_ERR_INVALID),
     ("finish", dict(det=0, ws_bytes=100), ea.ATTN_ERR_WORKSPACE),

@@ -86,13 +86,15 @@ def test_parts_match_the_single_call(cuda_device):
     assert torch.equal(dv.to(torch.bfloat16), rv)
 
 
-@pytest.mark.parametrize("d", [64, 128])
-def test_parts_on_views_of_the_whole_sequence(cuda_device, d):
+@pytest.mark.parametrize("d,H,Hkv", [(32, 2, 2), (64, 2, 2), (128, 2, 2), (128, 4, 2), (64, 4, 1)])
+def test_parts_on_views_of_the_whole_sequence(cuda_device, d, H, Hkv):
     """Query and key row ranges passed as views (no copies): the first 256 queries against each
     key half, the last 256 against all keys (workspace rows from 256), unmasked; the sums equal
-    the whole gradient, and the folded forward on the same views equals the whole forward."""
+    the whole gradient, and the folded forward on the same views equals the whole forward. Also
+    with grouped-query heads (dK, dV summed over each group)."""
     n = 512
-    q, k, v, do = attn_inputs.random_draws((2, 2, n, d), seed=90 + d, count=4)
+    q, do = attn_inputs.random_draws((2, H, n, d), seed=90 + d + H, count=2)
+    k, v = attn_inputs.random_draws((2, Hkv, n, d), seed=91 + d + Hkv, count=2)
     dev = torch.device("cuda:0")
     gq, gk, gv, gdo = (x.to(dev) for x in (q, k, v, do))
     scale = 1.0 / math.sqrt(d)
@@ -125,3 +127,53 @@ def test_parts_on_views_of_the_whole_sequence(cuda_device, d):
         assert grad_close(to_np(dq), rq)
         assert grad_close(to_np(dk), rk)
         assert grad_close(to_np(dv), rv)
+
+
+@pytest.mark.parametrize("d,H,Hkv", [(32, 3, 3), (64, 3, 1), (128, 3, 3)])
+def test_query_block_that_starts_64_rows_in(cuda_device, d, H, Hkv):
+    """Queries [0, 64) see keys [0, 64), queries [64, 256) all 256 keys: one launch of every
+    query against the first 64 keys, one of the last 192 queries (workspace rows from 64, so a
+    128-row query tile reaches 64 rows past the head's workspace rows, into the next head's and,
+    for the last head, past the end) against the other keys. A query block's gradient is that of
+    its own attention, so the oracle takes the two blocks apart and dK, dV are the sums; dQ of
+    every head must be untouched by its neighbour's tiles."""
+    n, m = 256, 64
+    q, do = attn_inputs.random_draws((1, H, n, d), seed=70 + d + H, count=2)
+    k, v = attn_inputs.random_draws((1, Hkv, n, d), seed=71 + d + Hkv, count=2)
+    scale = 1.0 / math.sqrt(d)
+    oa, la = oracle.fwd_ex(q[:, :, :m], k[:, :, :m], v[:, :, :m], scale, -1, -1)
+    ob, lb = oracle.fwd_ex(q[:, :, m:], k, v, scale, -1, -1)
+    dev = torch.device("cuda:0")
+    gq, gk, gv, gdo = (x.to(dev) for x in (q, k, v, do))
+    o = torch.from_numpy(np.concatenate([oa, ob], 2)).to(dev, torch.bfloat16)
+    lse = torch.from_numpy(np.concatenate([la, lb], 2)).to(dev, torch.float32)
+    aq, ak, av = oracle.bwd_ex(q[:, :, :m], k[:, :, :m], v[:, :, :m], do[:, :, :m], scale, -1, -1)
+    bq, bk, bv = oracle.bwd_ex(q[:, :, m:], k, v, do[:, :, m:], scale, -1, -1)
+    rq = np.concatenate([aq, bq], 2)
+    rk, rv = bk.copy(), bv.copy()
+    rk[:, :, :m] += ak
+    rv[:, :, :m] += av
+    for det in (False, True):
+        bs = ea.BackwardSum(o, gdo, lse, deterministic=det)
+        dk = torch.zeros(gk.shape, dtype=torch.float32, device=dev)
+        dv = torch.zeros_like(dk)
+        for a0, b0, b1 in ((0, 0, m), (m, m, n)):
+            bs.add(gq[:, :, a0:], gk[:, :, b0:b1], gv[:, :, b0:b1], gdo[:, :, a0:],
+                   dk[:, :, b0:b1], dv[:, :, b0:b1], scale=scale, q_row0=a0)
+        dq = bs.finish(scale=scale)
+        torch.cuda.synchronize()
+        assert ea.device_status() == ea.ATTN_OK
+        for h in range(H):
+            assert grad_close(to_np(dq[:, h]), rq[:, h])
+        assert grad_close(to_np(dk), rk)
+        assert grad_close(to_np(dv), rv)
+
+
+def test_query_rows_off_a_64_row_boundary_are_refused(cuda_device):
+    q, k, v, do = (x.to("cuda:0") for x in attn_inputs.random_draws((1, 1, 256, 64), seed=3,
+                                                                     count=4))
+    o, lse = ea.forward(q, k, v)
+    bs = ea.BackwardSum(o, do, lse)
+    dk = torch.zeros(k.shape, dtype=torch.float32, device=q.device)
+    with pytest.raises(ValueError):
+        bs.add(q[:, :, 32:], k, v, do[:, :, 32:], dk, torch.zeros_like(dk), q_row0=32)

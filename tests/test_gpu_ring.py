@@ -39,7 +39,8 @@ def _unsplit(parts, world, zigzag=False):
     (3, False, 2, 2, 300, 64, False), (4, True, 4, 2, 200, 64, False),
     (2, False, 2, 1, 512, 32, False), (8, True, 1, 1, 128, 128, False),
     (2, True, 2, 2, 384, 128, True), (4, True, 4, 2, 256, 64, True),
-    (3, False, 2, 2, 300, 128, True), (8, True, 1, 1, 128, 128, True)])
+    (3, False, 2, 2, 300, 128, True), (8, True, 1, 1, 128, 128, True),
+    (2, True, 2, 2, 256, 32, True), (4, True, 4, 1, 128, 64, True)])
 def test_emulated_ring_equals_full_attention(cuda_device, world, causal, H, Hkv, n_chunk, d,
                                              zigzag):
     n = world * n_chunk
