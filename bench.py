@@ -510,6 +510,26 @@ def main():
                                 device_id=dev)
 
     import exact_attention_138_b200 as ea
+    stream = torch.cuda.current_stream()
+
+    # --- the pages' small forward-only cases, per launch with L2 flushed in between. They run
+    # before the long step, whose power draw can leave the SM clock below its maximum for a
+    # while; the clock they saw is recorded beside them.
+    small = None
+    if not args.no_small_cases and world == 1:
+        hbm = load_peaks()[0].get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        fma = fma_peak_tflops(1965.0)
+        with ClockSampler(local) as small_clocks:
+            small = {name: time_forward_case(ea, attn_inputs.WORKLOADS[name], dev, stream,
+                                             args.small_case_launches, args.warmup, hbm, fma)
+                     for name in SMALL_CASES}
+            # the row-tiling case's bf16 inputs quantised to E4M3, through the FP8 forward
+            small["rowtile_e4m3_4096x64"] = time_forward_case(
+                ea, attn_inputs.WORKLOADS["rowtile_bf16_4096x64"], dev, stream,
+                args.small_case_launches, args.warmup, hbm, fma, e4m3=True)
+        small["peaks"] = {"hbm_gbs": hbm, "fp32_fma_tflops": fma,
+                          "fp32_fma_kind": "148 SMs x 128 lanes x 2 FLOP x 1965 MHz"}
+        small["clocks"] = small_clocks.summary()
 
     # --- inputs: each rank draws its own batch (seed 9 + rank), rounded to bf16 on the host
     q_h, k_h, v_h, do_h = attn_inputs.bf16_draws(w.shape, factor=w.factor, seed=rank_seed(rank))
@@ -520,7 +540,6 @@ def main():
     det = bool(args.deterministic)
     ws = torch.empty(ea.attn_bwd_workspace_bytes(w.B, w.H, w.n, w.d, int(det)), dtype=torch.uint8,
                      device=dev)
-    stream = torch.cuda.current_stream()
 
     def step():
         ea.forward(q, k, v, causal=True, scale=w.scale, out=o, lse=lse, stream=stream)
@@ -618,21 +637,6 @@ def main():
     variants = None
     if not args.no_variants and world == 1:
         variants = time_variants(args, w, ea, q, k, v, do, ws, stream, fwd_flops + bwd_flops)
-
-    # --- extra: the pages' small forward-only cases, per launch with L2 flushed in between
-    small = None
-    if not args.no_small_cases and world == 1:
-        hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-        fma = fma_peak_tflops(1965.0)
-        small = {name: time_forward_case(ea, attn_inputs.WORKLOADS[name], dev, stream,
-                                         args.small_case_launches, args.warmup, hbm, fma)
-                 for name in SMALL_CASES}
-        # the row-tiling case's bf16 inputs quantised to E4M3, through the FP8 forward
-        small["rowtile_e4m3_4096x64"] = time_forward_case(
-            ea, attn_inputs.WORKLOADS["rowtile_bf16_4096x64"], dev, stream,
-            args.small_case_launches, args.warmup, hbm, fma, e4m3=True)
-        small["peaks"] = {"hbm_gbs": hbm, "fp32_fma_tflops": fma,
-                          "fp32_fma_kind": "148 SMs x 128 lanes x 2 FLOP x 1965 MHz"}
 
     # --- end to end through the public API with host buffers (pinned), copies inside the timing.
     # Three streams run as a pipeline: while step k computes, step k+1's inputs travel host ->
