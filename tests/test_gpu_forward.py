@@ -105,11 +105,13 @@ def test_gqa_forward_fp32(cuda_device, Hkv):
     assert np.abs(to_np(lse) - rlse).max() <= TOL_LSE["fp32"]
 
 
-# fp32 grids on both sides of the key split. A query tile is 64 rows; when the tiles alone leave
-# the GPU under-filled the kernel splits each tile's key range over a cluster of 2-8 CTAs and
-# merges their (m, l, O) on chip. (2,8,1000,64) and (1,12,1000,128) give 256 and 192 tiles (no
-# split, many key tiles per CTA); (1,1,1000,128) 16 tiles (8 shares, some empty under the causal
-# mask); (2,3,700,32) 66 tiles (4 uneven shares of 11 key tiles).
+# fp32 grids on both sides of the key split. The launcher picks the query-tile height (64 rows
+# down to 32 in steps of 4; 2 threads per row, so heights that are not multiples of 16 leave the
+# CTA's last warp partial) and the key split (1-8 CTAs of a cluster, merging their (m, l, O) on
+# chip) from a cost model over resident CTAs and clusters. With a B200's counts these shapes give
+# 56-row tiles without a split (2,8,1000,64), 60-row tiles in pairs (1,12,1000,128), 64-row tiles
+# in 8 shares, some empty under the causal mask (1,1,1000,128), and 4 uneven shares of 11 key
+# tiles (2,3,700,32).
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("shape", [(2, 8, 1000, 64), (1, 12, 1000, 128), (1, 1, 1000, 128),
                                    (2, 3, 700, 32)], ids=lambda s: "x".join(map(str, s)))
