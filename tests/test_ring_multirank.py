@@ -147,3 +147,13 @@ def test_hop_launches_cover_the_visible_pairs_once(world, causal):
                     assert got.get(key) == w, (p, r, key)
                 if zigzag and any(w is not None for w in want.values()):
                     assert len(launches) == 1
+
+
+def test_gpu_ring_backward_refuses_query_views_off_64_rows():
+    """The library's backward adds a launch's queries from 64-row boundaries of the rank's
+    queries; a causal zigzag ring whose chunk length is not a multiple of 64 is refused with a
+    message before anything is launched (the check needs no GPU)."""
+    from exact_attention_138_b200 import ring
+    ops = ring.CudaOps()
+    with pytest.raises(ValueError, match="64"):
+        ops.bwd_add(None, None, None, None, None, None, None, 1.0, None, 150)
