@@ -1,24 +1,24 @@
 // Forward pass in plain fp32 on the FMA pipes, for the float32 examples of "Efficient Attention"
 // (efficient_attention.py: (2,3,128,32) and the (4096,64) row-tiling case), whose results are
-// compared at an absolute tolerance of 1e-5. TF32 tensor-core products cannot meet that, so
-// every product here is an fp32 FFMA; each exponential is one FFMA (score · scale·log2 e minus the
-// running maximum, rounded once) and the MUFU's 2^x, whose relative error of a few 1e-7 stays
-// far inside that tolerance.
+// compared at an absolute tolerance of 1e-5. TF32 tensor-core products cannot meet that, so every
+// product here is an fp32 fused multiply-add (packed two to an instruction); each exponential is
+// one FMA (score · scale·log2 e minus the running maximum, rounded once) and the MUFU's 2^x,
+// whose relative error of a few 1e-7 stays far inside that tolerance.
 //
 // Same method as the bf16 kernel (tiles of Q/K/V in on-chip memory, online softmax with running
 // max m and sum l, output rescaled by the exponential of the change of m; "Attention Mechanism:
 // Revolusi Representasi Sequence", §13), laid out for SIMT. One CTA works on a tile of BM query
 // rows (BM = 64, or a smaller multiple of 4 down to 32 when that balances a small grid over the
-// SMs) of one (b,h) with 2·BM threads as a (BM/4) x 8 grid (ty, tx). Thread (ty, tx) owns rows ty + i·BM/4
-// (i < 4) and keys tx + 8·jj (jj < 8) of the BM x 64 score tile, and the same rows x columns
-// tx·4 + 32·g + e (e < 4) of the output accumulator. A warp thus covers 16 rows x 64 keys (or
-// 16 rows x all d columns): per 4-wide step of the reduction it reads 4 Q rows and 8 K rows
+// SMs) of one (b,h) with 2·BM threads as a (BM/4) x 8 grid (ty, tx). Thread (ty, tx) owns rows
+// ty + i·BM/4 (i < 4) and keys tx + 8·jj (jj < 8) of the BM x 64 score tile, and the same rows x
+// columns tx·4 + 32·g + e (e < 4) of the output accumulator. A warp thus covers 16 rows x 64 keys
+// (or 16 rows x all d columns): per 4-wide step of the reduction it reads 4 Q rows and 8 K rows
 // (or 4 P rows and 4·d/32 V words) as conflict-free 16-byte words (rows are padded so that
 // consecutive rows start 4 or 8 banks apart), against 128 (or 64·d/32) products, which packed
 // fp32x2 FMAs do two at a time (a 16-byte word is two fp32 pairs), so that instruction issue
-// leaves room for the FMA pipes. The next K/V tile is copied in with cp.async while the current one is
-// used. Scores are kept in the base-2 domain (scale·log2 e folded into one FFMA before ex2),
-// and key tiles that every row of the CTA sees skip the mask.
+// leaves room for the FMA pipes. The next K/V tile is copied in with cp.async while the current
+// one is used. Scores are kept in the base-2 domain (scale·log2 e folded into one FMA before
+// ex2), and key tiles that every row of the CTA sees skip the mask.
 //
 // Small grids (the pages' examples have 12 and 64 query tiles for 148 SMs) split each query
 // tile's key range over a thread-block cluster of up to 8 CTAs. Each CTA keeps its own (m, l, O)
@@ -88,7 +88,7 @@ __device__ __forceinline__ void load_rows(float* dst, int ld, const float* src, 
     }
 }
 
-// Online-softmax step of one thread for one key tile: s (raw scores of rows ty + i·R, keys
+// Online-softmax step of one thread for one key tile: s (raw scores of rows ty + i·BM/4, keys
 // tx + 8·jj) becomes P = 2^(s·sl2 - m) with m the rows' new running maxima (base 2); l and the
 // output accumulator (column pairs) are rescaled. MASK: keys outside a row's [klo, khi] are
 // dropped.
@@ -284,7 +284,8 @@ __global__ void __launch_bounds__(128, F32Cfg<D>::MIN_BLOCKS)
                 ulonglong2 t[NG];    // V row j + jj, this thread's columns as fp32 pairs
 #pragma unroll
                 for (int g = 0; g < NG; ++g)
-                    t[g] = *reinterpret_cast<const ulonglong2*>(Vs + (j + jj) * D + g * 32 + tx * 4);
+                    t[g] = *reinterpret_cast<const ulonglong2*>(Vs + (j + jj) * D + g * 32 +
+                                                                tx * 4);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const float p = jj == 0 ? pv[i].x : jj == 1 ? pv[i].y
@@ -351,7 +352,8 @@ __global__ void __launch_bounds__(128, F32Cfg<D>::MIN_BLOCKS)
         *reinterpret_cast<float4*>(O + base + static_cast<size_t>(qidx) * D + c4 * 4) = o;
         // LSE = ln(2^M · L) = M·ln 2 + ln L (M, the base-2 maximum, is what the weights used)
         if (c4 == 0)
-            lse[static_cast<size_t>(bh) * nq + qidx] = L > 0.f ? fmaf(M, kF32Ln2, logf(L)) : -INFINITY;
+            lse[static_cast<size_t>(bh) * nq + qidx] =
+                L > 0.f ? fmaf(M, kF32Ln2, logf(L)) : -INFINITY;
     }
     if (split > 1) cluster.sync();   // peers may still be reading this CTA's shared memory
 }
